@@ -1,0 +1,297 @@
+"""ctypes binding of ``libspark_bsa.so`` (include/spark_bsa.h).
+
+Argument marshalling only: every step of the forward pass runs in the library's sm_100a
+kernels.  PyTorch provides device memory, the current CUDA stream and dtype/shape checks.
+There is no fallback: if the library is missing or was built for another GPU the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .build import LIB_PATH
+
+__all__ = [
+    "SparkError", "SPARK_BF16", "SPARK_F32", "DEVERR", "Layout", "lib",
+    "spark_status_string", "spark_bsa_topk_count", "spark_bsa_workspace_layout",
+    "spark_bsa_workspace_size", "spark_bsa_forward", "spark_bsa_read_error",
+    "spark_bsa_gather_q", "spark_bsa_anchor", "spark_bsa_gather_kv_summarize",
+    "spark_bsa_route", "spark_bsa_attend", "workspace_views",
+]
+
+SPARK_BF16, SPARK_F32 = 0, 1
+DEVERR = {"perm": 0x1, "offsets": 0x2, "sel": 0x4, "timeout": 0x8}
+EXPORTED = [
+    "spark_status_string", "spark_bsa_topk_count", "spark_bsa_workspace_layout",
+    "spark_bsa_workspace_size", "spark_bsa_forward", "spark_bsa_read_error",
+    "spark_bsa_gather_q", "spark_bsa_anchor", "spark_bsa_gather_kv_summarize",
+    "spark_bsa_route", "spark_bsa_attend",
+]
+
+
+class SparkError(RuntimeError):
+    def __init__(self, fn, status, msg=""):
+        super().__init__(f"{fn} failed: {spark_status_string(status)} ({status}) {msg}".strip())
+        self.status = status
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "Qp", "Kp", "Vp", "qbar_blocks", "qbar", "kbar", "k_tilde", "v_tilde", "cbias", "sel",
+        "err", "total")] + [("k", ctypes.c_int)]
+
+
+_LIB = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_D = ctypes.c_double
+_SZ = ctypes.c_size_t
+
+
+def lib():
+    """Loads the library once; raises if it has not been built."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m block_sparse_attention_gather_b200.build`"
+            " (nvcc, sm_100a). There is no fallback implementation.")
+    L = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "spark_status_string": (ctypes.c_char_p, [_I]),
+        "spark_bsa_topk_count": (_I, [_I, _D]),
+        "spark_bsa_workspace_layout": (_I, [_I, _I, _I, _I, _I, _D, ctypes.POINTER(Layout)]),
+        "spark_bsa_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _D]),
+        "spark_bsa_forward": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _I, _D, _P,
+                                   _P, _SZ, _P]),
+        "spark_bsa_read_error": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
+        "spark_bsa_gather_q": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]),
+        "spark_bsa_anchor": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
+        "spark_bsa_gather_kv_summarize": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P,
+                                               _P, _P, _P, _P, _P, _P]),
+        "spark_bsa_route": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+        "spark_bsa_attend": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _P, _I, _I, _I,
+                                  _I, _P, _I, _P, _P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _LIB = L
+    return L
+
+
+# ---------------------------------------------------------------------------- helpers
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _code(dtype):
+    if dtype == torch.bfloat16:
+        return SPARK_BF16
+    if dtype == torch.float32:
+        return SPARK_F32
+    raise TypeError(f"unsupported dtype {dtype}")
+
+
+def _check(fn, status):
+    if status != 0:
+        raise SparkError(fn, status)
+
+
+# ------------------------------------------------------------------------- host calls
+
+def spark_status_string(status: int) -> str:
+    return lib().spark_status_string(int(status)).decode()
+
+
+def spark_bsa_topk_count(nkb: int, topk_ratio: float) -> int:
+    return int(lib().spark_bsa_topk_count(int(nkb), float(topk_ratio)))
+
+
+def spark_bsa_workspace_layout(H, N, d, nqb, nkb, topk_ratio) -> Layout:
+    L = Layout()
+    _check("spark_bsa_workspace_layout",
+           lib().spark_bsa_workspace_layout(H, N, d, nqb, nkb, float(topk_ratio), ctypes.byref(L)))
+    return L
+
+
+def spark_bsa_workspace_size(H, N, d, nqb, nkb, topk_ratio) -> int:
+    return int(lib().spark_bsa_workspace_size(H, N, d, nqb, nkb, float(topk_ratio)))
+
+
+def workspace_views(workspace: torch.Tensor, layout: Layout, H, N, d, nqb, nkb) -> dict:
+    """Typed views of the intermediates a spark_bsa_forward call left in `workspace`."""
+    def view(off, count, dt):
+        nbytes = count * torch.empty(0, dtype=dt).element_size()
+        return workspace[off:off + nbytes].view(dt)
+    k = layout.k
+    return {
+        "Qp": view(layout.Qp, H * N * d, torch.bfloat16).view(H, N, d),
+        "Kp": view(layout.Kp, H * N * d, torch.bfloat16).view(H, N, d),
+        "Vp": view(layout.Vp, H * N * d, torch.bfloat16).view(H, N, d),
+        "qbar_blocks": view(layout.qbar_blocks, H * nqb * d, torch.float32).view(H, nqb, d),
+        "qbar": view(layout.qbar, H * d, torch.float32).view(H, d),
+        "kbar": view(layout.kbar, H * nkb * d, torch.float32).view(H, nkb, d),
+        "k_tilde": view(layout.k_tilde, H * nkb * d, torch.bfloat16).view(H, nkb, d),
+        "v_tilde": view(layout.v_tilde, H * nkb * d, torch.bfloat16).view(H, nkb, d),
+        "cbias": view(layout.cbias, H * nkb, torch.float32).view(H, nkb),
+        "sel": view(layout.sel, H * nqb * k, torch.int32).view(H, nqb, k),
+        "err": view(layout.err, 1, torch.int32),
+    }
+
+
+# --------------------------------------------------------------------------- device calls
+
+def spark_bsa_forward(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, topk_ratio, out=None,
+                      workspace=None, stream=None):
+    """The whole forward pass on the current CUDA stream; returns (out, workspace, layout)."""
+    _need(Q, "Q", (torch.bfloat16, torch.float32))
+    dev = Q.device
+    for n, t in (("K", K), ("V", V)):
+        _need(t, n, Q.dtype, dev)
+    H, N, d = Q.shape
+    if K.shape != Q.shape or V.shape != Q.shape:
+        raise ValueError("Q, K, V must share the shape [H, N, d]")
+    for n, t in (("q_perm", q_perm), ("k_perm", k_perm)):
+        _need(t, n, torch.int32, dev)
+        if t.shape != (H, N):
+            raise ValueError(f"{n} must have shape [H, N]")
+    for n, t in (("q_offsets", q_offsets), ("k_offsets", k_offsets)):
+        _need(t, n, torch.int32, dev)
+    nqb, nkb = q_offsets.numel() - 1, k_offsets.numel() - 1
+    layout = spark_bsa_workspace_layout(H, N, d, nqb, nkb, topk_ratio)
+    if out is None:
+        out = torch.empty_like(Q)
+    _need(out, "out", Q.dtype, dev)
+    if workspace is None:
+        workspace = torch.empty(layout.total, dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    st = lib().spark_bsa_forward(_ptr(Q), _ptr(K), _ptr(V), _code(Q.dtype), H, N, d,
+                                 _ptr(q_perm), _ptr(k_perm), _ptr(q_offsets), nqb,
+                                 _ptr(k_offsets), nkb, float(topk_ratio), _ptr(out),
+                                 _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("spark_bsa_forward", st)
+    return out, workspace, layout
+
+
+def spark_bsa_read_error(err_word: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream and returns the device error word (0 = no error)."""
+    _need(err_word, "err_word")
+    flags = ctypes.c_uint32(0)
+    st = lib().spark_bsa_read_error(_ptr(err_word), _stream(stream), ctypes.byref(flags))
+    if st not in (0, 5):
+        raise SparkError("spark_bsa_read_error", st)
+    return int(flags.value)
+
+
+def spark_bsa_gather_q(Q, q_perm, q_offsets, Qp=None, qbar_blocks=None, err=None, stream=None):
+    _need(Q, "Q", (torch.bfloat16, torch.float32))
+    H, N, d = Q.shape
+    nqb = q_offsets.numel() - 1
+    Qp = torch.empty(H, N, d, dtype=torch.bfloat16, device=Q.device) if Qp is None else Qp
+    qbar_blocks = (torch.empty(H, nqb, d, dtype=torch.float32, device=Q.device)
+                   if qbar_blocks is None else qbar_blocks)
+    for n, t, dt in (("q_perm", q_perm, torch.int32), ("q_offsets", q_offsets, torch.int32),
+                     ("Qp", Qp, torch.bfloat16), ("qbar_blocks", qbar_blocks, torch.float32)):
+        _need(t, n, dt, Q.device)
+    st = lib().spark_bsa_gather_q(_ptr(Q), _code(Q.dtype), H, N, d, _ptr(q_perm),
+                                  _ptr(q_offsets), nqb, _ptr(Qp), _ptr(qbar_blocks), _ptr(err),
+                                  _stream(stream))
+    _check("spark_bsa_gather_q", st)
+    return Qp, qbar_blocks
+
+
+def spark_bsa_anchor(qbar_blocks, q_offsets, N, qbar=None, stream=None):
+    _need(qbar_blocks, "qbar_blocks", torch.float32)
+    H, nqb, d = qbar_blocks.shape
+    qbar = torch.empty(H, d, dtype=torch.float32, device=qbar_blocks.device) if qbar is None else qbar
+    _need(q_offsets, "q_offsets", torch.int32, qbar_blocks.device)
+    _need(qbar, "qbar", torch.float32, qbar_blocks.device)
+    st = lib().spark_bsa_anchor(_ptr(qbar_blocks), _ptr(q_offsets), H, N, d, nqb, _ptr(qbar),
+                                _stream(stream))
+    _check("spark_bsa_anchor", st)
+    return qbar
+
+
+def spark_bsa_gather_kv_summarize(K, V, k_perm, k_offsets, qbar, err=None, stream=None):
+    _need(K, "K", (torch.bfloat16, torch.float32))
+    _need(V, "V", K.dtype, K.device)
+    H, N, d = K.shape
+    nkb = k_offsets.numel() - 1
+    dev = K.device
+    _need(k_perm, "k_perm", torch.int32, dev)
+    _need(k_offsets, "k_offsets", torch.int32, dev)
+    _need(qbar, "qbar", torch.float32, dev)
+    Kp = torch.empty(H, N, d, dtype=torch.bfloat16, device=dev)
+    Vp = torch.empty_like(Kp)
+    kbar = torch.empty(H, nkb, d, dtype=torch.float32, device=dev)
+    k_tilde = torch.empty(H, nkb, d, dtype=torch.bfloat16, device=dev)
+    v_tilde = torch.empty_like(k_tilde)
+    cbias = torch.empty(H, nkb, dtype=torch.float32, device=dev)
+    st = lib().spark_bsa_gather_kv_summarize(
+        _ptr(K), _ptr(V), _code(K.dtype), H, N, d, _ptr(k_perm), _ptr(k_offsets), nkb,
+        _ptr(qbar), _ptr(Kp), _ptr(Vp), _ptr(kbar), _ptr(k_tilde), _ptr(v_tilde), _ptr(cbias),
+        _ptr(err), _stream(stream))
+    _check("spark_bsa_gather_kv_summarize", st)
+    return Kp, Vp, kbar, k_tilde, v_tilde, cbias
+
+
+def spark_bsa_route(qbar_blocks, kbar, k, err=None, stream=None):
+    _need(qbar_blocks, "qbar_blocks", torch.float32)
+    _need(kbar, "kbar", torch.float32, qbar_blocks.device)
+    H, nqb, d = qbar_blocks.shape
+    nkb = kbar.shape[1]
+    sel = torch.empty(H, nqb, k, dtype=torch.int32, device=qbar_blocks.device)
+    st = lib().spark_bsa_route(_ptr(qbar_blocks), _ptr(kbar), H, nqb, nkb, d, int(k), _ptr(sel),
+                               _ptr(err), _stream(stream))
+    _check("spark_bsa_route", st)
+    return sel
+
+
+def spark_bsa_attend(Qp, Kp, Vp, k_tilde, v_tilde, cbias, sel, q_perm, q_offsets, k_offsets,
+                     out_dtype=torch.bfloat16, out=None, err=None, stream=None):
+    _need(Qp, "Qp", torch.bfloat16)
+    dev = Qp.device
+    H, N, d = Qp.shape
+    for n, t, dt in (("Kp", Kp, torch.bfloat16), ("Vp", Vp, torch.bfloat16),
+                     ("k_tilde", k_tilde, torch.bfloat16), ("v_tilde", v_tilde, torch.bfloat16),
+                     ("cbias", cbias, torch.float32), ("sel", sel, torch.int32),
+                     ("q_perm", q_perm, torch.int32), ("q_offsets", q_offsets, torch.int32),
+                     ("k_offsets", k_offsets, torch.int32)):
+        _need(t, n, dt, dev)
+    nqb, nkb = q_offsets.numel() - 1, k_offsets.numel() - 1
+    k = sel.shape[-1]
+    if out is None:
+        out = torch.empty(H, N, d, dtype=out_dtype, device=dev)
+    _need(out, "out", out_dtype, dev)
+    st = lib().spark_bsa_attend(_ptr(Qp), _ptr(Kp), _ptr(Vp), _ptr(k_tilde), _ptr(v_tilde),
+                                _ptr(cbias), _ptr(sel), k, _ptr(q_perm), _ptr(q_offsets), nqb,
+                                _ptr(k_offsets), nkb, H, N, d, _ptr(out), _code(out_dtype),
+                                _ptr(err), _stream(stream))
+    _check("spark_bsa_attend", st)
+    return out

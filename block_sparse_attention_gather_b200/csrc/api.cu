@@ -1,0 +1,270 @@
+// C ABI of the library (include/spark_bsa.h): argument checks, workspace layout, TMA
+// descriptor encoding and the launch sequence of the forward pass.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "../../include/spark_bsa.h"
+#include "spark_kernels.cuh"
+
+using namespace spark;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+int topk_count(int nkb, double ratio) {
+  if (nkb < 1 || !(ratio > 0.0) || !(ratio <= 1.0)) return -1;
+  double kk = std::ceil(ratio * static_cast<double>(nkb) - 1e-9);
+  int k = static_cast<int>(kk);
+  if (k < 1) k = 1;
+  if (k > nkb) k = nkb;
+  return k;
+}
+
+spark_status check_sizes(int H, int N, int d, int nqb, int nkb) {
+  if (H < 1 || N < 1 || nqb < 1 || nkb < 1 || nqb > N || nkb > N) return SPARK_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SPARK_ERR_UNSUPPORTED;
+  if (H > 65535 || nkb > kMaxNkb) return SPARK_ERR_UNSUPPORTED;
+  return SPARK_OK;
+}
+
+spark_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// 3-D bf16 tensor [H][rows][d] with a 128-row x 64-column box and 128-byte swizzle.
+bool encode_rows_map(CUtensorMap* m, const void* base, int H, int rows, int d) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(H)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+spark_status layout_of(int H, int N, int d, int nqb, int nkb, double ratio,
+                       spark_bsa_layout* L) {
+  spark_status st = check_sizes(H, N, d, nqb, nkb);
+  if (st != SPARK_OK) return st;
+  const int k = topk_count(nkb, ratio);
+  if (k < 0) return SPARK_ERR_INVALID_ARG;
+  const size_t hnd = static_cast<size_t>(H) * N * d;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  L->Qp = take(hnd * 2);
+  L->Kp = take(hnd * 2);
+  L->Vp = take(hnd * 2);
+  L->qbar_blocks = take(static_cast<size_t>(H) * nqb * d * 4);
+  L->qbar = take(static_cast<size_t>(H) * d * 4);
+  L->kbar = take(static_cast<size_t>(H) * nkb * d * 4);
+  L->k_tilde = take(static_cast<size_t>(H) * nkb * d * 2);
+  L->v_tilde = take(static_cast<size_t>(H) * nkb * d * 2);
+  L->cbias = take(static_cast<size_t>(H) * nkb * 4);
+  L->sel = take(static_cast<size_t>(H) * nqb * k * 4);
+  L->err = take(4);
+  L->total = off;
+  L->k = k;
+  return SPARK_OK;
+}
+
+spark_status attend_impl(const void* Qp, const void* Kp, const void* Vp, const void* k_tilde,
+                         const void* v_tilde, const float* cbias, const int32_t* sel, int k,
+                         const int32_t* q_perm, const int32_t* q_offsets, int nqb,
+                         const int32_t* k_offsets, int nkb, int H, int N, int d, void* out,
+                         int out_dtype, uint32_t* err, cudaStream_t s) {
+  AttendMaps maps;
+  if (!encode_rows_map(&maps.k, Kp, H, N, d) || !encode_rows_map(&maps.v, Vp, H, N, d) ||
+      !encode_rows_map(&maps.kt, k_tilde, H, nkb, d) ||
+      !encode_rows_map(&maps.vt, v_tilde, H, nkb, d))
+    return SPARK_ERR_CUDA;
+  maps.q_base = Qp;
+  return from_cuda(launch_attend(maps, cbias, sel, k, q_perm, q_offsets, nqb, k_offsets, nkb, H,
+                                 N, d, out, out_dtype, err, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* spark_status_string(int status) {
+  switch (status) {
+    case SPARK_OK: return "SPARK_OK";
+    case SPARK_ERR_INVALID_ARG: return "SPARK_ERR_INVALID_ARG";
+    case SPARK_ERR_UNSUPPORTED: return "SPARK_ERR_UNSUPPORTED";
+    case SPARK_ERR_WORKSPACE: return "SPARK_ERR_WORKSPACE";
+    case SPARK_ERR_CUDA: return "SPARK_ERR_CUDA";
+    case SPARK_ERR_DEVICE_CHECK: return "SPARK_ERR_DEVICE_CHECK";
+    default: return "SPARK_UNKNOWN_STATUS";
+  }
+}
+
+int spark_bsa_topk_count(int nkb, double topk_ratio) { return topk_count(nkb, topk_ratio); }
+
+spark_status spark_bsa_workspace_layout(int H, int N, int d, int nqb, int nkb,
+                                        double topk_ratio, spark_bsa_layout* layout) {
+  if (layout == nullptr) return SPARK_ERR_INVALID_ARG;
+  return layout_of(H, N, d, nqb, nkb, topk_ratio, layout);
+}
+
+size_t spark_bsa_workspace_size(int H, int N, int d, int nqb, int nkb, double topk_ratio) {
+  spark_bsa_layout L;
+  return layout_of(H, N, d, nqb, nkb, topk_ratio, &L) == SPARK_OK ? L.total : 0;
+}
+
+spark_status spark_bsa_read_error(const uint32_t* err_word, void* stream, uint32_t* flags) {
+  if (err_word == nullptr || flags == nullptr) return SPARK_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, err_word, sizeof(v), cudaMemcpyDeviceToHost,
+                                  as_stream(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return SPARK_ERR_CUDA;
+  *flags = v;
+  return v == 0 ? SPARK_OK : SPARK_ERR_DEVICE_CHECK;
+}
+
+spark_status spark_bsa_gather_q(const void* Q, int dtype, int H, int N, int d,
+                                const int32_t* q_perm, const int32_t* q_block_offsets, int nqb,
+                                void* Qp, float* qbar_blocks, uint32_t* err, void* stream) {
+  if (!Q || !q_perm || !q_block_offsets || !Qp || !qbar_blocks) return SPARK_ERR_INVALID_ARG;
+  if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  spark_status st = check_sizes(H, N, d, nqb, 1);
+  if (st != SPARK_OK) return st;
+  if (!aligned(Q, 16) || !aligned(Qp, 16)) return SPARK_ERR_INVALID_ARG;
+  return from_cuda(launch_gather_q(Q, dtype, H, N, d, q_perm, q_block_offsets, nqb, Qp,
+                                   qbar_blocks, err, as_stream(stream)));
+}
+
+spark_status spark_bsa_anchor(const float* qbar_blocks, const int32_t* q_block_offsets, int H,
+                              int N, int d, int nqb, float* qbar, void* stream) {
+  if (!qbar_blocks || !q_block_offsets || !qbar) return SPARK_ERR_INVALID_ARG;
+  spark_status st = check_sizes(H, N, d, nqb, 1);
+  if (st != SPARK_OK) return st;
+  return from_cuda(launch_anchor(qbar_blocks, q_block_offsets, H, N, d, nqb, qbar,
+                                 as_stream(stream)));
+}
+
+spark_status spark_bsa_gather_kv_summarize(const void* K, const void* V, int dtype, int H,
+                                           int N, int d, const int32_t* k_perm,
+                                           const int32_t* k_block_offsets, int nkb,
+                                           const float* qbar, void* Kp, void* Vp, float* kbar,
+                                           void* k_tilde, void* v_tilde, float* cbias,
+                                           uint32_t* err, void* stream) {
+  if (!K || !V || !k_perm || !k_block_offsets || !qbar || !Kp || !Vp || !kbar || !k_tilde ||
+      !v_tilde || !cbias)
+    return SPARK_ERR_INVALID_ARG;
+  if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  spark_status st = check_sizes(H, N, d, 1, nkb);
+  if (st != SPARK_OK) return st;
+  if (!aligned(K, 16) || !aligned(V, 16) || !aligned(Kp, 16) || !aligned(Vp, 16))
+    return SPARK_ERR_INVALID_ARG;
+  return from_cuda(launch_gather_kv_summary(K, V, dtype, H, N, d, k_perm, k_block_offsets, nkb,
+                                            qbar, Kp, Vp, kbar, k_tilde, v_tilde, cbias, err,
+                                            as_stream(stream)));
+}
+
+spark_status spark_bsa_route(const float* qbar_blocks, const float* kbar, int H, int nqb,
+                             int nkb, int d, int k, int32_t* sel, uint32_t* err, void* stream) {
+  if (!qbar_blocks || !kbar || !sel) return SPARK_ERR_INVALID_ARG;
+  if (H < 1 || nqb < 1 || nkb < 1 || k < 1 || k > nkb) return SPARK_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SPARK_ERR_UNSUPPORTED;
+  if (H > 65535 || nkb > kMaxNkb) return SPARK_ERR_UNSUPPORTED;
+  return from_cuda(launch_route(qbar_blocks, kbar, H, nqb, nkb, d, k, sel, err,
+                                as_stream(stream)));
+}
+
+spark_status spark_bsa_attend(const void* Qp, const void* Kp, const void* Vp,
+                              const void* k_tilde, const void* v_tilde, const float* cbias,
+                              const int32_t* sel, int k, const int32_t* q_perm,
+                              const int32_t* q_block_offsets, int nqb,
+                              const int32_t* k_block_offsets, int nkb, int H, int N, int d,
+                              void* out, int out_dtype, uint32_t* err, void* stream) {
+  if (!Qp || !Kp || !Vp || !k_tilde || !v_tilde || !cbias || !sel || !q_perm ||
+      !q_block_offsets || !k_block_offsets || !out)
+    return SPARK_ERR_INVALID_ARG;
+  if (out_dtype != SPARK_BF16 && out_dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  spark_status st = check_sizes(H, N, d, nqb, nkb);
+  if (st != SPARK_OK) return st;
+  if (k < 1 || k > nkb) return SPARK_ERR_INVALID_ARG;
+  if (!aligned(Qp, 16) || !aligned(Kp, 16) || !aligned(Vp, 16) || !aligned(k_tilde, 16) ||
+      !aligned(v_tilde, 16) || !aligned(out, 16))
+    return SPARK_ERR_INVALID_ARG;
+  return attend_impl(Qp, Kp, Vp, k_tilde, v_tilde, cbias, sel, k, q_perm, q_block_offsets, nqb,
+                     k_block_offsets, nkb, H, N, d, out, out_dtype, err, as_stream(stream));
+}
+
+spark_status spark_bsa_forward(const void* Q, const void* K, const void* V, int dtype, int H,
+                               int N, int d, const int32_t* q_perm, const int32_t* k_perm,
+                               const int32_t* q_block_offsets, int nqb,
+                               const int32_t* k_block_offsets, int nkb, double topk_ratio,
+                               void* out, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (!Q || !K || !V || !q_perm || !k_perm || !q_block_offsets || !k_block_offsets || !out)
+    return SPARK_ERR_INVALID_ARG;
+  if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  spark_bsa_layout L;
+  spark_status st = layout_of(H, N, d, nqb, nkb, topk_ratio, &L);
+  if (st != SPARK_OK) return st;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16))
+    return SPARK_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < L.total || !aligned(workspace, kAlign))
+    return SPARK_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* Qp = ws + L.Qp;
+  void* Kp = ws + L.Kp;
+  void* Vp = ws + L.Vp;
+  float* qbar_blocks = reinterpret_cast<float*>(ws + L.qbar_blocks);
+  float* qbar = reinterpret_cast<float*>(ws + L.qbar);
+  float* kbar = reinterpret_cast<float*>(ws + L.kbar);
+  void* kt = ws + L.k_tilde;
+  void* vt = ws + L.v_tilde;
+  float* cbias = reinterpret_cast<float*>(ws + L.cbias);
+  int32_t* sel = reinterpret_cast<int32_t*>(ws + L.sel);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.err);
+
+  if (cudaMemsetAsync(err, 0, sizeof(uint32_t), s) != cudaSuccess) return SPARK_ERR_CUDA;
+  if (launch_gather_q(Q, dtype, H, N, d, q_perm, q_block_offsets, nqb, Qp, qbar_blocks, err, s) !=
+      cudaSuccess)
+    return SPARK_ERR_CUDA;
+  if (launch_anchor(qbar_blocks, q_block_offsets, H, N, d, nqb, qbar, s) != cudaSuccess)
+    return SPARK_ERR_CUDA;
+  if (launch_gather_kv_summary(K, V, dtype, H, N, d, k_perm, k_block_offsets, nkb, qbar, Kp, Vp,
+                               kbar, kt, vt, cbias, err, s) != cudaSuccess)
+    return SPARK_ERR_CUDA;
+  if (launch_route(qbar_blocks, kbar, H, nqb, nkb, d, L.k, sel, err, s) != cudaSuccess)
+    return SPARK_ERR_CUDA;
+  return attend_impl(Qp, Kp, Vp, kt, vt, cbias, sel, L.k, q_perm, q_block_offsets, nqb,
+                     k_block_offsets, nkb, H, N, d, out, dtype, err, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,413 @@
+// Two-branch block-sparse attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Spark-H3 blog, "Spark-Reblock", BSA equations: for query block A the keys are the exact
+// rows of every selected key block plus one summary row per unselected block (section
+// "Spark-Reweight": weighted summary k~_B, v~_B with logit offset c_B = b_B + log|B|), and
+// a single row-wise softmax normalises both branches.
+//
+// One CTA per (query block A, head h); 7 warps with fixed roles:
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  Loads its Q row into TMEM,
+//              then per key tile reads the S row from TMEM, applies the scale, the column
+//              mask / summary offsets, and an online softmax with lazy rescaling (the running
+//              max used for the exponentials only moves when a tile's max exceeds it by more
+//              than 8 in log2 units, and only then is the O row in TMEM rescaled); writes P
+//              (bf16) into TMEM; finally normalises O and scatters the rows to
+//              out[h, q_perm[h, i], :].
+//   warp 4     TMA producer of K tiles (3-stage ring).
+//   warp 5     TMA producer of V tiles (3-stage ring).
+//   warp 6     MMA issuer (one thread): S = Q K^T with Q read from TMEM, O += P V with P read
+//              from TMEM; S is double-buffered in TMEM so S(t+2) overlaps softmax(t+1).
+//
+// Tile list of a CTA: the k selected blocks in ascending order (a 128-row TMA box starting at
+// the block's first row; rows past the block are masked), then ceil(nkb/128) tiles of the
+// summary rows (rows past nkb are zero-filled by TMA and masked, selected blocks masked).
+//
+// TMEM columns (512 allocated, one CTA per SM): Q [0,D/2), P [64,128), S0 [128,256),
+// S1 [256,384), O [384,384+D).
+//
+// Every wait is bounded (spark_ptx.cuh); on expiry the kernel flags kErrTimeout, stops every
+// role, drains the copies and MMAs it issued, frees TMEM and returns.
+#include "spark_kernels.cuh"
+
+namespace spark {
+
+namespace {
+
+constexpr int kStages = 3;
+constexpr int kThreads = 224;
+constexpr uint32_t kColQ = 0, kColP = 64, kColS0 = 128, kColS1 = 256, kColO = 384;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+struct __align__(8) Barriers {
+  uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages];
+  uint64_t qready, sfull[2], pready, pvdone, drain;
+};
+
+__device__ __forceinline__ bool wait_bounded_ignore_abort(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_test(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
+// Row range of key tile t and how many of its 128 rows are valid.
+struct TileInfo {
+  int y;          // first row (in Kp/Vp for exact tiles, in k~/v~ for summary tiles)
+  int nvalid;     // exact tiles: block size (rows >= nvalid are masked)
+  bool exact;
+};
+
+__device__ __forceinline__ TileInfo tile_info(int t, int k, const int32_t* sel_row,
+                                              const int32_t* k_offsets, int nkb, int N) {
+  TileInfo ti;
+  if (t < k) {
+    int B = sel_row[t];
+    B = min(max(B, 0), nkb - 1);
+    const int lo = min(max(k_offsets[B], 0), N - 1);
+    const int hi = min(max(k_offsets[B + 1], lo), N);
+    ti.y = lo;
+    ti.nvalid = min(hi - lo, kMaxBlock);
+    ti.exact = true;
+  } else {
+    ti.y = (t - k) * 128;
+    ti.nvalid = 128;
+    ti.exact = false;
+  }
+  return ti;
+}
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attend_kernel(
+    const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+    const __grid_constant__ CUtensorMap map_kt, const __grid_constant__ CUtensorMap map_vt,
+    const __nv_bfloat16* __restrict__ Qp, const float* __restrict__ cbias,
+    const int32_t* __restrict__ sel, int k, const int32_t* __restrict__ q_perm,
+    const int32_t* __restrict__ q_offsets, int nqb, const int32_t* __restrict__ k_offsets,
+    int nkb, int N, void* __restrict__ out, int out_dtype, uint32_t* err) {
+  constexpr int TILE_BYTES = 128 * D * 2;        // one K or V tile (bf16)
+  constexpr int NATOM = D / 64;                  // 128-byte swizzle atoms across d
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* kst = smem;
+  uint8_t* vst = smem + kStages * TILE_BYTES;
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + 2 * kStages * TILE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* selmask = reinterpret_cast<uint32_t*>(tmem_slot + 4);
+
+  const int A = blockIdx.x, h = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  __shared__ int s_skip;
+  if (tid == 0) s_skip = launch_timed_out(err) ? 1 : 0;   // an earlier CTA gave up
+  __syncthreads();
+  if (s_skip) return;                                      // uniform: no work, nothing held
+  const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
+  const int T = k + nct;
+  const int32_t* sel_row = sel + (static_cast<size_t>(h) * nqb + A) * k;
+  const int nwords = (nkb + 31) / 32;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->kfull[s], 1);
+      mbar_init(&bars->kempty[s], 1);
+      mbar_init(&bars->vfull[s], 1);
+      mbar_init(&bars->vempty[s], 1);
+    }
+    mbar_init(&bars->qready, 128);
+    mbar_init(&bars->sfull[0], 1);
+    mbar_init(&bars->sfull[1], 1);
+    mbar_init(&bars->pready, 128);
+    mbar_init(&bars->pvdone, 1);
+    mbar_init(&bars->drain, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  for (int i = tid; i < nwords; i += kThreads) selmask[i] = 0u;
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  for (int i = tid; i < k; i += kThreads) {
+    const int B = sel_row[i];
+    if (B >= 0 && B < nkb) atomicOr(&selmask[B >> 5], 1u << (B & 31));
+    else flag_error(err, kErrSel);
+  }
+  __syncthreads();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 4 || warp == 5) {
+    // ------------------------------------------------------------- TMA producers
+    if (lane == 0) {
+      const bool is_k = (warp == 4);
+      uint8_t* ring = is_k ? kst : vst;
+      uint64_t* full = is_k ? bars->kfull : bars->vfull;
+      uint64_t* empty = is_k ? bars->kempty : bars->vempty;
+      const CUtensorMap* mx = is_k ? &map_k : &map_v;
+      const CUtensorMap* ms = is_k ? &map_kt : &map_vt;
+      tma_prefetch_desc(mx);
+      tma_prefetch_desc(ms);
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int s = t % kStages;
+        if (t >= kStages && !mbar_wait(&empty[s], ((t / kStages) - 1) & 1, abort_flag, err)) break;
+        const TileInfo ti = tile_info(t, k, sel_row, k_offsets, nkb, N);
+        mbar_arrive_expect_tx(&full[s], TILE_BYTES);
+        for (int a = 0; a < NATOM; ++a)
+          tma_load_3d(ring + s * TILE_BYTES + a * 16384, ti.exact ? mx : ms, &full[s], a * 64,
+                      ti.y, h);
+        issued = t + 1;
+      }
+      if (*abort_flag) {
+        // drain: wait for every load still in flight (the last round of each stage)
+        for (int t = max(0, issued - kStages); t < issued; ++t)
+          wait_bounded_ignore_abort(&full[t % kStages], (t / kStages) & 1);
+      }
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idO = idesc_bf16(128, D, false, true);
+      bool ok = mbar_wait(&bars->qready, 0, abort_flag, err);
+      tc_fence_after_sync();
+      auto issue_s = [&](int t) -> bool {
+        const int s = t % kStages;
+        if (!mbar_wait(&bars->kfull[s], (t / kStages) & 1, abort_flag, err)) return false;
+        tc_fence_after_sync();
+        const uint32_t dcol = tbase + ((t & 1) ? kColS1 : kColS0);
+        const uint32_t kaddr = smem_u32(kst + s * TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t bdesc = sdesc_sw128(kaddr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          mma_ts(dcol, tbase + kColQ + kk * 8, bdesc, idS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bars->sfull[t & 1]);
+        tc_commit(&bars->kempty[s]);
+        return true;
+      };
+      if (ok && T > 0) ok = issue_s(0);
+      if (ok && T > 1) ok = issue_s(1);
+      for (int t = 0; ok && t < T; ++t) {
+        if (!mbar_wait(&bars->pready, t & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after_sync();
+        const int s = t % kStages;
+        if (!mbar_wait(&bars->vfull[s], (t / kStages) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after_sync();
+        const uint32_t vaddr = smem_u32(vst + s * TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bdesc = sdesc_sw128(vaddr + kk * 2048, 16384, 1024);
+          mma_ts(tbase + kColO, tbase + kColP + kk * 8, bdesc, idO, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&bars->pvdone);
+        tc_commit(&bars->vempty[s]);
+        if (t + 2 < T) ok = issue_s(t + 2);
+      }
+      // make sure nothing this thread issued is still running before TMEM is freed
+      tc_commit(&bars->drain);
+      wait_bounded_ignore_abort(&bars->drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax rows
+    const int row = tid;                                  // 0..127 == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int qlo = q_offsets[A];
+    const int qhi = q_offsets[A + 1];
+    const int qsize = max(0, min(qhi - qlo, kMaxBlock));
+    // Q row -> TMEM (rows past the block read the next rows; they are never stored)
+    {
+      const int qrow = min(max(qlo, 0), N - 1) + row;
+      const bool in = qrow < N;
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(
+          Qp + (static_cast<size_t>(h) * N + (in ? qrow : 0)) * D);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const uint4 v = in ? *reinterpret_cast<const uint4*>(src + c * 32 + j) : make_uint4(0, 0, 0, 0);
+          r[j] = v.x; r[j + 1] = v.y; r[j + 2] = v.z; r[j + 3] = v.w;
+        }
+        tmem_st32(tbase + lane_off + kColQ + c * 32, r);
+      }
+    }
+    tc_fence_before_sync();
+    mbar_arrive(&bars->qready);
+
+    const float scale_log2 = kLog2e * rsqrtf(static_cast<float>(D));
+    const float* cb = cbias + static_cast<size_t>(h) * nkb;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      ok = mbar_wait(&bars->sfull[t & 1], (t >> 1) & 1, abort_flag, err);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }   // collectives below
+      tc_fence_after_sync();
+      const TileInfo ti = tile_info(t, k, sel_row, k_offsets, nkb, N);
+      const uint32_t scol = tbase + lane_off + ((t & 1) ? kColS1 : kColS0);
+      float x[128];
+      {
+        uint32_t r[64];
+        tmem_ld64(scol, r);
+#pragma unroll
+        for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(r[j]);
+        tmem_ld64(scol + 64, r);
+#pragma unroll
+        for (int j = 0; j < 64; ++j) x[64 + j] = __uint_as_float(r[j]);
+      }
+      float mt = -INFINITY;
+      if (ti.exact) {
+#pragma unroll
+        for (int j = 0; j < 128; ++j) {
+          x[j] = (j < ti.nvalid) ? x[j] * scale_log2 : -INFINITY;
+          mt = fmaxf(mt, x[j]);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 128; ++j) {
+          const int B = ti.y + j;
+          const bool live = B < nkb && !((selmask[B >> 5] >> (B & 31)) & 1u);
+          x[j] = live ? fmaf(x[j], scale_log2, cb[B] * kLog2e) : -INFINITY;
+          mt = fmaxf(mt, x[j]);
+        }
+      }
+      bool need = false;
+      float m_new = m_run;
+      if (t == 0) {
+        m_new = mt;
+      } else if (mt > m_run + kRescaleThreshold) {
+        need = true;
+        m_new = mt;
+      }
+      float rowsum = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        const float p0 = ex2_approx(x[2 * j] - m_new);
+        const float p1 = ex2_approx(x[2 * j + 1] - m_new);
+        rowsum += p0 + p1;
+        pk[j] = pack_bf16(p0, p1);
+      }
+      // P and O of the previous tile are in use until its PV MMA completes
+      if (t > 0) {
+        ok = mbar_wait(&bars->pvdone, (t - 1) & 1, abort_flag, err);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after_sync();
+      }
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
+        l_run *= alpha;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tbase + lane_off + kColO + c * 32, r);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+          tmem_st32(tbase + lane_off + kColO + c * 32, r);
+        }
+      }
+      l_run += rowsum;
+      m_run = m_new;
+      {
+        uint32_t r[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = pk[j];
+        tmem_st32(tbase + lane_off + kColP, r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = pk[32 + j];
+        tmem_st32(tbase + lane_off + kColP + 32, r);
+      }
+      tc_fence_before_sync();
+      mbar_arrive(&bars->pready);
+    }
+    // ---- epilogue: O / l scattered to the original token order
+    bool fine = ok && T > 0;
+    if (fine) fine = mbar_wait(&bars->pvdone, (T - 1) & 1, abort_flag, err);
+    if (__all_sync(0xffffffffu, fine)) {
+      tc_fence_after_sync();
+      const float inv = 1.f / l_run;
+      int tok = -1;
+      if (row < qsize) {
+        tok = q_perm[static_cast<size_t>(h) * N + qlo + row];
+        if (tok < 0 || tok >= N) {
+          flag_error(err, kErrPerm);
+          tok = -1;
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tbase + lane_off + kColO + c * 32, r);
+        if (tok >= 0) {
+          const size_t o = (static_cast<size_t>(h) * N + tok) * D + c * 32;
+          if (out_dtype == 0) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + o);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 v;
+              v.x = pack_bf16(__uint_as_float(r[8 * j + 0]) * inv, __uint_as_float(r[8 * j + 1]) * inv);
+              v.y = pack_bf16(__uint_as_float(r[8 * j + 2]) * inv, __uint_as_float(r[8 * j + 3]) * inv);
+              v.z = pack_bf16(__uint_as_float(r[8 * j + 4]) * inv, __uint_as_float(r[8 * j + 5]) * inv);
+              v.w = pack_bf16(__uint_as_float(r[8 * j + 6]) * inv, __uint_as_float(r[8 * j + 7]) * inv);
+              dst[j] = v;
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + o);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(__uint_as_float(r[4 * j]) * inv, __uint_as_float(r[4 * j + 1]) * inv,
+                                   __uint_as_float(r[4 * j + 2]) * inv, __uint_as_float(r[4 * j + 3]) * inv);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+static size_t attend_smem_bytes(int d, int nkb) {
+  const size_t tile = static_cast<size_t>(128) * d * 2;
+  return 1024 + 2 * kStages * tile + sizeof(Barriers) + 16 + ((nkb + 31) / 32) * 4 + 16;
+}
+
+template <int D>
+static cudaError_t launch_attend_t(const AttendMaps& m, const float* cbias, const int32_t* sel,
+                                   int k, const int32_t* q_perm, const int32_t* q_offsets,
+                                   int nqb, const int32_t* k_offsets, int nkb, int H, int N,
+                                   void* out, int out_dtype, uint32_t* err, cudaStream_t s) {
+  const size_t smem = attend_smem_bytes(D, nkb);
+  cudaError_t e = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(nqb, H);
+  attend_kernel<D><<<grid, kThreads, smem, s>>>(m.k, m.v, m.kt, m.vt,
+                                                 static_cast<const __nv_bfloat16*>(m.q_base),
+                                                 cbias, sel, k, q_perm, q_offsets, nqb, k_offsets,
+                                                 nkb, N, out, out_dtype, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attend(const AttendMaps& maps, const float* cbias, const int32_t* sel, int k,
+                          const int32_t* q_perm, const int32_t* q_offsets, int nqb,
+                          const int32_t* k_offsets, int nkb, int H, int N, int d, void* out,
+                          int out_dtype, uint32_t* err, cudaStream_t s) {
+  if (d == 128)
+    return launch_attend_t<128>(maps, cbias, sel, k, q_perm, q_offsets, nqb, k_offsets, nkb, H,
+                                N, out, out_dtype, err, s);
+  return launch_attend_t<64>(maps, cbias, sel, k, q_perm, q_offsets, nqb, k_offsets, nkb, H, N,
+                             out, out_dtype, err, s);
+}
+
+}  // namespace spark

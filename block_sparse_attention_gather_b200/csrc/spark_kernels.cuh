@@ -1,0 +1,40 @@
+// Kernel launchers shared by the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include "spark_ptx.cuh"
+
+namespace spark {
+
+constexpr int kMaxBlock = 128;     // tokens per block (one MMA tile of keys / queries)
+constexpr int kMaxNkb = 12800;     // key blocks per head accepted by the routing kernel
+
+cudaError_t launch_gather_q(const void* Q, int dtype, int H, int N, int d,
+                            const int32_t* q_perm, const int32_t* q_offsets, int nqb, void* Qp,
+                            float* qbar_blocks, uint32_t* err, cudaStream_t s);
+
+cudaError_t launch_anchor(const float* qbar_blocks, const int32_t* q_offsets, int H, int N,
+                          int d, int nqb, float* qbar, cudaStream_t s);
+
+cudaError_t launch_gather_kv_summary(const void* K, const void* V, int dtype, int H, int N,
+                                     int d, const int32_t* k_perm, const int32_t* k_offsets,
+                                     int nkb, const float* qbar, void* Kp, void* Vp,
+                                     float* kbar, void* k_tilde, void* v_tilde, float* cbias,
+                                     uint32_t* err, cudaStream_t s);
+
+cudaError_t launch_route(const float* qbar_blocks, const float* kbar, int H, int nqb, int nkb,
+                         int d, int k, int32_t* sel, uint32_t* err, cudaStream_t s);
+
+// Operands of the attention kernel: TMA descriptors (encoded on the host by api.cu) of the
+// reblocked K, V ([H,N,d] bf16) and of the summaries k~, v~ ([H,nkb,d] bf16), and the
+// reblocked queries, which the kernel reads with plain loads.
+struct AttendMaps {
+  CUtensorMap k, v, kt, vt;
+  const void* q_base;
+};
+
+cudaError_t launch_attend(const AttendMaps& maps, const float* cbias, const int32_t* sel, int k,
+                          const int32_t* q_perm, const int32_t* q_offsets, int nqb,
+                          const int32_t* k_offsets, int nkb, int H, int N, int d, void* out,
+                          int out_dtype, uint32_t* err, cudaStream_t s);
+
+}  // namespace spark

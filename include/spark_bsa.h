@@ -1,0 +1,181 @@
+/*
+ * spark_bsa.h - C ABI of the B200 (sm_100a) two-branch block-sparse attention forward.
+ *
+ * The operation is the Spark-Attn forward described in the blog "Spark-H3: Adaptive Block
+ * Sparse Attention for MiniMax-H3":
+ *
+ *   - section "Spark-Reblock": tokens are permuted into blocks (token ids track membership)
+ *     and, per query block A,  BSA(Q_A) = Softmax(Q_A K~_A^T / sqrt(d)) V~_A,  where K~_A,
+ *     V~_A hold the exact rows of every selected key block B in S_A and one summary per
+ *     unselected block; a single row-wise softmax covers both branches; S_A is a fixed
+ *     Top-K budget ("top 10%" of key blocks);
+ *   - section "Discussion": blocks are scored from block-level means;
+ *   - section "Spark-Reweight": each key block is scored once with a representative query
+ *     (the mean of the head's queries); the scores give weighted key/value summaries and a
+ *     log-mass bias so that exp(effective logit) equals E[exp(q.k)] instead of exp(E[q.k]).
+ *
+ * Definitions used by every entry point (sigma = 1/sqrt(d)):
+ *   Qp[h,i] = Q[h, q_perm[h,i]],  Kp[h,j] = K[h, k_perm[h,j]],  Vp[h,j] = V[h, k_perm[h,j]]
+ *   qbar[h]       = mean over all N queries of head h                    (the anchor)
+ *   qbar_A[h,A]   = mean of Qp rows of query block A;  kbar[h,B] = mean of Kp rows of block B
+ *   s_j           = sigma * qbar . Kp_j;  w = softmax of s over the rows j of block B
+ *   k~_B = sum_j w_j Kp_j,  v~_B = sum_j w_j Vp_j
+ *   c_B  = log(mean_j exp s_j) - sigma * qbar . k~_B + log|B|   (bias b plus log|B|)
+ *   S[h,A,B]      = sigma * qbar_A . kbar_B;  sel[h,A,:] = the k largest (ties: smaller B),
+ *                   stored ascending,  k = clamp(ceil(topk_ratio*nkb - 1e-9), 1, nkb)
+ *   out[h, q_perm[h,i]] = softmax over { sigma q_i.k_j : j in selected blocks } union
+ *                         { sigma q_i.k~_B + c_B : B unselected } applied to {v_j} U {v~_B}
+ *
+ * Conventions:
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise; every buffer is
+ *     owned by the caller; the library allocates nothing and keeps no state between calls
+ *     (a per-process cache of the driver entry point used to encode TMA descriptors aside).
+ *   - Tensors are contiguous, row-major: Q/K/V/out [H,N,d]; perms [H,N] int32 (row i of the
+ *     reblocked layout holds original token perm[i]; one permutation per head); block
+ *     offsets [nb+1] int32, shared by all heads, 0 = off[0] < off[1] < ... < off[nb] = N,
+ *     every block 1..128 tokens.  q_perm == k_perm with equal offsets is legal (the pages'
+ *     reblock_layout=q_reuse_k).
+ *   - d must be 64 or 128.  bf16 inputs give bf16 out; fp32 inputs are rounded to bf16
+ *     (round-to-nearest-even) on entry and give fp32 out.  Internally: bf16 tensor-core
+ *     operands, fp32 accumulation, fp32 softmax, fp32 means, summaries' bias and scores.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are asynchronous
+ *     on that stream; no entry point synchronises except spark_bsa_read_error.
+ *   - Host-checkable problems return a status before anything is launched.  Problems only
+ *     visible in device data (a permutation entry outside [0,N), bad offsets, a selected
+ *     id outside [0,nkb)) never cause out-of-bounds accesses: the kernels skip the access
+ *     and set bits in the device error word, which spark_bsa_read_error returns.
+ */
+#ifndef SPARK_BSA_H_
+#define SPARK_BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPARK_API __attribute__((visibility("default")))
+#else
+#define SPARK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SPARK_OK = 0,
+  SPARK_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, ratio outside (0,1] ... */
+  SPARK_ERR_UNSUPPORTED = 2,   /* d not in {64,128}, a size beyond the library's limits   */
+  SPARK_ERR_WORKSPACE = 3,     /* workspace too small or misaligned                       */
+  SPARK_ERR_CUDA = 4,          /* a CUDA runtime/driver call or a launch failed           */
+  SPARK_ERR_DEVICE_CHECK = 5   /* the device error word is non-zero                       */
+} spark_status;
+
+typedef enum { SPARK_BF16 = 0, SPARK_F32 = 1 } spark_dtype;
+
+/* Bits of the device error word. */
+#define SPARK_DEVERR_PERM 0x1u     /* a permutation entry outside [0, N)                      */
+#define SPARK_DEVERR_OFFSETS 0x2u  /* a block outside [1,128] tokens or offsets not 0..N     */
+#define SPARK_DEVERR_SEL 0x4u      /* a selected block id outside [0, nkb)                    */
+#define SPARK_DEVERR_TIMEOUT 0x8u  /* a bounded in-kernel wait expired (kernel bug)          */
+
+/* Library limits (SPARK_ERR_UNSUPPORTED beyond them). */
+#define SPARK_MAX_BLOCK 128        /* tokens per block                                        */
+#define SPARK_MAX_NKB 12800        /* key blocks per head                                     */
+
+/* Human-readable name of a status code; never NULL. */
+SPARK_API const char* spark_status_string(int status);
+
+/* k = clamp(ceil(topk_ratio * nkb - 1e-9), 1, nkb) - the blog's "top ratio" budget with
+ * a guard against binary rounding of the ratio.  Returns -1 if nkb < 1 or the ratio is
+ * outside (0, 1]. */
+SPARK_API int spark_bsa_topk_count(int nkb, double topk_ratio);
+
+/* Byte offsets of the intermediates inside a spark_bsa_forward workspace.  Each offset is
+ * 256-byte aligned; `total` is the workspace size in bytes. */
+typedef struct {
+  size_t Qp, Kp, Vp;          /* bf16 [H,N,d] reblocked Q, K, V                          */
+  size_t qbar_blocks;         /* fp32 [H,nqb,d] query-block means                        */
+  size_t qbar;                /* fp32 [H,d] per-head anchor                              */
+  size_t kbar;                /* fp32 [H,nkb,d] key-block means                          */
+  size_t k_tilde, v_tilde;    /* bf16 [H,nkb,d] weighted summaries                       */
+  size_t cbias;               /* fp32 [H,nkb] summary offsets c_B = b_B + log|B|        */
+  size_t sel;                 /* int32 [H,nqb,k] selected key blocks, ascending          */
+  size_t err;                 /* uint32 device error word                                */
+  size_t total;
+  int k;                      /* the Top-K count                                         */
+} spark_bsa_layout;
+
+/* Fills *layout for the given sizes.  Pure host arithmetic. */
+SPARK_API spark_status spark_bsa_workspace_layout(int H, int N, int d, int nqb, int nkb,
+                                        double topk_ratio, spark_bsa_layout* layout);
+
+/* Workspace bytes spark_bsa_forward needs (0 if the arguments are invalid). */
+SPARK_API size_t spark_bsa_workspace_size(int H, int N, int d, int nqb, int nkb, double topk_ratio);
+
+/* The whole forward pass: gather + query-block means, anchor, key/value gather fused with
+ * the key-block means and Spark-Reweight summaries, block scoring + Top-K, and the
+ * two-branch tcgen05 attention.  `workspace` (device, 256-byte aligned, at least
+ * spark_bsa_workspace_size bytes) receives the intermediates at the offsets of
+ * spark_bsa_workspace_layout, so callers may inspect them after the call; its error word is
+ * cleared by the call.  `out` is [H,N,d] of `dtype`, in the ORIGINAL token order. */
+SPARK_API spark_status spark_bsa_forward(const void* Q, const void* K, const void* V, int dtype, int H,
+                               int N, int d, const int32_t* q_perm, const int32_t* k_perm,
+                               const int32_t* q_block_offsets, int nqb,
+                               const int32_t* k_block_offsets, int nkb, double topk_ratio,
+                               void* out, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Synchronises `stream`, then copies the device error word at `err_word` (device pointer,
+ * e.g. workspace + layout.err) into *flags (host).  Returns SPARK_ERR_DEVICE_CHECK when it
+ * is non-zero. */
+SPARK_API spark_status spark_bsa_read_error(const uint32_t* err_word, void* stream, uint32_t* flags);
+
+/* ---- The steps of the forward pass, one kernel each, on caller buffers. ----
+ * `err` is a device uint32 error word (may be NULL: bad device data is then skipped
+ * silently).  Bits are OR-ed in; the word is never cleared by these calls. */
+
+/* Step 1 (queries; blog "Spark-Reblock" token permutation, "Discussion" block means):
+ * Qp[h,i,:] = bf16(Q[h,q_perm[h,i],:]);  qbar_blocks[h,A,:] = mean of block A's Qp rows. */
+SPARK_API spark_status spark_bsa_gather_q(const void* Q, int dtype, int H, int N, int d,
+                                const int32_t* q_perm, const int32_t* q_block_offsets, int nqb,
+                                void* Qp, float* qbar_blocks, uint32_t* err, void* stream);
+
+/* Step 2 (blog "Spark-Reweight": the representative query; one anchor per head):
+ * qbar[h,:] = (sum_A |A| * qbar_blocks[h,A,:]) / N. */
+SPARK_API spark_status spark_bsa_anchor(const float* qbar_blocks, const int32_t* q_block_offsets, int H,
+                              int N, int d, int nqb, float* qbar, void* stream);
+
+/* Steps 1+3 fused (keys/values; blog "Spark-Reweight" weighted summaries and log-mass bias):
+ * Kp, Vp (bf16 [H,N,d]) gathered by k_perm; kbar (fp32 [H,nkb,d]) block means;
+ * k_tilde, v_tilde (bf16 [H,nkb,d]) and cbias (fp32 [H,nkb]) as defined above, with
+ * c_B computed against the bf16-rounded k~_B that the attention step consumes. */
+SPARK_API spark_status spark_bsa_gather_kv_summarize(const void* K, const void* V, int dtype, int H,
+                                           int N, int d, const int32_t* k_perm,
+                                           const int32_t* k_block_offsets, int nkb,
+                                           const float* qbar, void* Kp, void* Vp, float* kbar,
+                                           void* k_tilde, void* v_tilde, float* cbias,
+                                           uint32_t* err, void* stream);
+
+/* Step 4 (blog "Discussion": block-mean scoring; "Spark-Reblock": fixed Top-K budget):
+ * fp32 scores sigma*qbar_A.kbar_B, the k largest per (h,A) with ties to the smaller B,
+ * written ascending to sel [H,nqb,k].  1 <= k <= nkb <= SPARK_MAX_NKB. */
+SPARK_API spark_status spark_bsa_route(const float* qbar_blocks, const float* kbar, int H, int nqb,
+                             int nkb, int d, int k, int32_t* sel, uint32_t* err, void* stream);
+
+/* Step 5 (blog "Spark-Reblock" BSA equations with the Spark-Reweight summaries): the
+ * two-branch attention of every (h, A), one online softmax over the exact rows of the
+ * selected blocks and the summary rows (logit sigma q.k~_B + c_B) of the others, written to
+ * out[h, q_perm[h,i], :] (out dtype `out_dtype`).  Qp/Kp/Vp/k_tilde/v_tilde are bf16 and
+ * must be 16-byte aligned; sel [H,nqb,k] ascending, distinct. */
+SPARK_API spark_status spark_bsa_attend(const void* Qp, const void* Kp, const void* Vp,
+                              const void* k_tilde, const void* v_tilde, const float* cbias,
+                              const int32_t* sel, int k, const int32_t* q_perm,
+                              const int32_t* q_block_offsets, int nqb,
+                              const int32_t* k_block_offsets, int nkb, int H, int N, int d,
+                              void* out, int out_dtype, uint32_t* err, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARK_BSA_H_ */
