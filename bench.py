@@ -1,0 +1,472 @@
+#!/usr/bin/env python
+"""Benchmark of the two-branch block-sparse attention forward on B200.
+
+Workload: the 768p video-latent shape (H=24 heads, N=241920 tokens = 60 x 48 x 84, d=128,
+bf16), mixture-structured Q/K with a reblock-like layout, 128-token blocks, topk_ratio 0.1.
+Metric: ms per call and dense-equivalent TFLOP/s (4*H*N^2*d per call), with the roofline of
+the dominant kernel (the tcgen05 attention) against the measured bf16 tensor peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path: query gather + block means, anchor, key/value
+gather fused with the summaries, block scoring + Top-K, two-branch attention - five kernel
+launches through the C ABI on one stream, inputs resident in HBM (4.5 GB, larger than L2).
+With --gpus N > 1 (launched by torchrun) every rank runs an independent replica on its own
+GPU: the path has no exchange step (weak scaling, no collective on the data path).
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/call and dense-equiv TFLOP/s at 10% density, 768p shape; % tensor/HBM roofline"
+UNIT = "dense-equiv TFLOP/s"
+DEFAULT_WORKLOAD = "768p-24x241920-d128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attention_768p_dram.json")
+KERNELS = ["gather_q", "anchor", "gather_kv_summary", "route", "attend"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.out = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        mx = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[0] > 0.3 * mx] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[2])
+                          if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------ the hot path
+
+class HotPath:
+    """Preallocated buffers and the five step entry points of the C ABI, called with raw
+    device pointers on one stream."""
+
+    def __init__(self, x, ratio, device):
+        from block_sparse_attention_gather_b200 import (lib, spark_bsa_workspace_layout,
+                                                        workspace_views)
+        self.L = lib()
+        self.x = x
+        Q = x["Q"]
+        self.H, self.N, self.d = Q.shape
+        self.nqb = x["q_offsets"].numel() - 1
+        self.nkb = x["k_offsets"].numel() - 1
+        self.ratio = ratio
+        self.layout = spark_bsa_workspace_layout(self.H, self.N, self.d, self.nqb, self.nkb, ratio)
+        self.k = self.layout.k
+        self.ws = torch.empty(self.layout.total, dtype=torch.uint8, device=device)
+        self.v = workspace_views(self.ws, self.layout, self.H, self.N, self.d, self.nqb, self.nkb)
+        self.out = torch.empty_like(Q)
+        self.dtype_code = 0 if Q.dtype == torch.bfloat16 else 1
+        self.stream = torch.cuda.current_stream(device)
+
+    def _p(self, t):
+        return ctypes.c_void_p(t.data_ptr())
+
+    def step(self, events=None):
+        """One pass of the whole path; if `events` (6 CUDA events) is given, records one
+        before each kernel and one after the last."""
+        L, x, v, p = self.L, self.x, self.v, self._p
+        s = ctypes.c_void_p(self.stream.cuda_stream)
+        H, N, d, nqb, nkb, k = self.H, self.N, self.d, self.nqb, self.nkb, self.k
+        err = p(v["err"])
+        rec = (lambda i: events[i].record(self.stream)) if events else (lambda i: None)
+        rec(0)
+        st = L.spark_bsa_gather_q(p(x["Q"]), self.dtype_code, H, N, d, p(x["q_perm"]),
+                                  p(x["q_offsets"]), nqb, p(v["Qp"]), p(v["qbar_blocks"]), err, s)
+        rec(1)
+        st |= L.spark_bsa_anchor(p(v["qbar_blocks"]), p(x["q_offsets"]), H, N, d, nqb,
+                                 p(v["qbar"]), s)
+        rec(2)
+        st |= L.spark_bsa_gather_kv_summarize(p(x["K"]), p(x["V"]), self.dtype_code, H, N, d,
+                                              p(x["k_perm"]), p(x["k_offsets"]), nkb,
+                                              p(v["qbar"]), p(v["Kp"]), p(v["Vp"]), p(v["kbar"]),
+                                              p(v["k_tilde"]), p(v["v_tilde"]), p(v["cbias"]),
+                                              err, s)
+        rec(3)
+        st |= L.spark_bsa_route(p(v["qbar_blocks"]), p(v["kbar"]), H, nqb, nkb, d, k,
+                                p(v["sel"]), err, s)
+        rec(4)
+        st |= L.spark_bsa_attend(p(v["Qp"]), p(v["Kp"]), p(v["Vp"]), p(v["k_tilde"]),
+                                 p(v["v_tilde"]), p(v["cbias"]), p(v["sel"]), k,
+                                 p(x["q_perm"]), p(x["q_offsets"]), nqb, p(x["k_offsets"]), nkb,
+                                 H, N, d, p(self.out), self.dtype_code, err, s)
+        rec(5)
+        if st != 0:
+            raise RuntimeError(f"a step entry point failed (status bits {st})")
+
+
+def attention_flops(hp):
+    """Algorithmic tensor-core FLOPs of one attention launch, from the selection it used:
+    4 d sum_{h,A} |A| (sum_{B in S_A} |B| + (nkb - k))."""
+    qo = hp.x["q_offsets"].long()
+    ko = hp.x["k_offsets"].long()
+    qs = (qo[1:] - qo[:-1]).double()                    # [nqb]
+    ks = (ko[1:] - ko[:-1]).double()                    # [nkb]
+    sel = hp.v["sel"].long()                            # [H,nqb,k]
+    exact = ks[sel].sum(-1)                             # [H,nqb]
+    cols = exact + (hp.nkb - hp.k)
+    return float(4.0 * hp.d * (cols * qs[None, :]).sum().item())
+
+
+def kernel_bytes(hp):
+    """Algorithmic HBM bytes per launch of the four bandwidth-bound kernels."""
+    H, N, d, nqb, nkb, k = hp.H, hp.N, hp.d, hp.nqb, hp.nkb, hp.k
+    e = hp.x["Q"].element_size()
+    return {
+        "gather_q": H * N * d * (e + 2) + H * N * 4 + H * nqb * d * 4,
+        "anchor": H * nqb * d * 4 + H * d * 4,
+        "gather_kv_summary": 2 * H * N * d * (e + 2) + H * N * 4 + H * nkb * d * (4 + 2 + 2) + H * nkb * 4,
+        "route": H * (nqb + nkb) * d * 4 + H * nqb * k * 4,
+    }
+
+
+def file_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(hp):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    try:
+        with open(PROFILE_SUMMARY) as f:
+            prof = json.load(f)
+    except (OSError, ValueError):
+        return None
+    src = os.path.join(ROOT, "block_sparse_attention_gather_b200", "csrc", "attention.cu")
+    if prof.get("attention_cu_sha256_16") != file_hash(src):
+        return None
+    per_unit = prof.get("dram_bytes_per_query_block")
+    if per_unit is None:
+        return None
+    return per_unit * hp.H * hp.nqb
+
+
+# ----------------------------------------------------------------------- CPU oracle leg
+
+def oracle_sample(w, n_heads=1, n_units=16, seed=0):
+    """Times the float64 oracle on a bounded sample of workload `w`: the full summaries and
+    routing of `n_heads` heads plus the attention of `n_units` query blocks; returns the
+    extrapolated seconds of one full call and a description."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from block_sparse_attention_gather_b200.workloads import make_inputs
+    from dataclasses import replace
+    from oracle import spark_oracle as O
+
+    ws = replace(w, H=n_heads)                 # same N, d, structure, seed; fewer heads
+    x = make_inputs(ws, device="cpu")
+    f64 = lambda t: t.to(torch.bfloat16).to(torch.float64).numpy()
+    qo = x["q_offsets"].numpy().astype(np.int64)
+    ko = x["k_offsets"].numpy().astype(np.int64)
+    nqb = len(qo) - 1
+    t_prep = 0.0
+    t_att = 0.0
+    n_att = 0
+    rng = np.random.default_rng(seed)
+    for h in range(n_heads):
+        Q, K, V = f64(x["Q"][h]), f64(x["K"][h]), f64(x["V"][h])
+        qp = x["q_perm"][h].numpy().astype(np.int64)
+        kp = x["k_perm"][h].numpy().astype(np.int64)
+        t0 = time.perf_counter()
+        r = O.forward_head(Q, K, V, qp, kp, qo, ko, w.ratio, blocks=[])
+        t_prep += time.perf_counter() - t0
+        blocks = rng.choice(nqb, size=n_units // n_heads, replace=False)
+        Qp, Kp, Vp = Q[qp], K[kp], V[kp]
+        scale = 1.0 / math.sqrt(w.d)
+        t0 = time.perf_counter()
+        for A in blocks:
+            O.attend_block(Qp[qo[A]:qo[A + 1]], Kp, Vp, ko, r.sel[A], r.k_tilde, r.v_tilde,
+                           r.c, scale)
+        t_att += time.perf_counter() - t0
+        n_att += len(blocks)
+    per_call = (t_prep / n_heads) * w.H + (t_att / n_att) * w.H * nqb
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    desc = (f"oracle (float64 numpy) on {n_heads} of {w.H} heads (summaries + routing, full) and "
+            f"{n_att} of {w.H * nqb} query blocks (attention); extrapolated linearly to one "
+            f"full call; measured {t_prep + t_att:.1f} s")
+    return per_call, threads, desc
+
+
+def dense_flops(w):
+    return 4.0 * w.H * float(w.N) ** 2 * w.d
+
+
+# --------------------------------------------------------------------------------- main
+
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def run_reference(args, world, rank):
+    from block_sparse_attention_gather_b200.workloads import WORKLOADS
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    times = []
+    for i in range(args.warmup + args.steps):
+        per_call, threads, desc = oracle_sample(w, n_heads=1, n_units=4, seed=i)
+        if i >= args.warmup:
+            times.append(per_call)
+    t = statistics.mean(times)
+    value = dense_flops(w) / t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "H": w.H, "N": w.N, "d": w.d, "topk_ratio": w.ratio,
+                   "block": w.block, "layout": w.layout, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = init_dist()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    if args.warmup < 3:
+        raise SystemExit("at least 3 warm-up steps are required")
+    from block_sparse_attention_gather_b200.workloads import WORKLOADS, make_inputs
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w, device=device)
+    hp = HotPath(x, w.ratio, device)
+    peaks, peak_kind = load_peaks()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        hp.step()
+    torch.cuda.synchronize()
+    flags = int(hp.v["err"].item())
+    if flags:
+        raise RuntimeError(f"device error word {flags:#x} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    clocks = ClockSampler(device)
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        hp.step(evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    clock_info = clocks.stop()
+
+    per_kernel = {n: [] for n in KERNELS}
+    totals = []
+    for e in evs:
+        for j, n in enumerate(KERNELS):
+            per_kernel[n].append(e[j].elapsed_time(e[j + 1]))
+        totals.append(e[0].elapsed_time(e[5]))
+    total_ms = sum(totals)
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([total_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    dflops = dense_flops(w)
+    value = world * dflops * args.steps / (total_ms / 1e3) / 1e12
+    flags = int(hp.v["err"].item())
+    if flags:
+        raise RuntimeError(f"device error word {flags:#x} after the timed region")
+
+    att_flops = attention_flops(hp)
+    att_ms = statistics.mean(per_kernel["attend"])
+    achieved = att_flops / (att_ms / 1e3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    kb = kernel_bytes(hp)
+    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    kernels = {}
+    for n in KERNELS:
+        ms = statistics.mean(per_kernel[n])
+        entry = {"ms": ms, "share": ms / ms_per_step}
+        if n in kb:
+            gbs = kb[n] / (ms / 1e3) / 1e9
+            entry.update({"bytes": kb[n], "GB/s": gbs, "hbm_frac": gbs / hbm_peak})
+        else:
+            entry.update({"flops": att_flops, "TFLOP/s": achieved, "tensor_frac": achieved / peak})
+        kernels[n] = entry
+
+    # ---- end to end through the public call with host buffers (pinned), copies timed
+    e2e = None
+    if args.e2e_steps > 0:
+        from block_sparse_attention_gather_b200 import spark_bsa_forward
+        host = {n: x[n].to("cpu").pin_memory() for n in
+                ("Q", "K", "V", "q_perm", "k_perm", "q_offsets", "k_offsets")}
+        dev_in = {n: torch.empty_like(x[n]) for n in host}
+        out_host = torch.empty(hp.out.shape, dtype=hp.out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_host.numel() * out_host.element_size()
+        s = torch.cuda.current_stream(device)
+
+        def e2e_step():
+            for n in host:
+                dev_in[n].copy_(host[n], non_blocking=True)
+            o, _, _ = spark_bsa_forward(dev_in["Q"], dev_in["K"], dev_in["V"], dev_in["q_perm"],
+                                        dev_in["k_perm"], dev_in["q_offsets"],
+                                        dev_in["k_offsets"], w.ratio, out=hp.out,
+                                        workspace=hp.ws)
+            out_host.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(s)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(s)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            import torch.distributed as dist
+            tt = torch.tensor([e_ms], device=device, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": world * dflops * args.e2e_steps / (e_ms / 1e3) / 1e12, "unit": UNIT,
+               "ms_per_call": e_ms / args.e2e_steps, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+        del host, dev_in, out_host
+
+    traffic = profiled_traffic(hp)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "H": w.H, "N": w.N, "d": w.d, "topk_ratio": w.ratio,
+                   "k": hp.k, "nqb": hp.nqb, "nkb": hp.nkb, "block": w.block,
+                   "layout": w.layout, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (4.5 GB of Q/K/V per call), no flush"},
+        "actual_tflops": att_flops / (ms_per_step / 1e3) / 1e12 * world,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_kind": f"bf16 sustained, {peak_kind}",
+                     "kernel": "attend (tcgen05 two-branch attention)",
+                     "algorithmic_flops_per_launch": att_flops},
+        "kernels": kernels,
+        "gpu_launches": 5 * args.steps,
+        "clocks": clock_info,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        per_call, threads, desc = oracle_sample(w, n_heads=2, n_units=64)
+        line["cpu_baseline"] = {"value": dflops / per_call / 1e12, "unit": UNIT,
+                                "cores": threads, "kind": "oracle", "sample": desc,
+                                "ms_per_call_extrapolated": per_call * 1e3}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -34,7 +34,9 @@ namespace spark {
 namespace {
 
 constexpr int kStages = 3;
-constexpr int kThreads = 224;
+constexpr int kSoftmaxThreads = 256;            // 8 warps: 4 row quarters x 2 column halves
+constexpr int kWarpK = 8, kWarpV = 9, kWarpMma = 10;
+constexpr int kThreads = 352;
 constexpr uint32_t kColQ = 0, kColP = 64, kColS0 = 128, kColS1 = 256, kColO = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
@@ -42,6 +44,7 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units
 struct __align__(8) Barriers {
   uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages];
   uint64_t qready, sfull[2], pready, pvdone, drain;
+  uint64_t pair[4];        // the two softmax warps of a row quarter: one phase per exchange
 };
 
 __device__ __forceinline__ bool wait_bounded_ignore_abort(uint64_t* bar, uint32_t parity) {
@@ -103,6 +106,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   const int A = blockIdx.x, h = blockIdx.y;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   __shared__ int s_skip;
+  __shared__ float red_max[2][2][128];     // [tile parity][column half][row]
+  __shared__ float red_l[2][128];          // [column half][row]
   if (tid == 0) s_skip = launch_timed_out(err) ? 1 : 0;   // an earlier CTA gave up
   __syncthreads();
   if (s_skip) return;                                      // uniform: no work, nothing held
@@ -118,12 +123,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       mbar_init(&bars->vfull[s], 1);
       mbar_init(&bars->vempty[s], 1);
     }
-    mbar_init(&bars->qready, 128);
+    mbar_init(&bars->qready, kSoftmaxThreads);
     mbar_init(&bars->sfull[0], 1);
     mbar_init(&bars->sfull[1], 1);
-    mbar_init(&bars->pready, 128);
+    mbar_init(&bars->pready, kSoftmaxThreads);
     mbar_init(&bars->pvdone, 1);
     mbar_init(&bars->drain, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&bars->pair[q], 64);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -143,10 +149,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   __syncthreads();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 4 || warp == 5) {
+  if (warp == kWarpK || warp == kWarpV) {
     // ------------------------------------------------------------- TMA producers
     if (lane == 0) {
-      const bool is_k = (warp == 4);
+      const bool is_k = (warp == kWarpK);
       uint8_t* ring = is_k ? kst : vst;
       uint64_t* full = is_k ? bars->kfull : bars->vfull;
       uint64_t* empty = is_k ? bars->kempty : bars->vempty;
@@ -171,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           wait_bounded_ignore_abort(&full[t % kStages], (t / kStages) & 1);
       }
     }
-  } else if (warp == 6) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
@@ -217,26 +223,39 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     }
   } else {
     // ------------------------------------------------------------------ softmax rows
-    const int row = tid;                                  // 0..127 == TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // Warp w handles TMEM lanes 32*(w%4).. (query rows) and S columns 64*(w/4)..+63; the
+    // two warps of a row quarter exchange their partial row maxima once per tile.
+    const int q4 = warp & 3, half = warp >> 2;
+    const int row = q4 * 32 + lane;                       // 0..127 == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    uint64_t* pair_bar = &bars->pair[q4];                 // exchange barrier of the pair
+    const int col0 = half * 64;                           // first S column of this warp
+    constexpr int OH = D / 2;                             // O columns per warp
     const int qlo = q_offsets[A];
     const int qhi = q_offsets[A + 1];
     const int qsize = max(0, min(qhi - qlo, kMaxBlock));
-    // Q row -> TMEM (rows past the block read the next rows; they are never stored)
+    // this warp's half of the Q row -> TMEM (rows past the block are never stored)
     {
       const int qrow = min(max(qlo, 0), N - 1) + row;
       const bool in = qrow < N;
       const uint32_t* src = reinterpret_cast<const uint32_t*>(
-          Qp + (static_cast<size_t>(h) * N + (in ? qrow : 0)) * D);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+          Qp + (static_cast<size_t>(h) * N + (in ? qrow : 0)) * D) + half * (D / 4);
+      if constexpr (D == 128) {
         uint32_t r[32];
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
-          const uint4 v = in ? *reinterpret_cast<const uint4*>(src + c * 32 + j) : make_uint4(0, 0, 0, 0);
+          const uint4 v = in ? *reinterpret_cast<const uint4*>(src + j) : make_uint4(0, 0, 0, 0);
           r[j] = v.x; r[j + 1] = v.y; r[j + 2] = v.z; r[j + 3] = v.w;
         }
-        tmem_st32(tbase + lane_off + kColQ + c * 32, r);
+        tmem_st32(tbase + lane_off + kColQ + half * 32, r);
+      } else {
+        uint32_t r[16];
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+          const uint4 v = in ? *reinterpret_cast<const uint4*>(src + j) : make_uint4(0, 0, 0, 0);
+          r[j] = v.x; r[j + 1] = v.y; r[j + 2] = v.z; r[j + 3] = v.w;
+        }
+        tmem_st16(tbase + lane_off + kColQ + half * 16, r);
       }
     }
     tc_fence_before_sync();
@@ -251,33 +270,43 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }   // collectives below
       tc_fence_after_sync();
       const TileInfo ti = tile_info(t, k, sel_row, k_offsets, nkb, N);
-      const uint32_t scol = tbase + lane_off + ((t & 1) ? kColS1 : kColS0);
-      float x[128];
+      float x[64];
       {
         uint32_t r[64];
-        tmem_ld64(scol, r);
+        tmem_ld64(tbase + lane_off + ((t & 1) ? kColS1 : kColS0) + col0, r);
 #pragma unroll
         for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(r[j]);
-        tmem_ld64(scol + 64, r);
-#pragma unroll
-        for (int j = 0; j < 64; ++j) x[64 + j] = __uint_as_float(r[j]);
       }
-      float mt = -INFINITY;
+      // x holds raw scores on exact tiles (scale folded into the exponent below) and
+      // log2-domain logits with the summary offsets on summary tiles; masked = -inf.
       if (ti.exact) {
+        if (ti.nvalid < col0 + 64) {
 #pragma unroll
-        for (int j = 0; j < 128; ++j) {
-          x[j] = (j < ti.nvalid) ? x[j] * scale_log2 : -INFINITY;
-          mt = fmaxf(mt, x[j]);
+          for (int j = 0; j < 64; ++j)
+            if (col0 + j >= ti.nvalid) x[j] = -INFINITY;
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 128; ++j) {
-          const int B = ti.y + j;
+        for (int j = 0; j < 64; ++j) {
+          const int B = ti.y + col0 + j;
           const bool live = B < nkb && !((selmask[B >> 5] >> (B & 31)) & 1u);
           x[j] = live ? fmaf(x[j], scale_log2, cb[B] * kLog2e) : -INFINITY;
-          mt = fmaxf(mt, x[j]);
         }
       }
+      float mx[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mx[a] = x[a];
+#pragma unroll
+      for (int j = 8; j < 64; ++j) mx[j & 7] = fmaxf(mx[j & 7], x[j]);
+      float mloc = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      if (ti.exact) mloc *= scale_log2;                   // -inf stays -inf
+      // combine with the other column half of the same rows (double-buffered slot)
+      red_max[t & 1][half][row] = mloc;
+      mbar_arrive(pair_bar);
+      ok = mbar_wait(pair_bar, t & 1, abort_flag, err);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      const float mt = fmaxf(mloc, red_max[t & 1][half ^ 1][row]);
       bool need = false;
       float m_new = m_run;
       if (t == 0) {
@@ -286,15 +315,30 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         need = true;
         m_new = mt;
       }
-      float rowsum = 0.f;
-      uint32_t pk[64];
+      float sum[8];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const float p0 = ex2_approx(x[2 * j] - m_new);
-        const float p1 = ex2_approx(x[2 * j + 1] - m_new);
-        rowsum += p0 + p1;
-        pk[j] = pack_bf16(p0, p1);
+      for (int a = 0; a < 8; ++a) sum[a] = 0.f;
+      uint32_t pk[32];
+      if (ti.exact) {
+        const float nm = -m_new;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float p0 = ex2_approx(fmaf(x[2 * j], scale_log2, nm));
+          const float p1 = ex2_approx(fmaf(x[2 * j + 1], scale_log2, nm));
+          sum[j & 7] += p0 + p1;
+          pk[j] = pack_bf16(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float p0 = ex2_approx(x[2 * j] - m_new);
+          const float p1 = ex2_approx(x[2 * j + 1] - m_new);
+          sum[j & 7] += p0 + p1;
+          pk[j] = pack_bf16(p0, p1);
+        }
       }
+      const float rowsum = ((sum[0] + sum[1]) + (sum[2] + sum[3])) +
+                           ((sum[4] + sum[5]) + (sum[6] + sum[7]));
       // P and O of the previous tile are in use until its PV MMA completes
       if (t > 0) {
         ok = mbar_wait(&bars->pvdone, (t - 1) & 1, abort_flag, err);
@@ -305,48 +349,49 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
         l_run *= alpha;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < OH / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(tbase + lane_off + kColO + c * 32, r);
+          const uint32_t oa = tbase + lane_off + kColO + half * OH + c * 32;
+          tmem_ld32(oa, r);
 #pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-          tmem_st32(tbase + lane_off + kColO + c * 32, r);
+          tmem_st32(oa, r);
         }
       }
       l_run += rowsum;
       m_run = m_new;
-      {
-        uint32_t r[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = pk[j];
-        tmem_st32(tbase + lane_off + kColP, r);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = pk[32 + j];
-        tmem_st32(tbase + lane_off + kColP + 32, r);
-      }
+      tmem_st32(tbase + lane_off + kColP + half * 32, pk);
       tc_fence_before_sync();
       mbar_arrive(&bars->pready);
     }
     // ---- epilogue: O / l scattered to the original token order
     bool fine = ok && T > 0;
     if (fine) fine = mbar_wait(&bars->pvdone, (T - 1) & 1, abort_flag, err);
+    // the pair exchanges its partial row sums (bounded wait: a partner that gave up early
+    // cannot block this warp)
+    if (fine) {
+      red_l[half][row] = l_run;
+      mbar_arrive(pair_bar);
+      fine = mbar_wait(pair_bar, T & 1, abort_flag, err);
+    }
     if (__all_sync(0xffffffffu, fine)) {
+      const float l_tot = l_run + red_l[half ^ 1][row];
       tc_fence_after_sync();
-      const float inv = 1.f / l_run;
+      const float inv = 1.f / l_tot;
       int tok = -1;
       if (row < qsize) {
         tok = q_perm[static_cast<size_t>(h) * N + qlo + row];
         if (tok < 0 || tok >= N) {
-          flag_error(err, kErrPerm);
+          if (half == 0) flag_error(err, kErrPerm);
           tok = -1;
         }
       }
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < OH / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tbase + lane_off + kColO + c * 32, r);
+        tmem_ld32(tbase + lane_off + kColO + half * OH + c * 32, r);
         if (tok >= 0) {
-          const size_t o = (static_cast<size_t>(h) * N + tok) * D + c * 32;
+          const size_t o = (static_cast<size_t>(h) * N + tok) * D + half * OH + c * 32;
           if (out_dtype == 0) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + o);
 #pragma unroll
