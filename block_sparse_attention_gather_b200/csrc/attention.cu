@@ -40,11 +40,15 @@ constexpr int kThreads = 352;
 constexpr uint32_t kColQ = 0, kColP = 64, kColS0 = 128, kColS1 = 256, kColO = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr int kMaxSmemBias = 6144;          // summary offsets kept in shared memory (floats)
+
+// Which of a thread's 32 exponential pairs per tile go to the polynomial (FMA pipe) instead
+// of MUFU: 8 of 32, which balances the two pipes against the tensor-core time of a tile.
+__device__ __forceinline__ constexpr bool poly_pair(int j) { return (j & 3) == 3; }
 
 struct __align__(8) Barriers {
   uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages];
-  uint64_t qready, sfull[2], pready, pvdone, drain;
-  uint64_t pair[4];        // the two softmax warps of a row quarter: one phase per exchange
+  uint64_t qready, sfull[2], sfree[2], pready, pvdone, drain;
 };
 
 __device__ __forceinline__ bool wait_bounded_ignore_abort(uint64_t* bar, uint32_t parity) {
@@ -62,24 +66,45 @@ struct TileInfo {
   bool exact;
 };
 
-__device__ __forceinline__ TileInfo tile_info(int t, int k, const int32_t* sel_row,
-                                              const int32_t* k_offsets, int nkb, int N) {
-  TileInfo ti;
-  if (t < k) {
-    int B = sel_row[t];
-    B = min(max(B, 0), nkb - 1);
-    const int lo = min(max(k_offsets[B], 0), N - 1);
-    const int hi = min(max(k_offsets[B + 1], lo), N);
-    ti.y = lo;
-    ti.nvalid = min(hi - lo, kMaxBlock);
-    ti.exact = true;
-  } else {
-    ti.y = (t - k) * 128;
-    ti.nvalid = 128;
-    ti.exact = false;
+// Walks the tile list with the metadata of tile t+1 (and the selected id of tile t+2)
+// loaded one step ahead, so that the dependent global loads (selected id, then the block's
+// offsets) never sit on a role's critical path.
+struct TileCursor {
+  const int32_t* sel_row;
+  const int32_t* k_offsets;
+  int k, nkb, N;
+  int b_ahead;        // selected id of tile t+2
+  TileInfo next;      // metadata of tile t+1
+
+  __device__ __forceinline__ TileInfo info(int t, int B) const {
+    TileInfo ti;
+    if (t < k) {
+      B = min(max(B, 0), nkb - 1);
+      const int lo = min(max(k_offsets[B], 0), N - 1);
+      const int hi = min(max(k_offsets[B + 1], lo), N);
+      ti.y = lo;
+      ti.nvalid = min(hi - lo, kMaxBlock);
+      ti.exact = true;
+    } else {
+      ti.y = (t - k) * 128;
+      ti.nvalid = 128;
+      ti.exact = false;
+    }
+    return ti;
   }
-  return ti;
-}
+  __device__ __forceinline__ void init() {
+    const int b0 = (k > 0) ? sel_row[0] : 0;
+    b_ahead = (k > 1) ? sel_row[1] : 0;
+    next = info(0, b0);
+  }
+  // returns the metadata of tile t and starts the loads for tiles t+1 and t+2
+  __device__ __forceinline__ TileInfo advance(int t) {
+    const TileInfo cur = next;
+    next = info(t + 1, b_ahead);
+    b_ahead = (t + 2 < k) ? sel_row[t + 2] : 0;
+    return cur;
+  }
+};
 
 }  // namespace
 
@@ -102,6 +127,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* selmask = reinterpret_cast<uint32_t*>(tmem_slot + 4);
+  // summary-row offsets of this CTA in log2 units, -inf for selected blocks and padding
+  // (when nct*128 <= kMaxSmemBias; larger problems read them from global memory)
+  float* biasrow = reinterpret_cast<float*>(selmask + ((nkb + 31) / 32 + 3) / 4 * 4);
 
   const int A = blockIdx.x, h = blockIdx.y;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -115,6 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   const int T = k + nct;
   const int32_t* sel_row = sel + (static_cast<size_t>(h) * nqb + A) * k;
   const int nwords = (nkb + 31) / 32;
+  const bool bias_smem = nct > 0 && nct * 128 <= kMaxSmemBias;
+  const float* cb = cbias + static_cast<size_t>(h) * nkb;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -129,11 +159,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     mbar_init(&bars->pready, kSoftmaxThreads);
     mbar_init(&bars->pvdone, 1);
     mbar_init(&bars->drain, 1);
-    for (int q = 0; q < 4; ++q) mbar_init(&bars->pair[q], 64);
+    mbar_init(&bars->sfree[0], kSoftmaxThreads);
+    mbar_init(&bars->sfree[1], kSoftmaxThreads);
     *abort_flag = 0;
     mbar_fence_init();
   }
   for (int i = tid; i < nwords; i += kThreads) selmask[i] = 0u;
+  if (bias_smem)
+    for (int i = tid; i < nct * 128; i += kThreads) biasrow[i] = (i < nkb) ? cb[i] * kLog2e : -INFINITY;
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -143,8 +176,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   tc_fence_after_sync();
   for (int i = tid; i < k; i += kThreads) {
     const int B = sel_row[i];
-    if (B >= 0 && B < nkb) atomicOr(&selmask[B >> 5], 1u << (B & 31));
-    else flag_error(err, kErrSel);
+    if (B >= 0 && B < nkb) {
+      atomicOr(&selmask[B >> 5], 1u << (B & 31));
+      if (bias_smem) biasrow[B] = -INFINITY;
+    } else {
+      flag_error(err, kErrSel);
+    }
   }
   __syncthreads();
   const uint32_t tbase = *tmem_slot;
@@ -161,10 +198,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       tma_prefetch_desc(mx);
       tma_prefetch_desc(ms);
       int issued = 0;
+      TileCursor cur{sel_row, k_offsets, k, nkb, N};
+      cur.init();
       for (int t = 0; t < T; ++t) {
         const int s = t % kStages;
+        const TileInfo ti = cur.advance(t);
         if (t >= kStages && !mbar_wait(&empty[s], ((t / kStages) - 1) & 1, abort_flag, err)) break;
-        const TileInfo ti = tile_info(t, k, sel_row, k_offsets, nkb, N);
         mbar_arrive_expect_tx(&full[s], TILE_BYTES);
         for (int a = 0; a < NATOM; ++a)
           tma_load_3d(ring + s * TILE_BYTES + a * 16384, ti.exact ? mx : ms, &full[s], a * 64,
@@ -187,7 +226,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       auto issue_s = [&](int t) -> bool {
         const int s = t % kStages;
         if (!mbar_wait(&bars->kfull[s], (t / kStages) & 1, abort_flag, err)) return false;
-        tc_fence_after_sync();
         const uint32_t dcol = tbase + ((t & 1) ? kColS1 : kColS0);
         const uint32_t kaddr = smem_u32(kst + s * TILE_BYTES);
 #pragma unroll
@@ -202,11 +240,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       if (ok && T > 0) ok = issue_s(0);
       if (ok && T > 1) ok = issue_s(1);
       for (int t = 0; ok && t < T; ++t) {
+        // S(t+2) goes into the buffer of S(t) as soon as the softmax has read S(t), so that
+        // the tensor cores compute it while the softmax of tile t runs
+        if (t + 2 < T) {
+          if (!mbar_wait(&bars->sfree[t & 1], (t >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after_sync();
+          if (!(ok = issue_s(t + 2))) break;
+        }
         if (!mbar_wait(&bars->pready, t & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after_sync();
         const int s = t % kStages;
         if (!mbar_wait(&bars->vfull[s], (t / kStages) & 1, abort_flag, err)) { ok = false; break; }
-        tc_fence_after_sync();
         const uint32_t vaddr = smem_u32(vst + s * TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -215,7 +259,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         }
         tc_commit(&bars->pvdone);
         tc_commit(&bars->vempty[s]);
-        if (t + 2 < T) ok = issue_s(t + 2);
       }
       // make sure nothing this thread issued is still running before TMEM is freed
       tc_commit(&bars->drain);
@@ -228,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     const int q4 = warp & 3, half = warp >> 2;
     const int row = q4 * 32 + lane;                       // 0..127 == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    uint64_t* pair_bar = &bars->pair[q4];                 // exchange barrier of the pair
+    const uint32_t bar_id = 1 + q4;                       // named barrier of the warp pair
     const int col0 = half * 64;                           // first S column of this warp
     constexpr int OH = D / 2;                             // O columns per warp
     const int qlo = q_offsets[A];
@@ -262,20 +305,29 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     mbar_arrive(&bars->qready);
 
     const float scale_log2 = kLog2e * rsqrtf(static_cast<float>(D));
-    const float* cb = cbias + static_cast<size_t>(h) * nkb;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
+    TileCursor cur{sel_row, k_offsets, k, nkb, N};
+    cur.init();
+    // The loop never exits early: the two warps of a row quarter must execute the same
+    // sequence of named-barrier exchanges.  After a failed (bounded) wait `ok` stays false
+    // for the warp and every later TMEM access, arrival and store of the warp is skipped.
     for (int t = 0; t < T; ++t) {
-      ok = mbar_wait(&bars->sfull[t & 1], (t >> 1) & 1, abort_flag, err);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }   // collectives below
-      tc_fence_after_sync();
-      const TileInfo ti = tile_info(t, k, sel_row, k_offsets, nkb, N);
+      const TileInfo ti = cur.advance(t);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->sfull[t & 1], (t >> 1) & 1, abort_flag, err));
       float x[64];
-      {
+      if (ok) {
+        tc_fence_after_sync();
         uint32_t r[64];
         tmem_ld64(tbase + lane_off + ((t & 1) ? kColS1 : kColS0) + col0, r);
 #pragma unroll
         for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(r[j]);
+        // S(t) is in registers: its TMEM buffer may take S(t+2)
+        tc_fence_before_sync();
+        mbar_arrive(&bars->sfree[t & 1]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) x[j] = -INFINITY;
       }
       // x holds raw scores on exact tiles (scale folded into the exponent below) and
       // log2-domain logits with the summary offsets on summary tiles; masked = -inf.
@@ -285,27 +337,41 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           for (int j = 0; j < 64; ++j)
             if (col0 + j >= ti.nvalid) x[j] = -INFINITY;
         }
+      } else if (bias_smem) {
+        const float4* br = reinterpret_cast<const float4*>(biasrow + ti.y + col0);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float4 b = br[j];
+          x[4 * j] = fmaf(x[4 * j], scale_log2, b.x);
+          x[4 * j + 1] = fmaf(x[4 * j + 1], scale_log2, b.y);
+          x[4 * j + 2] = fmaf(x[4 * j + 2], scale_log2, b.z);
+          x[4 * j + 3] = fmaf(x[4 * j + 3], scale_log2, b.w);
+        }
       } else {
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
           const int B = ti.y + col0 + j;
-          const bool live = B < nkb && !((selmask[B >> 5] >> (B & 31)) & 1u);
-          x[j] = live ? fmaf(x[j], scale_log2, cb[B] * kLog2e) : -INFINITY;
+          const int Bc = min(B, nkb - 1);
+          const float c = cb[Bc];                         // unconditional: loads batch up
+          const uint32_t bits = selmask[Bc >> 5];
+          const bool live = B < nkb && !((bits >> (Bc & 31)) & 1u);
+          x[j] = live ? fmaf(x[j], scale_log2, c * kLog2e) : -INFINITY;
         }
       }
-      float mx[8];
+      // row maximum of this half: four chains of three-input maxima
+      float mx[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mx[a] = x[a];
-#pragma unroll
-      for (int j = 8; j < 64; ++j) mx[j & 7] = fmaxf(mx[j & 7], x[j]);
-      float mloc = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int j = 4; j < 64; j += 8) {
+        mx[0] = fmax3(mx[0], x[j], x[j + 1]);
+        mx[1] = fmax3(mx[1], x[j + 2], x[j + 3]);
+        mx[2] = fmax3(mx[2], x[j + 4], x[j + 5]);
+        mx[3] = fmax3(mx[3], x[j + 6], x[j + 7]);
+      }
+      float mloc = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
       if (ti.exact) mloc *= scale_log2;                   // -inf stays -inf
       // combine with the other column half of the same rows (double-buffered slot)
       red_max[t & 1][half][row] = mloc;
-      mbar_arrive(pair_bar);
-      ok = mbar_wait(pair_bar, t & 1, abort_flag, err);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      named_bar_sync(bar_id, 64);
       const float mt = fmaxf(mloc, red_max[t & 1][half ^ 1][row]);
       bool need = false;
       float m_new = m_run;
@@ -315,36 +381,36 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         need = true;
         m_new = mt;
       }
-      float sum[8];
-#pragma unroll
-      for (int a = 0; a < 8; ++a) sum[a] = 0.f;
+      // p = 2^(x*c - m) on exact tiles (raw scores), 2^(x - m) on summary tiles, two
+      // columns at a time; a quarter of the pairs use the FMA-pipe polynomial
+      const uint64_t c2 = f2_splat(ti.exact ? scale_log2 : 1.f);
+      const uint64_t nm2 = f2_splat(-m_new);
+      uint64_t sum2[4] = {0, 0, 0, 0};
       uint32_t pk[32];
-      if (ti.exact) {
-        const float nm = -m_new;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float p0 = ex2_approx(fmaf(x[2 * j], scale_log2, nm));
-          const float p1 = ex2_approx(fmaf(x[2 * j + 1], scale_log2, nm));
-          sum[j & 7] += p0 + p1;
-          pk[j] = pack_bf16(p0, p1);
+      for (int j = 0; j < 32; ++j) {
+        const uint64_t a2 = f2_fma(f2_pack(x[2 * j], x[2 * j + 1]), c2, nm2);
+        float p0, p1;
+        if (poly_pair(j)) {
+          exp2_poly2(a2, p0, p1);
+        } else {
+          float a0, a1;
+          f2_unpack(a2, a0, a1);
+          p0 = ex2_approx(a0);
+          p1 = ex2_approx(a1);
         }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float p0 = ex2_approx(x[2 * j] - m_new);
-          const float p1 = ex2_approx(x[2 * j + 1] - m_new);
-          sum[j & 7] += p0 + p1;
-          pk[j] = pack_bf16(p0, p1);
-        }
+        sum2[j & 3] = f2_add(sum2[j & 3], f2_pack(p0, p1));
+        pk[j] = pack_bf16(p0, p1);
       }
-      const float rowsum = ((sum[0] + sum[1]) + (sum[2] + sum[3])) +
-                           ((sum[4] + sum[5]) + (sum[6] + sum[7]));
+      float s0, s1;
+      f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
+      const float rowsum = s0 + s1;
       // P and O of the previous tile are in use until its PV MMA completes
-      if (t > 0) {
-        ok = mbar_wait(&bars->pvdone, (t - 1) & 1, abort_flag, err);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after_sync();
+      if (ok && t > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->pvdone, (t - 1) & 1, abort_flag, err));
+        if (ok) tc_fence_after_sync();
       }
+      if (!ok) continue;
       if (__any_sync(0xffffffffu, need)) {
         const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
         l_run *= alpha;
@@ -367,14 +433,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     // ---- epilogue: O / l scattered to the original token order
     bool fine = ok && T > 0;
     if (fine) fine = mbar_wait(&bars->pvdone, (T - 1) & 1, abort_flag, err);
-    // the pair exchanges its partial row sums (bounded wait: a partner that gave up early
-    // cannot block this warp)
+    fine = __all_sync(0xffffffffu, fine);
+    // the pair exchanges its partial row sums (both warps always reach this barrier)
+    red_l[half][row] = l_run;
+    named_bar_sync(bar_id, 64);
     if (fine) {
-      red_l[half][row] = l_run;
-      mbar_arrive(pair_bar);
-      fine = mbar_wait(pair_bar, T & 1, abort_flag, err);
-    }
-    if (__all_sync(0xffffffffu, fine)) {
       const float l_tot = l_run + red_l[half ^ 1][row];
       tc_fence_after_sync();
       const float inv = 1.f / l_tot;
@@ -422,9 +485,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   }
 }
 
-static size_t attend_smem_bytes(int d, int nkb) {
+static size_t attend_smem_bytes(int d, int nkb, int k) {
   const size_t tile = static_cast<size_t>(128) * d * 2;
-  return 1024 + 2 * kStages * tile + sizeof(Barriers) + 16 + ((nkb + 31) / 32) * 4 + 16;
+  const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
+  const size_t words = ((nkb + 31) / 32 + 3) / 4 * 4;
+  const size_t bias = (nct > 0 && nct * 128 <= kMaxSmemBias) ? static_cast<size_t>(nct) * 128 * 4 : 0;
+  return 1024 + 2 * kStages * tile + sizeof(Barriers) + 16 + words * 4 + bias;
 }
 
 template <int D>
@@ -432,7 +498,7 @@ static cudaError_t launch_attend_t(const AttendMaps& m, const float* cbias, cons
                                    int k, const int32_t* q_perm, const int32_t* q_offsets,
                                    int nqb, const int32_t* k_offsets, int nkb, int H, int N,
                                    void* out, int out_dtype, uint32_t* err, cudaStream_t s) {
-  const size_t smem = attend_smem_bytes(D, nkb);
+  const size_t smem = attend_smem_bytes(D, nkb, k);
   cudaError_t e = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
