@@ -1,0 +1,133 @@
+"""The C ABI without a GPU: the library loads, exports every function the header declares,
+and rejects bad arguments on the host before anything touches a device."""
+
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spark_bsa.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_sparse_attention_gather_b200.build import build_library, is_stale
+    if is_stale():
+        build_library()
+    from block_sparse_attention_gather_b200 import lib
+    return lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"SPARK_API\s+[\w\s\*]+?\b(spark_\w+)\s*\(", src)
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in spark_bsa.h but not exported"
+    from block_sparse_attention_gather_b200 import EXPORTED
+    assert set(EXPORTED) == set(names)
+
+
+def test_status_strings(L):
+    from block_sparse_attention_gather_b200 import spark_status_string
+    for code, name in [(0, "SPARK_OK"), (1, "SPARK_ERR_INVALID_ARG"), (2, "SPARK_ERR_UNSUPPORTED"),
+                       (3, "SPARK_ERR_WORKSPACE"), (4, "SPARK_ERR_CUDA"),
+                       (5, "SPARK_ERR_DEVICE_CHECK")]:
+        assert spark_status_string(code) == name
+    assert spark_status_string(99) == "SPARK_UNKNOWN_STATUS"
+
+
+def test_topk_count_matches_the_oracle(L):
+    from block_sparse_attention_gather_b200 import spark_bsa_topk_count
+    from oracle import spark_oracle as O
+    for nkb in (1, 2, 7, 16, 256, 473, 1890, 2520, 12800):
+        for ratio in (1e-6, 0.01, 0.05, 0.1, 0.125, 0.2, 0.3, 1 / 3, 0.5, 0.95, 1.0):
+            assert spark_bsa_topk_count(nkb, ratio) == O.topk_count(ratio, nkb)
+    assert spark_bsa_topk_count(10, 0.0) == -1
+    assert spark_bsa_topk_count(10, 1.5) == -1
+    assert spark_bsa_topk_count(0, 0.5) == -1
+
+
+def test_workspace_layout(L):
+    from block_sparse_attention_gather_b200 import (spark_bsa_workspace_layout,
+                                                    spark_bsa_workspace_size)
+    H, N, d, nqb, nkb = 24, 241920, 128, 1890, 1890
+    lay = spark_bsa_workspace_layout(H, N, d, nqb, nkb, 0.1)
+    assert lay.k == 189
+    offs = [lay.Qp, lay.Kp, lay.Vp, lay.qbar_blocks, lay.qbar, lay.kbar, lay.k_tilde,
+            lay.v_tilde, lay.cbias, lay.sel, lay.err, lay.total]
+    assert all(o % 256 == 0 for o in offs)
+    assert offs == sorted(offs)
+    sizes = [H * N * d * 2] * 3 + [H * nqb * d * 4, H * d * 4, H * nkb * d * 4,
+                                   H * nkb * d * 2, H * nkb * d * 2, H * nkb * 4,
+                                   H * nqb * 189 * 4, 4]
+    for a, b, sz in zip(offs, offs[1:], sizes):
+        assert b - a >= sz
+    assert spark_bsa_workspace_size(H, N, d, nqb, nkb, 0.1) == lay.total
+    assert spark_bsa_workspace_size(H, N, 96, nqb, nkb, 0.1) == 0
+
+
+def _fwd(L, **kw):
+    """spark_bsa_forward with fake but aligned pointers: only host checks may run."""
+    p = ctypes.c_void_p(0x100000)
+    a = dict(Q=p, K=p, V=p, dtype=0, H=2, N=1000, d=128, q_perm=p, k_perm=p, qo=p, nqb=10,
+             ko=p, nkb=10, ratio=0.2, out=p, ws=p, ws_bytes=0, stream=None)
+    a.update(kw)
+    return L.spark_bsa_forward(a["Q"], a["K"], a["V"], a["dtype"], a["H"], a["N"], a["d"],
+                               a["q_perm"], a["k_perm"], a["qo"], a["nqb"], a["ko"], a["nkb"],
+                               a["ratio"], a["out"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def test_forward_rejects_bad_arguments_on_the_host(L):
+    assert _fwd(L, Q=None) == INVALID
+    assert _fwd(L, out=None) == INVALID
+    assert _fwd(L, dtype=7) == INVALID
+    assert _fwd(L, d=96) == UNSUPPORTED
+    assert _fwd(L, H=0) == INVALID
+    assert _fwd(L, nqb=0) == INVALID
+    assert _fwd(L, nkb=2000) == INVALID            # more blocks than tokens
+    assert _fwd(L, N=20000, nkb=12801) == UNSUPPORTED
+    assert _fwd(L, ratio=0.0) == INVALID
+    assert _fwd(L, ratio=1.01) == INVALID
+    assert _fwd(L, ratio=float("nan")) == INVALID
+    assert _fwd(L, Q=ctypes.c_void_p(0x100004)) == INVALID      # not 16-byte aligned
+    assert _fwd(L, ws=None) == WORKSPACE
+    assert _fwd(L, ws_bytes=1024) == WORKSPACE                  # too small
+    assert _fwd(L, ws=ctypes.c_void_p(0x100010), ws_bytes=1 << 40) == WORKSPACE   # misaligned
+
+
+def test_step_entry_points_reject_bad_arguments(L):
+    p = ctypes.c_void_p(0x100000)
+    assert L.spark_bsa_gather_q(None, 0, 1, 10, 128, p, p, 1, p, p, None, None) == INVALID
+    assert L.spark_bsa_gather_q(p, 0, 1, 10, 80, p, p, 1, p, p, None, None) == UNSUPPORTED
+    assert L.spark_bsa_anchor(p, p, 1, 10, 128, 0, p, None) == INVALID
+    assert L.spark_bsa_route(p, p, 1, 4, 4, 128, 5, p, None, None) == INVALID     # k > nkb
+    assert L.spark_bsa_route(p, p, 1, 4, 4, 128, 0, p, None, None) == INVALID
+    assert L.spark_bsa_route(p, p, 1, 4, 13000, 128, 5, p, None, None) == UNSUPPORTED
+    assert L.spark_bsa_attend(p, p, p, p, p, p, p, 0, p, p, 1, p, 1, 1, 10, 128, p, 0, None,
+                              None) == INVALID                                   # k = 0
+    assert L.spark_bsa_attend(p, p, p, p, p, p, p, 1, p, p, 1, p, 1, 1, 10, 128, p, 3, None,
+                              None) == INVALID                                   # out dtype
+    assert L.spark_bsa_gather_kv_summarize(p, p, 0, 1, 10, 128, p, p, 1, p, p, p, p, p, p,
+                                           None, None, None) == INVALID          # cbias NULL
+    flags = ctypes.c_uint32(0)
+    assert L.spark_bsa_read_error(None, None, ctypes.byref(flags)) == INVALID
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    code = ("import block_sparse_attention_gather_b200._native as n;"
+            f"n.LIB_PATH = {str(tmp_path / 'nope.so')!r};"
+            "n._LIB = None\n"
+            "try:\n    n.lib()\nexcept RuntimeError as e:\n    print('RAISED', 'no fallback' in str(e))")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
+    assert "RAISED True" in r.stdout, r.stderr

@@ -333,10 +333,54 @@ def pin_literal_copies():
     return err
 
 
+def pin_block_means():
+    """Block means: |B|-weighted means add up to the column sums of all rows, each mean lies
+    between the block's column minimum and maximum, and a constant block gives the constant."""
+    rng = np.random.default_rng(51)
+    X = rng.standard_normal((300, 6))
+    offs = random_offsets(rng, 300, 1, 40)
+    m = O.block_means(X, offs)
+    sizes = (offs[1:] - offs[:-1]).astype(np.float64)
+    err = float(np.abs((sizes[:, None] * m).sum(0) - X.sum(0)).max())
+    for B in range(len(offs) - 1):
+        blk = X[offs[B]:offs[B + 1]]
+        if not ((m[B] >= blk.min(0) - 1e-12).all() and (m[B] <= blk.max(0) + 1e-12).all()):
+            err = max(err, 1.0)
+    Xc = np.repeat(rng.standard_normal((len(offs) - 1, 6)), offs[1:] - offs[:-1], axis=0)
+    err = max(err, float(np.abs(O.block_means(Xc, offs) - Xc[offs[:-1]]).max()))
+    return err
+
+
+def pin_dense_reference():
+    """The oracle's dense attention (used by the GPU tests at ratio 1) against torch's
+    scaled-dot-product attention."""
+    rng = np.random.default_rng(52)
+    Q, K, V = (rng.standard_normal((70, 16)) for _ in range(3))
+    return float(np.abs(O.dense_attention(Q, K, V) - sdpa(Q, K, V)).max())
+
+
+def pin_diagnostics():
+    """Attention-mass recall is 1 when every block is selected; the log-mass error is 0 when
+    every key block holds identical keys (the summary row is then exact)."""
+    p = random_problem(53, H=1, N=90, d=8, lo=3, hi=12)
+    Qp = p["Q"][0][p["q_perm"][0]]
+    Kp = p["K"][0][p["k_perm"][0]]
+    offs = p["k_offsets"]
+    nkb = len(offs) - 1
+    err = abs(O.attention_mass_recall(Qp[:10], Kp, offs, np.arange(nkb)) - 1.0)
+    rng = np.random.default_rng(54)
+    for B in range(nkb):
+        Kp[offs[B]:offs[B + 1]] = rng.standard_normal(8)
+    kt, vt, c = O.summarize(Kp, Kp, offs, rng.standard_normal(8), 1 / math.sqrt(8))
+    err = max(err, O.log_mass_error(Qp[:10], Kp, offs, [0, 1], kt, c))
+    return err
+
+
 PINS = [pin_dense_at_ratio_one, pin_identical_keys_in_blocks, pin_identical_queries,
         pin_anchor_centred_query, pin_log_mass_identity, pin_golden_single_block,
         pin_golden_tiny_forward, pin_bruteforce_topk, pin_scores_are_block_mass_order,
-        pin_invariances, pin_literal_copies]
+        pin_invariances, pin_literal_copies, pin_block_means, pin_dense_reference,
+        pin_diagnostics]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -462,6 +506,14 @@ def _mut_transposed_scores(orig):
     return "route_scores", lambda qb, kb, scale: scale * (kb @ qb.T)
 
 
+def _mut_block_mean_off_by_one(orig):
+    def f(Xp, offsets):
+        offsets = np.asarray(offsets)
+        return np.stack([Xp[offsets[b]:max(offsets[b + 1] - 1, offsets[b] + 1)].mean(0)
+                         for b in range(len(offsets) - 1)])
+    return "block_means", f
+
+
 def _mut_lowest_scores(orig):
     def f(scores_A, k):
         return orig(-scores_A, k)
@@ -470,7 +522,7 @@ def _mut_lowest_scores(orig):
 
 MUTATIONS = [_mut_drop_log_size, _mut_uniform_weights, _mut_value_from_keys, _mut_sign_bias,
              _mut_anchor_half, _mut_no_scale, _mut_ties_to_larger, _mut_ignore_perm,
-             _mut_transposed_scores, _mut_lowest_scores]
+             _mut_transposed_scores, _mut_lowest_scores, _mut_block_mean_off_by_one]
 
 
 @pytest.mark.parametrize("mutation", MUTATIONS, ids=lambda f: f.__name__)
