@@ -19,7 +19,7 @@ __all__ = [
     "spark_status_string", "spark_bsa_topk_count", "spark_bsa_workspace_layout",
     "spark_bsa_workspace_size", "spark_bsa_forward", "spark_bsa_read_error",
     "spark_bsa_gather_q", "spark_bsa_anchor", "spark_bsa_gather_kv_summarize",
-    "spark_bsa_route", "spark_bsa_attend", "workspace_views",
+    "spark_bsa_route", "spark_bsa_attend", "workspace_views", "spark_bsa_forward_noalloc",
 ]
 
 SPARK_BF16, SPARK_F32 = 0, 1
@@ -28,7 +28,7 @@ EXPORTED = [
     "spark_status_string", "spark_bsa_topk_count", "spark_bsa_workspace_layout",
     "spark_bsa_workspace_size", "spark_bsa_forward", "spark_bsa_read_error",
     "spark_bsa_gather_q", "spark_bsa_anchor", "spark_bsa_gather_kv_summarize",
-    "spark_bsa_route", "spark_bsa_attend",
+    "spark_bsa_route", "spark_bsa_attend", "spark_bsa_forward_noalloc",
 ]
 
 
@@ -76,6 +76,8 @@ def lib():
         "spark_bsa_route": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
         "spark_bsa_attend": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _P, _I, _I, _I,
                                   _I, _P, _I, _P, _P]),
+        "spark_bsa_forward_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _I,
+                                           _D, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -294,4 +296,26 @@ def spark_bsa_attend(Qp, Kp, Vp, k_tilde, v_tilde, cbias, sel, q_perm, q_offsets
                                 _ptr(k_offsets), nkb, H, N, d, _ptr(out), _code(out_dtype),
                                 _ptr(err), _stream(stream))
     _check("spark_bsa_attend", st)
+    return out
+
+
+def spark_bsa_forward_noalloc(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, topk_ratio,
+                              out, stream=None):
+    """The forward pass with the library's static scratch array as its workspace (for callers
+    that cannot allocate device memory while they run); `out` must be preallocated.  Small
+    problems only: the workspace must fit SPARK_NOALLOC_SCRATCH_BYTES (16 MiB)."""
+    _need(Q, "Q", (torch.bfloat16, torch.float32))
+    dev = Q.device
+    H, N, d = Q.shape
+    for n, t in (("K", K), ("V", V), ("out", out)):
+        _need(t, n, Q.dtype, dev)
+    for n, t in (("q_perm", q_perm), ("k_perm", k_perm), ("q_offsets", q_offsets),
+                 ("k_offsets", k_offsets)):
+        _need(t, n, torch.int32, dev)
+    nqb, nkb = q_offsets.numel() - 1, k_offsets.numel() - 1
+    st = lib().spark_bsa_forward_noalloc(_ptr(Q), _ptr(K), _ptr(V), _code(Q.dtype), H, N, d,
+                                         _ptr(q_perm), _ptr(k_perm), _ptr(q_offsets), nqb,
+                                         _ptr(k_offsets), nkb, float(topk_ratio), _ptr(out),
+                                         _stream(stream))
+    _check("spark_bsa_forward_noalloc", st)
     return out

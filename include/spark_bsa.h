@@ -174,6 +174,32 @@ SPARK_API spark_status spark_bsa_attend(const void* Qp, const void* Kp, const vo
                               const int32_t* k_block_offsets, int nkb, int H, int N, int d,
                               void* out, int out_dtype, uint32_t* err, void* stream);
 
+/* ---- Forward pass without any allocation ----
+ * No counterpart in the pages: this entry point exists for callers that cannot allocate
+ * device memory while they run (a memory budget owned by a host framework, work recorded into
+ * a CUDA stream capture, a real-time path where an allocation may block or fail).  It is
+ * spark_bsa_forward with its workspace taken from a static device array of
+ * SPARK_NOALLOC_SCRATCH_BYTES bytes inside the library instead of from the caller; it calls no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *   - Problems whose spark_bsa_workspace_size exceeds SPARK_NOALLOC_SCRATCH_BYTES are rejected
+ *     with SPARK_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device (with that device current) resolves the array's device
+ *     address; make that first call before any stream capture.
+ *   - Every GPU on which this entry point is used holds the array until the process exits.
+ *   - All calls share the one array and it keeps the last call's contents; the call clears
+ *     the error word itself.  Calls that overlap on the GPU (two streams, or two host threads)
+ *     race on the array: serialise them.
+ *   - The device error word lives in the array and is not returned; bad device data is still
+ *     skipped by the kernels. */
+#define SPARK_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+SPARK_API spark_status spark_bsa_forward_noalloc(const void* Q, const void* K, const void* V,
+                                                 int dtype, int H, int N, int d,
+                                                 const int32_t* q_perm, const int32_t* k_perm,
+                                                 const int32_t* q_block_offsets, int nqb,
+                                                 const int32_t* k_block_offsets, int nkb,
+                                                 double topk_ratio, void* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
