@@ -103,11 +103,10 @@ spark_status attend_impl(const void* Qp, const void* Kp, const void* Vp, const v
                          const int32_t* k_offsets, int nkb, int H, int N, int d, void* out,
                          int out_dtype, uint32_t* err, cudaStream_t s) {
   AttendMaps maps;
-  if (!encode_rows_map(&maps.k, Kp, H, N, d) || !encode_rows_map(&maps.v, Vp, H, N, d) ||
-      !encode_rows_map(&maps.kt, k_tilde, H, nkb, d) ||
+  if (!encode_rows_map(&maps.q, Qp, H, N, d) || !encode_rows_map(&maps.k, Kp, H, N, d) ||
+      !encode_rows_map(&maps.v, Vp, H, N, d) || !encode_rows_map(&maps.kt, k_tilde, H, nkb, d) ||
       !encode_rows_map(&maps.vt, v_tilde, H, nkb, d))
     return SPARK_ERR_CUDA;
-  maps.q_base = Qp;
   return from_cuda(launch_attend(maps, cbias, sel, k, q_perm, q_offsets, nqb, k_offsets, nkb, H,
                                  N, d, out, out_dtype, err, s));
 }

@@ -25,11 +25,9 @@ cudaError_t launch_route(const float* qbar_blocks, const float* kbar, int H, int
                          int d, int k, int32_t* sel, uint32_t* err, cudaStream_t s);
 
 // Operands of the attention kernel: TMA descriptors (encoded on the host by api.cu) of the
-// reblocked K, V ([H,N,d] bf16) and of the summaries k~, v~ ([H,nkb,d] bf16), and the
-// reblocked queries, which the kernel reads with plain loads.
+// reblocked Q, K, V ([H,N,d] bf16) and of the summaries k~, v~ ([H,nkb,d] bf16).
 struct AttendMaps {
-  CUtensorMap k, v, kt, vt;
-  const void* q_base;
+  CUtensorMap q, k, v, kt, vt;
 };
 
 cudaError_t launch_attend(const AttendMaps& maps, const float* cbias, const int32_t* sel, int k,

@@ -69,6 +69,20 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same test, but a thread whose phase is not complete yet is suspended until it completes or
+// about `hint_ns` nanoseconds pass, instead of spinning on the barrier's shared-memory word.
+__device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // True once any CTA of the launch recorded a timeout in the error word.
 __device__ __forceinline__ bool launch_timed_out(const uint32_t* err) {
   return err != nullptr && (*reinterpret_cast<const volatile uint32_t*>(err) & kErrTimeout);
@@ -83,8 +97,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_test(bar, parity)) return true;
-    if ((it & 31u) == 0u) {
+    if (mbar_test_sleep(bar, parity, 200000u)) return true;   // sleeps at most ~0.2 ms
+    {
       if (*abort_flag) return false;
       if (launch_timed_out(err)) {
         *abort_flag = 1;
