@@ -456,7 +456,7 @@ def main():
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        per_call, threads, desc = oracle_sample(w, n_heads=2, n_units=64)
+        per_call, threads, desc = oracle_sample(w, n_heads=2, n_units=320)
         line["cpu_baseline"] = {"value": dflops / per_call / 1e12, "unit": UNIT,
                                 "cores": threads, "kind": "oracle", "sample": desc,
                                 "ms_per_call_extrapolated": per_call * 1e3}

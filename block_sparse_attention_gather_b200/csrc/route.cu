@@ -1,42 +1,57 @@
 // Block scoring + per-query-block Top-K (Spark-H3 blog, "Discussion": blocks are scored from
 // block-level means; "Spark-Reblock": a fixed Top-K budget of key blocks per query block).
 //
-// One CTA per (R consecutive query blocks, head), 256 threads:
+// One CTA per (R consecutive query blocks, head), 512 threads:
 //   phase 1  S[r, B] = qbar_A(r) . kbar_B in fp32 (sequential FMA over d) for every key
-//            block, staged through shared memory in 32-block tiles; the scores of the R
-//            rows stay in shared memory.  The positive factor 1/sqrt(d) is left out: it does
-//            not change the order.
-//   phase 2  one warp per row: an exact radix select (four 8-bit passes over the
-//            order-preserving uint32 image of the fp32 score) finds the k-th largest key T
-//            and how many keys equal to T are still needed; a ballot scan in ascending block
-//            order then writes every B with key > T and the lowest-indexed keys == T, so the
-//            selection is stored ascending and ties go to the smaller block index.
+//            block.  A thread owns two key blocks at a time: their kbar rows stream through
+//            its registers in 8-element chunks straight from global memory (L2-resident:
+//            every CTA of the head reads them), the next chunk in flight while the current
+//            one is used, and the R query rows come from shared memory stored d-major, so
+//            each load is a warp-wide broadcast of four rows.  The scores of the R
+//            rows stay in shared memory as order-preserving uint32 keys.  The positive factor
+//            1/sqrt(d) is left out: it does not change the order.
+//   phase 2  one warp per row: an exact radix select (four 8-bit passes over the keys) finds
+//            the k-th largest key T and how many keys equal to T are still needed; a ballot
+//            scan in ascending block order then writes every B with key > T and the
+//            lowest-indexed keys == T, so the selection is stored ascending and ties go to
+//            the smaller block index.
 #include "spark_kernels.cuh"
 
 namespace spark {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kTileCols = 32;
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kCols = 2;          // key blocks a thread scores at once
+constexpr int kChunk = 8;         // d-elements of each kbar_B held in registers at a time
+constexpr bool kPrefetch = true;  // load the next chunk while the current one is in use
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+__device__ __forceinline__ float4 ld_nc_f4(const float4* p) {
+  float4 v;
+  asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
+
 }  // namespace
 
 template <int D, int R>
-__global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict__ qbar_blocks,
-                                                         const float* __restrict__ kbar, int nqb,
-                                                         int nkb, int k,
-                                                         int32_t* __restrict__ sel) {
+__global__ void __launch_bounds__(kThreads, 1) route_kernel(const float* __restrict__ qbar_blocks,
+                                                            const float* __restrict__ kbar,
+                                                            int nqb, int nkb, int k,
+                                                            int32_t* __restrict__ sel) {
+  static_assert(R % 4 == 0 && D % kChunk == 0, "tile shape");
   extern __shared__ __align__(16) float sm[];
-  float* scores = sm;                                   // [R][nkb]
-  float* qrows = scores + static_cast<size_t>(R) * nkb; // [R][D]
-  float* ktile = qrows + R * D;                         // [kTileCols][D + 1]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(ktile + kTileCols * (D + 1));  // [8][256]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sm);     // [R][nkb]
+  float* qT = sm + static_cast<size_t>(R) * nkb;        // [D][R]  (R*nkb*4 is 16-byte aligned)
+  uint32_t* hist = reinterpret_cast<uint32_t*>(qT + D * R);  // [kWarps][256]
 
   const int h = blockIdx.y;
   const int A0 = blockIdx.x * R;
@@ -44,56 +59,80 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
 
   for (int i = tid; i < R * D; i += kThreads) {
-    const int r = i / D;
-    qrows[i] = (r < rows) ? qbar_blocks[(static_cast<size_t>(h) * nqb + A0 + r) * D + i % D] : 0.f;
+    const int r = i / D, e = i % D;
+    qT[e * R + r] = (r < rows) ? qbar_blocks[(static_cast<size_t>(h) * nqb + A0 + r) * D + e] : 0.f;
   }
+  __syncthreads();
 
-  // ---- phase 1: scores
-  constexpr int OUT_PER_THREAD = (R * kTileCols) / kThreads;   // 2 (R=16), 1 (R=8)
-  constexpr int RSTEP = kThreads / kTileCols;                  // 8 rows per pass
-  const float* kb = kbar + static_cast<size_t>(h) * nkb * D;
-  for (int B0 = 0; B0 < nkb; B0 += kTileCols) {
-    __syncthreads();
-    for (int i = tid; i < kTileCols * D; i += kThreads) {
-      const int cb = i / D, e = i % D;
-      ktile[cb * (D + 1) + e] = (B0 + cb < nkb) ? kb[static_cast<size_t>(B0 + cb) * D + e] : 0.f;
+  // ---- phase 1: scores (no collectives inside: the ragged last pass needs no uniformity)
+  const float4* kb4 = reinterpret_cast<const float4*>(kbar + static_cast<size_t>(h) * nkb * D);
+  for (int B0 = tid; B0 < nkb; B0 += kCols * kThreads) {
+    float acc[kCols][R];
+    const float4* src[kCols];
+    bool live[kCols];
+#pragma unroll
+    for (int c = 0; c < kCols; ++c) {
+      live[c] = B0 + c * kThreads < nkb;
+      src[c] = kb4 + static_cast<size_t>(live[c] ? B0 + c * kThreads : B0) * (D / 4);
+#pragma unroll
+      for (int r = 0; r < R; ++r) acc[c][r] = 0.f;
     }
-    __syncthreads();
-    const int col = tid % kTileCols;
-    const int r0 = tid / kTileCols;
-    if (B0 + col < nkb) {
-      if constexpr (OUT_PER_THREAD >= 1) {
-        float acc[OUT_PER_THREAD > 0 ? OUT_PER_THREAD : 1];
+    float4 b[kCols][kChunk / 4];
 #pragma unroll
-        for (int o = 0; o < OUT_PER_THREAD; ++o) acc[o] = 0.f;
-        const float* kr = ktile + col * (D + 1);
-#pragma unroll 8
-        for (int e = 0; e < D; ++e) {
-          const float kv = kr[e];
+    for (int c = 0; c < kCols; ++c)
 #pragma unroll
-          for (int o = 0; o < OUT_PER_THREAD; ++o) acc[o] = fmaf(qrows[(r0 + o * RSTEP) * D + e], kv, acc[o]);
-        }
+      for (int j = 0; j < kChunk / 4; ++j) b[c][j] = ld_nc_f4(src[c] + j);
+#pragma unroll 1
+    for (int e0 = 0; e0 < D; e0 += kChunk) {
+      float4 nb[kCols][kChunk / 4];
+      if (kPrefetch && e0 + kChunk < D) {
 #pragma unroll
-        for (int o = 0; o < OUT_PER_THREAD; ++o)
-          scores[static_cast<size_t>(r0 + o * RSTEP) * nkb + B0 + col] = acc[o];
-      } else {
-        if (r0 < R) {
-          float acc = 0.f;
-          const float* kr = ktile + col * (D + 1);
-#pragma unroll 8
-          for (int e = 0; e < D; ++e) acc = fmaf(qrows[r0 * D + e], kr[e], acc);
-          scores[static_cast<size_t>(r0) * nkb + B0 + col] = acc;
+        for (int c = 0; c < kCols; ++c)
+#pragma unroll
+          for (int j = 0; j < kChunk / 4; ++j) nb[c][j] = ld_nc_f4(src[c] + (e0 + kChunk) / 4 + j);
+      }
+#pragma unroll
+      for (int j = 0; j < kChunk / 4; ++j) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4* a = reinterpret_cast<const float4*>(qT + (e0 + 4 * j + q) * R);
+#pragma unroll
+          for (int r4 = 0; r4 < R / 4; ++r4) {
+            const float4 av = a[r4];
+#pragma unroll
+            for (int c = 0; c < kCols; ++c) {
+              const float bv = q == 0 ? b[c][j].x : q == 1 ? b[c][j].y : q == 2 ? b[c][j].z : b[c][j].w;
+              acc[c][4 * r4 + 0] = fmaf(av.x, bv, acc[c][4 * r4 + 0]);
+              acc[c][4 * r4 + 1] = fmaf(av.y, bv, acc[c][4 * r4 + 1]);
+              acc[c][4 * r4 + 2] = fmaf(av.z, bv, acc[c][4 * r4 + 2]);
+              acc[c][4 * r4 + 3] = fmaf(av.w, bv, acc[c][4 * r4 + 3]);
+            }
+          }
         }
       }
+      if (e0 + kChunk < D) {
+#pragma unroll
+        for (int c = 0; c < kCols; ++c)
+#pragma unroll
+          for (int j = 0; j < kChunk / 4; ++j)
+            b[c][j] = kPrefetch ? nb[c][j] : ld_nc_f4(src[c] + (e0 + kChunk) / 4 + j);
+      }
     }
+#pragma unroll
+    for (int c = 0; c < kCols; ++c)
+      if (live[c]) {
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          keys[static_cast<size_t>(r) * nkb + B0 + c * kThreads] = order_key(acc[c][r]);
+      }
   }
   __syncthreads();
 
   // ---- phase 2: exact Top-K per row, one warp per row
   uint32_t* wh = hist + warp * 256;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int r = warp; r < rows; r += kThreads / 32) {
-    const float* srow = scores + static_cast<size_t>(r) * nkb;
+  for (int r = warp; r < rows; r += kWarps) {
+    const uint32_t* krow = keys + static_cast<size_t>(r) * nkb;
     int32_t* out = sel + (static_cast<size_t>(h) * nqb + A0 + r) * k;
     uint32_t prefix = 0, pmask = 0;
     int need = k;                      // still to take among keys matching `prefix`
@@ -102,7 +141,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
         for (int i = lane; i < 256; i += 32) wh[i] = 0;
         __syncwarp();
         for (int B = lane; B < nkb; B += 32) {
-          const uint32_t u = order_key(srow[B]);
+          const uint32_t u = krow[B];
           if ((u & pmask) == prefix) atomicAdd(&wh[(u >> shift) & 255u], 1u);
         }
         __syncwarp();
@@ -147,7 +186,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
     int taken = 0, eq_seen = 0;
     for (int B0 = 0; B0 < nkb; B0 += 32) {
       const int B = B0 + lane;
-      const uint32_t u = (B < nkb) ? order_key(srow[B]) : 0u;
+      const uint32_t u = (B < nkb) ? krow[B] : 0u;
       const bool valid = B < nkb;
       const bool gt = valid && (k == nkb || u > T);
       const bool eq = valid && k < nkb && u == T;
@@ -164,7 +203,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
 
 template <int D, int R>
 constexpr size_t route_smem_bytes(int nkb) {
-  return (static_cast<size_t>(R) * nkb + R * D + kTileCols * (D + 1)) * 4 + 8 * 256 * 4;
+  return (static_cast<size_t>(R) * nkb + R * D) * 4 + kWarps * 256 * 4;
 }
 
 constexpr size_t kRouteSmemLimit = 232448;   // 227 KB of opt-in shared memory per CTA
