@@ -21,6 +21,11 @@ Layouts (the reblocked partition is an input of the method):
 Block offsets are shared by all heads: fixed-size blocks whose last block takes the
 remainder, or sizes drawn uniformly in [lo, hi] until they cover N (the last block takes the
 remainder).
+
+Context (sink) tokens, when a workload has ``nc > 0``: Kc, Vc [H, nc, d] drawn after
+everything else from a generator of their own (so the video tensors do not change), keys
+from the same mixture as the video keys, values N(0, 1).  The pages give no context length;
+512 stands in for a text prompt's tokens.
 """
 
 from __future__ import annotations
@@ -47,6 +52,7 @@ class Workload:
     var_block: tuple | None = None   # (lo, hi) for variable block sizes
     n_components: int = 32
     spread: float = 0.3
+    nc: int = 0                # context (sink) tokens per head
 
     def with_ratio(self, ratio: float) -> "Workload":
         return replace(self, ratio=ratio, name=f"{self.name.rsplit('-r', 1)[0]}-r{ratio:g}")
@@ -67,6 +73,12 @@ WORKLOADS: dict[str, Workload] = {w.name: w for w in [
     Workload("768p-24x241920-d128-randperm", 24, 241920, 128, "bf16", 0.1, "random",
              "mixture", 1004),
     _mk_var(0.1), _mk_var(0.2), _mk_var(0.3), _mk_var(1.0),
+    Workload("tiny-ctx77-1x1024-d64-fp32", 1, 1024, 64, "fp32", 0.125, "identity", "iid",
+             1006, block=64, nc=77),
+    Workload("small-ctx300-8x16384-d128-randperm", 8, 16384, 128, "bf16", 0.1, "random",
+             "mixture", 1007, block=64, nc=300),
+    Workload("768p-ctx512-24x241920-d128", 24, 241920, 128, "bf16", 0.1, "reblock", "mixture",
+             1008, nc=512),
 ]}
 
 
@@ -100,7 +112,6 @@ def make_inputs(w: Workload, device="cpu") -> dict:
         hidx = torch.arange(H, device=device)[:, None]
         Q = (mu[hidx, comp] + w.spread * torch.randn(H, N, d, generator=g, device=device)).to(tdt)
         K = (mu[hidx, comp] + w.spread * torch.randn(H, N, d, generator=g, device=device)).to(tdt)
-        del mu
     else:
         raise ValueError(w.structure)
     V = torch.randn(H, N, d, generator=g, device=device).to(tdt)
@@ -126,9 +137,21 @@ def make_inputs(w: Workload, device="cpu") -> dict:
         raise ValueError(w.layout)
 
     offs = make_offsets(w).to(device)
-    return dict(Q=Q.contiguous(), K=K.contiguous(), V=V.contiguous(),
-                q_perm=q_perm.contiguous(), k_perm=k_perm.contiguous(),
-                q_offsets=offs, k_offsets=offs.clone(), ratio=w.ratio)
+    x = dict(Q=Q.contiguous(), K=K.contiguous(), V=V.contiguous(),
+             q_perm=q_perm.contiguous(), k_perm=k_perm.contiguous(),
+             q_offsets=offs, k_offsets=offs.clone(), ratio=w.ratio)
+    if w.nc > 0:
+        gc = torch.Generator(device=device).manual_seed(w.seed * 104729 + 11)
+        if w.structure == "mixture":
+            cc = torch.randint(0, w.n_components, (H, w.nc), generator=gc, device=device)
+            Kc = mu[torch.arange(H, device=device)[:, None], cc] + \
+                w.spread * torch.randn(H, w.nc, d, generator=gc, device=device)
+        else:
+            Kc = torch.randn(H, w.nc, d, generator=gc, device=device)
+        Vc = torch.randn(H, w.nc, d, generator=gc, device=device)
+        x["Kc"] = Kc.to(tdt).contiguous()
+        x["Vc"] = Vc.to(tdt).contiguous()
+    return x
 
 
 def sample_units(w: Workload, n_units: int, nqb: int, seed_offset: int = 0):

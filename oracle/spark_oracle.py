@@ -24,6 +24,8 @@ extension page "Spark-H3 (comfy.icu)", and the comfyui-wiki news article on Spar
   log-mass bias chosen so that the exponential of the effective logit equals the expected
   exponential E[exp(x)] instead of exp(E[x]); routing is unchanged.
 * comfyui-wiki news article, bullet on Spark-Reweight: one anchor (the query mean) per head.
+* Spark-H3 blog, section "Spark-Reblock", after the BSA equations: context (sink) tokens are
+  always attended exactly and do not count against the Top-K budget of video blocks.
 
 Readings taken where the pages leave a step open (each is also listed in the design notes):
 
@@ -34,10 +36,14 @@ R3  anchor: the mean over all N queries of the head.
 R4  routing score: S[A,B] = q_bar_A . k_bar_B / sqrt(d) with uniform block means.
 R5  k = clamp(ceil(ratio * nKB - 1e-9), 1, nKB).
 R6  ties in Top-K: the smaller block index wins; S_A is reported in ascending order.
-R7  no causal mask, no forced diagonal block, no sink tokens.
+R7  no causal mask and no forced diagonal block; sink tokens only as the context segment (R15).
 R8  each key block is either exact or compressed, never both.
 R9  the output row of reblocked position i is written back to original token q_perm[i].
 R10 permutations are per head; block offsets are shared by all heads.
+R15 context tokens (optional, Kc/Vc [nc, d] per head): every video query attends to all of
+    them exactly, inside the same row-wise softmax as both branches.  They form no block, take
+    no part in the anchor, the block means, the summaries or the routing, and k is still
+    taken over the nKB video blocks.  Context queries are not part of this operation.
 
 Parity: every function here is pinned by the CPU tests (dense attention at ratio 1, blocks of
 identical keys, identical queries, an anchor-centred query, the log-mass identity, hand
@@ -194,12 +200,14 @@ def route(qbar_blocks: np.ndarray, kbar: np.ndarray, scale: float, k: int):
 
 def attend_block(Qp_A: np.ndarray, Kp: np.ndarray, Vp: np.ndarray, k_offsets: np.ndarray,
                  sel_A: np.ndarray, k_tilde: np.ndarray, v_tilde: np.ndarray, c: np.ndarray,
-                 scale: float) -> np.ndarray:
+                 scale: float, Kc: np.ndarray | None = None,
+                 Vc: np.ndarray | None = None) -> np.ndarray:
     """Two-branch attention of one query block (Spark-H3 blog, BSA equations; R8).
 
     The exact branch holds every key row of the selected blocks; the compressed branch holds
-    one summary row per unselected block whose logit carries the offset c_B.  A single
-    row-wise softmax normalises the union.
+    one summary row per unselected block whose logit carries the offset c_B.  Context rows
+    Kc/Vc, when given, are exact keys outside the Top-K budget (R15).  A single row-wise
+    softmax normalises the union.
     """
     k_offsets = np.asarray(k_offsets, dtype=np.int64)
     nkb = len(k_offsets) - 1
@@ -214,6 +222,9 @@ def attend_block(Qp_A: np.ndarray, Kp: np.ndarray, Vp: np.ndarray, k_offsets: np
     if comp.size:
         logits.append(scale * (Qp_A @ k_tilde[comp].T) + c[comp][None, :])
         values.append(v_tilde[comp])
+    if Kc is not None and len(Kc):
+        logits.append(scale * (Qp_A @ np.asarray(Kc, dtype=np.float64).T))
+        values.append(np.asarray(Vc, dtype=np.float64))
     L = np.concatenate(logits, axis=1)
     Vcat = np.concatenate(values, axis=0)
     L = L - L.max(axis=1, keepdims=True)
@@ -237,13 +248,14 @@ class HeadResult:
 
 
 def forward_head(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, ratio, *, mode="reweight",
-                 sel=None, blocks=None) -> HeadResult:
+                 sel=None, blocks=None, Kc=None, Vc=None) -> HeadResult:
     """One head of the forward pass, steps in the pages' order.
 
     ``sel`` (optional [nQB,k]) replaces the routing result, e.g. with another implementation's
     selection when several selections are correct at a near-tie.  ``blocks`` (optional
     iterable of query-block ids) restricts the attention step to those blocks; summaries and
-    routing are always computed for the whole head.
+    routing are always computed for the whole head.  ``Kc``, ``Vc`` (optional [nc, d]) are the
+    head's context tokens (R15).
     """
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
@@ -253,6 +265,13 @@ def forward_head(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, ratio, *, mode="
     q_offsets = np.asarray(q_offsets, dtype=np.int64)
     k_offsets = np.asarray(k_offsets, dtype=np.int64)
     N, d = Q.shape
+    if (Kc is None) != (Vc is None):
+        raise ValueError("Kc and Vc go together")
+    if Kc is not None:
+        Kc = np.asarray(Kc, dtype=np.float64).reshape(-1, d)
+        Vc = np.asarray(Vc, dtype=np.float64).reshape(-1, d)
+        if Kc.shape != Vc.shape:
+            raise ValueError("Kc and Vc must have the same shape")
     scale = 1.0 / math.sqrt(d)
     nqb = len(q_offsets) - 1
     nkb = len(k_offsets) - 1
@@ -287,14 +306,15 @@ def forward_head(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, ratio, *, mode="
     todo = range(nqb) if blocks is None else blocks
     for A in todo:
         lo, hi = q_offsets[A], q_offsets[A + 1]
-        o = attend_block(Qp[lo:hi], Kp, Vp, k_offsets, sel[A], kt, vt, c, scale)
+        o = attend_block(Qp[lo:hi], Kp, Vp, k_offsets, sel[A], kt, vt, c, scale, Kc=Kc, Vc=Vc)
         out[q_perm[lo:hi]] = o
     return HeadResult(out, qbar, qbar_blocks, kbar, kt, vt, c, sel, S)
 
 
 def forward(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, ratio, *, mode="reweight",
-            sel=None, blocks=None):
-    """All heads: Q,K,V [H,N,d]; perms [H,N]; offsets shared.  Returns a list of HeadResult.
+            sel=None, blocks=None, Kc=None, Vc=None):
+    """All heads: Q,K,V [H,N,d]; perms [H,N]; offsets shared; optional context Kc,Vc
+    [H,nc,d].  Returns a list of HeadResult.
 
     ``blocks`` may be a dict head -> iterable of query blocks (heads absent are skipped for
     the attention step) or None for every block of every head.
@@ -308,7 +328,8 @@ def forward(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, ratio, *, mode="rewei
             bl = blocks
         res.append(forward_head(Q[h], K[h], V[h], q_perm[h], k_perm[h], q_offsets, k_offsets,
                                 ratio, mode=mode, sel=None if sel is None else sel[h],
-                                blocks=bl))
+                                blocks=bl, Kc=None if Kc is None else Kc[h],
+                                Vc=None if Vc is None else Vc[h]))
     return res
 
 

@@ -376,11 +376,73 @@ def pin_diagnostics():
     return err
 
 
+def _with_context(p, seed, nc):
+    rng = np.random.default_rng(seed)
+    H, _, d = p["Q"].shape
+    p["Kc"] = rng.standard_normal((H, nc, d)) * 1.5
+    p["Vc"] = rng.standard_normal((H, nc, d))
+    return p
+
+
+def pin_context_dense_at_ratio_one():
+    """Context tokens (Spark-H3 blog, "Spark-Reblock": context/sink tokens stay exact, outside
+    the Top-K budget): at topk_ratio = 1 the result is dense attention over the video keys
+    followed by the context keys, in one softmax."""
+    err = 0.0
+    for seed, nc in ((81, 1), (82, 13), (83, 40)):
+        p = _with_context(random_problem(seed), seed + 1, nc)
+        res = run(p, 1.0, Kc=p["Kc"], Vc=p["Vc"])
+        for h, r in enumerate(res):
+            ref = sdpa(p["Q"][h], np.concatenate([p["K"][h], p["Kc"][h]]),
+                       np.concatenate([p["V"][h], p["Vc"][h]]))
+            err = max(err, float(np.abs(r.out - ref).max()))
+    return err
+
+
+def pin_context_identical_keys():
+    """Context tokens with exact summaries (keys constant inside every video block, as in P2):
+    the result is dense over video + context keys at any ratio."""
+    err = 0.0
+    for seed, ratio, nc in ((84, 0.1, 7), (85, 0.3, 21)):
+        p = _with_context(random_problem(seed, N=120, lo=3, hi=20), seed + 1, nc)
+        rng = np.random.default_rng(seed + 100)
+        for h in range(p["Q"].shape[0]):
+            Kp = np.empty((p["Q"].shape[1], p["Q"].shape[2]))
+            for B in range(len(p["k_offsets"]) - 1):
+                Kp[p["k_offsets"][B]:p["k_offsets"][B + 1]] = rng.standard_normal(Kp.shape[1])
+            p["K"][h] = scatter_reblocked(Kp, p["k_perm"][h])
+        res = run(p, ratio, Kc=p["Kc"], Vc=p["Vc"])
+        for h, r in enumerate(res):
+            ref = sdpa(p["Q"][h], np.concatenate([p["K"][h], p["Kc"][h]]),
+                       np.concatenate([p["V"][h], p["Vc"][h]]))
+            err = max(err, float(np.abs(r.out - ref).max()))
+    return err
+
+
+def pin_context_outside_budget():
+    """Context tokens change neither the routing nor the summaries (outside the Top-K budget,
+    no part in the anchor), and an empty context is no context."""
+    p = random_problem(86, N=150, lo=4, hi=24)
+    base = run(p, 0.2)
+    q = _with_context(dict(p), 87, 9)
+    withc = run(q, 0.2, Kc=q["Kc"], Vc=q["Vc"])
+    empty = run(p, 0.2, Kc=np.zeros((2, 0, 8)), Vc=np.zeros((2, 0, 8)))
+    err = 0.0
+    for a, b, e in zip(base, withc, empty):
+        if not np.array_equal(a.sel, b.sel):
+            return float("inf")
+        err = max(err, float(np.abs(a.k_tilde - b.k_tilde).max()),
+                  float(np.abs(a.c - b.c).max()), float(np.abs(a.qbar - b.qbar).max()),
+                  float(np.abs(a.out - e.out).max()))
+    return err
+
+
 PINS = [pin_dense_at_ratio_one, pin_identical_keys_in_blocks, pin_identical_queries,
         pin_anchor_centred_query, pin_log_mass_identity, pin_golden_single_block,
         pin_golden_tiny_forward, pin_bruteforce_topk, pin_scores_are_block_mass_order,
         pin_invariances, pin_literal_copies, pin_block_means, pin_dense_reference,
-        pin_diagnostics]
+        pin_diagnostics, pin_context_dense_at_ratio_one, pin_context_identical_keys,
+        pin_context_outside_budget]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -486,8 +548,33 @@ def _mut_anchor_half(orig):
 
 
 def _mut_no_scale(orig):
-    def f(Qp_A, Kp, Vp, k_offsets, sel_A, kt, vt, c, scale):
-        return orig(Qp_A, Kp, Vp, k_offsets, sel_A, kt, vt, c, 1.0)
+    def f(Qp_A, Kp, Vp, k_offsets, sel_A, kt, vt, c, scale, **kw):
+        return orig(Qp_A, Kp, Vp, k_offsets, sel_A, kt, vt, c, 1.0, **kw)
+    return "attend_block", f
+
+
+def _mut_context_own_softmax(orig):
+    # context normalised by a softmax of its own and averaged in, instead of sharing the row
+    def f(Qp_A, Kp, Vp, k_offsets, sel_A, kt, vt, c, scale, Kc=None, Vc=None):
+        o = orig(Qp_A, Kp, Vp, k_offsets, sel_A, kt, vt, c, scale)
+        if Kc is None or not len(Kc):
+            return o
+        L = scale * (Qp_A @ Kc.T)
+        P = np.exp(L - L.max(1, keepdims=True))
+        return 0.5 * o + 0.5 * (P / P.sum(1, keepdims=True)) @ Vc
+    return "attend_block", f
+
+
+def _mut_context_unscaled(orig):
+    def f(Qp_A, Kp, Vp, k_offsets, sel_A, kt, vt, c, scale, Kc=None, Vc=None):
+        return orig(Qp_A, Kp, Vp, k_offsets, sel_A, kt, vt, c, scale,
+                    Kc=None if Kc is None else Kc / scale, Vc=Vc)
+    return "attend_block", f
+
+
+def _mut_context_values_from_keys(orig):
+    def f(Qp_A, Kp, Vp, k_offsets, sel_A, kt, vt, c, scale, Kc=None, Vc=None):
+        return orig(Qp_A, Kp, Vp, k_offsets, sel_A, kt, vt, c, scale, Kc=Kc, Vc=Kc)
     return "attend_block", f
 
 
@@ -522,7 +609,8 @@ def _mut_lowest_scores(orig):
 
 MUTATIONS = [_mut_drop_log_size, _mut_uniform_weights, _mut_value_from_keys, _mut_sign_bias,
              _mut_anchor_half, _mut_no_scale, _mut_ties_to_larger, _mut_ignore_perm,
-             _mut_transposed_scores, _mut_lowest_scores, _mut_block_mean_off_by_one]
+             _mut_transposed_scores, _mut_lowest_scores, _mut_block_mean_off_by_one,
+             _mut_context_own_softmax, _mut_context_unscaled, _mut_context_values_from_keys]
 
 
 @pytest.mark.parametrize("mutation", MUTATIONS, ids=lambda f: f.__name__)
