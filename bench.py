@@ -134,7 +134,16 @@ class HotPath:
         self.ratio = ratio
         self.layout = spark_bsa_workspace_layout(self.H, self.N, self.d, self.nqb, self.nkb, ratio)
         self.k = self.layout.k
-        self.ws = torch.empty(self.layout.total, dtype=torch.uint8, device=device)
+        # context (sink) tokens: bf16 rows are read in place, fp32 rows converted each step
+        self.nc = x["Kc"].shape[1] if x.get("Kc") is not None else 0
+        from block_sparse_attention_gather_b200 import spark_bsa_workspace_size_ctx
+        size = spark_bsa_workspace_size_ctx(self.H, self.N, self.d, self.nqb, self.nkb, ratio,
+                                            self.nc)
+        self.ws = torch.empty(size, dtype=torch.uint8, device=device)
+        self.convert_ctx = self.nc > 0 and Q.dtype != torch.bfloat16
+        if self.convert_ctx:
+            self.Kcb = torch.empty(self.H, self.nc, self.d, dtype=torch.bfloat16, device=device)
+            self.Vcb = torch.empty_like(self.Kcb)
         self.v = workspace_views(self.ws, self.layout, self.H, self.N, self.d, self.nqb, self.nkb)
         self.out = torch.empty_like(Q)
         self.dtype_code = 0 if Q.dtype == torch.bfloat16 else 1
@@ -167,10 +176,22 @@ class HotPath:
         st |= L.spark_bsa_route(p(v["qbar_blocks"]), p(v["kbar"]), H, nqb, nkb, d, k,
                                 p(v["sel"]), err, s)
         rec(4)
-        st |= L.spark_bsa_attend(p(v["Qp"]), p(v["Kp"]), p(v["Vp"]), p(v["k_tilde"]),
-                                 p(v["v_tilde"]), p(v["cbias"]), p(v["sel"]), k,
-                                 p(x["q_perm"]), p(x["q_offsets"]), nqb, p(x["k_offsets"]), nkb,
-                                 H, N, d, p(self.out), self.dtype_code, err, s)
+        if self.nc == 0:
+            st |= L.spark_bsa_attend(p(v["Qp"]), p(v["Kp"]), p(v["Vp"]), p(v["k_tilde"]),
+                                     p(v["v_tilde"]), p(v["cbias"]), p(v["sel"]), k,
+                                     p(x["q_perm"]), p(x["q_offsets"]), nqb, p(x["k_offsets"]),
+                                     nkb, H, N, d, p(self.out), self.dtype_code, err, s)
+        else:
+            Kc, Vc = x["Kc"], x["Vc"]
+            if self.convert_ctx:
+                st |= L.spark_bsa_context_bf16(p(Kc), p(Vc), self.dtype_code, H, self.nc, d,
+                                               p(self.Kcb), p(self.Vcb), s)
+                Kc, Vc = self.Kcb, self.Vcb
+            st |= L.spark_bsa_attend_ctx(p(v["Qp"]), p(v["Kp"]), p(v["Vp"]), p(v["k_tilde"]),
+                                         p(v["v_tilde"]), p(v["cbias"]), p(v["sel"]), k, p(Kc),
+                                         p(Vc), self.nc, p(x["q_perm"]), p(x["q_offsets"]),
+                                         nqb, p(x["k_offsets"]), nkb, H, N, d, p(self.out),
+                                         self.dtype_code, err, s)
         rec(5)
         if st != 0:
             raise RuntimeError(f"a step entry point failed (status bits {st})")
@@ -178,14 +199,14 @@ class HotPath:
 
 def attention_flops(hp):
     """Algorithmic tensor-core FLOPs of one attention launch, from the selection it used:
-    4 d sum_{h,A} |A| (sum_{B in S_A} |B| + (nkb - k))."""
+    4 d sum_{h,A} |A| (sum_{B in S_A} |B| + nc + (nkb - k)), nc = context tokens."""
     qo = hp.x["q_offsets"].long()
     ko = hp.x["k_offsets"].long()
     qs = (qo[1:] - qo[:-1]).double()                    # [nqb]
     ks = (ko[1:] - ko[:-1]).double()                    # [nkb]
     sel = hp.v["sel"].long()                            # [H,nqb,k]
     exact = ks[sel].sum(-1)                             # [H,nqb]
-    cols = exact + (hp.nkb - hp.k)
+    cols = exact + hp.nc + (hp.nkb - hp.k)
     return float(4.0 * hp.d * (cols * qs[None, :]).sum().item())
 
 
@@ -250,8 +271,10 @@ def oracle_sample(w, n_heads=1, n_units=16, seed=0):
         Q, K, V = f64(x["Q"][h]), f64(x["K"][h]), f64(x["V"][h])
         qp = x["q_perm"][h].numpy().astype(np.int64)
         kp = x["k_perm"][h].numpy().astype(np.int64)
+        Kc = f64(x["Kc"][h]) if x.get("Kc") is not None else None
+        Vc = f64(x["Vc"][h]) if x.get("Vc") is not None else None
         t0 = time.perf_counter()
-        r = O.forward_head(Q, K, V, qp, kp, qo, ko, w.ratio, blocks=[])
+        r = O.forward_head(Q, K, V, qp, kp, qo, ko, w.ratio, blocks=[], Kc=Kc, Vc=Vc)
         t_prep += time.perf_counter() - t0
         blocks = rng.choice(nqb, size=n_units // n_heads, replace=False)
         Qp, Kp, Vp = Q[qp], K[kp], V[kp]
@@ -259,7 +282,7 @@ def oracle_sample(w, n_heads=1, n_units=16, seed=0):
         t0 = time.perf_counter()
         for A in blocks:
             O.attend_block(Qp[qo[A]:qo[A + 1]], Kp, Vp, ko, r.sel[A], r.k_tilde, r.v_tilde,
-                           r.c, scale)
+                           r.c, scale, Kc=Kc, Vc=Vc)
         t_att += time.perf_counter() - t0
         n_att += len(blocks)
     per_call = (t_prep / n_heads) * w.H + (t_att / n_att) * w.H * nqb
@@ -271,7 +294,9 @@ def oracle_sample(w, n_heads=1, n_units=16, seed=0):
 
 
 def dense_flops(w):
-    return 4.0 * w.H * float(w.N) ** 2 * w.d
+    """Dense-equivalent FLOPs of one call: every video query against every video and context
+    key, 4 H N (N + nc) d."""
+    return 4.0 * w.H * float(w.N) * float(w.N + w.nc) * w.d
 
 
 # --------------------------------------------------------------------------------- main
@@ -395,9 +420,11 @@ def main():
     # ---- end to end through the public call with host buffers (pinned), copies timed
     e2e = None
     if args.e2e_steps > 0:
-        from block_sparse_attention_gather_b200 import spark_bsa_forward
-        host = {n: x[n].to("cpu").pin_memory() for n in
-                ("Q", "K", "V", "q_perm", "k_perm", "q_offsets", "k_offsets")}
+        from block_sparse_attention_gather_b200 import spark_bsa_forward, spark_bsa_forward_ctx
+        names = ["Q", "K", "V", "q_perm", "k_perm", "q_offsets", "k_offsets"]
+        if hp.nc:
+            names += ["Kc", "Vc"]
+        host = {n: x[n].to("cpu").pin_memory() for n in names}
         dev_in = {n: torch.empty_like(x[n]) for n in host}
         out_host = torch.empty(hp.out.shape, dtype=hp.out.dtype).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in host.values())
@@ -407,10 +434,17 @@ def main():
         def e2e_step():
             for n in host:
                 dev_in[n].copy_(host[n], non_blocking=True)
-            o, _, _ = spark_bsa_forward(dev_in["Q"], dev_in["K"], dev_in["V"], dev_in["q_perm"],
-                                        dev_in["k_perm"], dev_in["q_offsets"],
-                                        dev_in["k_offsets"], w.ratio, out=hp.out,
-                                        workspace=hp.ws)
+            if hp.nc:
+                o, _, _ = spark_bsa_forward_ctx(dev_in["Q"], dev_in["K"], dev_in["V"],
+                                                dev_in["Kc"], dev_in["Vc"], dev_in["q_perm"],
+                                                dev_in["k_perm"], dev_in["q_offsets"],
+                                                dev_in["k_offsets"], w.ratio, out=hp.out,
+                                                workspace=hp.ws)
+            else:
+                o, _, _ = spark_bsa_forward(dev_in["Q"], dev_in["K"], dev_in["V"],
+                                            dev_in["q_perm"], dev_in["k_perm"],
+                                            dev_in["q_offsets"], dev_in["k_offsets"], w.ratio,
+                                            out=hp.out, workspace=hp.ws)
             out_host.copy_(o, non_blocking=True)
 
         e2e_step()
@@ -441,7 +475,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "H": w.H, "N": w.N, "d": w.d, "topk_ratio": w.ratio,
-                   "k": hp.k, "nqb": hp.nqb, "nkb": hp.nkb, "block": w.block,
+                   "k": hp.k, "nqb": hp.nqb, "nkb": hp.nkb, "context_tokens": hp.nc,
+                   "block": w.block,
                    "layout": w.layout, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (4.5 GB of Q/K/V per call), no flush"},
         "actual_tflops": att_flops / (ms_per_step / 1e3) / 1e12 * world,
@@ -451,7 +486,7 @@ def main():
                      "kernel": "attend (tcgen05 two-branch attention)",
                      "algorithmic_flops_per_launch": att_flops},
         "kernels": kernels,
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": (5 + (2 if hp.convert_ctx else 0)) * args.steps,
         "clocks": clock_info,
         "e2e": e2e,
     }

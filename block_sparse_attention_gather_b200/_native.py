@@ -20,6 +20,8 @@ __all__ = [
     "spark_bsa_workspace_size", "spark_bsa_forward", "spark_bsa_read_error",
     "spark_bsa_gather_q", "spark_bsa_anchor", "spark_bsa_gather_kv_summarize",
     "spark_bsa_route", "spark_bsa_attend", "workspace_views", "spark_bsa_forward_noalloc",
+    "spark_bsa_workspace_size_ctx", "spark_bsa_forward_ctx", "spark_bsa_context_bf16",
+    "spark_bsa_attend_ctx",
 ]
 
 SPARK_BF16, SPARK_F32 = 0, 1
@@ -29,6 +31,8 @@ EXPORTED = [
     "spark_bsa_workspace_size", "spark_bsa_forward", "spark_bsa_read_error",
     "spark_bsa_gather_q", "spark_bsa_anchor", "spark_bsa_gather_kv_summarize",
     "spark_bsa_route", "spark_bsa_attend", "spark_bsa_forward_noalloc",
+    "spark_bsa_workspace_size_ctx", "spark_bsa_forward_ctx", "spark_bsa_context_bf16",
+    "spark_bsa_attend_ctx",
 ]
 
 
@@ -78,6 +82,12 @@ def lib():
                                   _I, _P, _I, _P, _P]),
         "spark_bsa_forward_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _I,
                                            _D, _P, _P]),
+        "spark_bsa_workspace_size_ctx": (_SZ, [_I, _I, _I, _I, _I, _D, _I]),
+        "spark_bsa_forward_ctx": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _I,
+                                       _P, _I, _D, _P, _P, _SZ, _P]),
+        "spark_bsa_context_bf16": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
+        "spark_bsa_attend_ctx": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _I,
+                                      _P, _I, _I, _I, _I, _P, _I, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -318,4 +328,101 @@ def spark_bsa_forward_noalloc(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, top
                                          _ptr(k_offsets), nkb, float(topk_ratio), _ptr(out),
                                          _stream(stream))
     _check("spark_bsa_forward_noalloc", st)
+    return out
+
+
+# ------------------------------------------------------------------ context (sink) tokens
+
+def spark_bsa_workspace_size_ctx(H, N, d, nqb, nkb, topk_ratio, nc) -> int:
+    return int(lib().spark_bsa_workspace_size_ctx(H, N, d, nqb, nkb, float(topk_ratio), int(nc)))
+
+
+def _context_args(Kc, Vc, H, d, dtype, dev):
+    if Kc is None and Vc is None:
+        return None, None, 0
+    _need(Kc, "Kc", dtype, dev)
+    _need(Vc, "Vc", dtype, dev)
+    if Kc.dim() != 3 or Kc.shape[0] != H or Kc.shape[2] != d or Vc.shape != Kc.shape:
+        raise ValueError("Kc and Vc must have the shape [H, nc, d]")
+    return Kc, Vc, Kc.shape[1]
+
+
+def spark_bsa_forward_ctx(Q, K, V, Kc, Vc, q_perm, k_perm, q_offsets, k_offsets, topk_ratio,
+                          out=None, workspace=None, stream=None):
+    """spark_bsa_forward with context (sink) tokens Kc, Vc [H, nc, d] (same dtype as Q);
+    returns (out, workspace, layout).  The workspace holds the layout's intermediates followed
+    by the bf16 context rows."""
+    _need(Q, "Q", (torch.bfloat16, torch.float32))
+    dev = Q.device
+    H, N, d = Q.shape
+    for n, t in (("K", K), ("V", V)):
+        _need(t, n, Q.dtype, dev)
+    if K.shape != Q.shape or V.shape != Q.shape:
+        raise ValueError("Q, K, V must share the shape [H, N, d]")
+    Kc, Vc, nc = _context_args(Kc, Vc, H, d, Q.dtype, dev)
+    for n, t in (("q_perm", q_perm), ("k_perm", k_perm)):
+        _need(t, n, torch.int32, dev)
+        if t.shape != (H, N):
+            raise ValueError(f"{n} must have shape [H, N]")
+    for n, t in (("q_offsets", q_offsets), ("k_offsets", k_offsets)):
+        _need(t, n, torch.int32, dev)
+    nqb, nkb = q_offsets.numel() - 1, k_offsets.numel() - 1
+    layout = spark_bsa_workspace_layout(H, N, d, nqb, nkb, topk_ratio)
+    size = spark_bsa_workspace_size_ctx(H, N, d, nqb, nkb, topk_ratio, nc)
+    if out is None:
+        out = torch.empty_like(Q)
+    _need(out, "out", Q.dtype, dev)
+    if workspace is None:
+        workspace = torch.empty(size, dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    st = lib().spark_bsa_forward_ctx(_ptr(Q), _ptr(K), _ptr(V), _ptr(Kc), _ptr(Vc), nc,
+                                     _code(Q.dtype), H, N, d, _ptr(q_perm), _ptr(k_perm),
+                                     _ptr(q_offsets), nqb, _ptr(k_offsets), nkb,
+                                     float(topk_ratio), _ptr(out), _ptr(workspace),
+                                     workspace.numel(), _stream(stream))
+    _check("spark_bsa_forward_ctx", st)
+    return out, workspace, layout
+
+
+def spark_bsa_context_bf16(Kc, Vc, Kc_bf16=None, Vc_bf16=None, stream=None):
+    """bf16 copies of the context rows ([H, nc, d]); returns (Kc_bf16, Vc_bf16)."""
+    _need(Kc, "Kc", (torch.bfloat16, torch.float32))
+    H, nc, d = Kc.shape
+    Kc, Vc, nc = _context_args(Kc, Vc, H, d, Kc.dtype, Kc.device)
+    if Kc_bf16 is None:
+        Kc_bf16 = torch.empty(H, nc, d, dtype=torch.bfloat16, device=Kc.device)
+    if Vc_bf16 is None:
+        Vc_bf16 = torch.empty(H, nc, d, dtype=torch.bfloat16, device=Kc.device)
+    _need(Kc_bf16, "Kc_bf16", torch.bfloat16, Kc.device)
+    _need(Vc_bf16, "Vc_bf16", torch.bfloat16, Kc.device)
+    st = lib().spark_bsa_context_bf16(_ptr(Kc), _ptr(Vc), _code(Kc.dtype), H, nc, d,
+                                      _ptr(Kc_bf16), _ptr(Vc_bf16), _stream(stream))
+    _check("spark_bsa_context_bf16", st)
+    return Kc_bf16, Vc_bf16
+
+
+def spark_bsa_attend_ctx(Qp, Kp, Vp, k_tilde, v_tilde, cbias, sel, Kc, Vc, q_perm, q_offsets,
+                         k_offsets, out_dtype=torch.bfloat16, out=None, err=None, stream=None):
+    """spark_bsa_attend with bf16 context rows Kc, Vc [H, nc, d]."""
+    _need(Qp, "Qp", torch.bfloat16)
+    dev = Qp.device
+    H, N, d = Qp.shape
+    for n, t, dt in (("Kp", Kp, torch.bfloat16), ("Vp", Vp, torch.bfloat16),
+                     ("k_tilde", k_tilde, torch.bfloat16), ("v_tilde", v_tilde, torch.bfloat16),
+                     ("cbias", cbias, torch.float32), ("sel", sel, torch.int32),
+                     ("q_perm", q_perm, torch.int32), ("q_offsets", q_offsets, torch.int32),
+                     ("k_offsets", k_offsets, torch.int32)):
+        _need(t, n, dt, dev)
+    Kc, Vc, nc = _context_args(Kc, Vc, H, d, torch.bfloat16, dev)
+    nqb, nkb = q_offsets.numel() - 1, k_offsets.numel() - 1
+    k = sel.shape[-1]
+    if out is None:
+        out = torch.empty(H, N, d, dtype=out_dtype, device=dev)
+    _need(out, "out", out_dtype, dev)
+    st = lib().spark_bsa_attend_ctx(_ptr(Qp), _ptr(Kp), _ptr(Vp), _ptr(k_tilde), _ptr(v_tilde),
+                                    _ptr(cbias), _ptr(sel), k, _ptr(Kc), _ptr(Vc), nc,
+                                    _ptr(q_perm), _ptr(q_offsets), nqb, _ptr(k_offsets), nkb,
+                                    H, N, d, _ptr(out), _code(out_dtype), _ptr(err),
+                                    _stream(stream))
+    _check("spark_bsa_attend_ctx", st)
     return out

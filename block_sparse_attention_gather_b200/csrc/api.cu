@@ -97,18 +97,99 @@ spark_status layout_of(int H, int N, int d, int nqb, int nkb, double ratio,
   return SPARK_OK;
 }
 
+// Bytes of one bf16 context tensor [H,nc,d] inside a workspace (256-byte aligned).
+size_t context_bytes(int H, int nc, int d) {
+  return align_up(static_cast<size_t>(H) * static_cast<size_t>(nc) * d * 2);
+}
+
 spark_status attend_impl(const void* Qp, const void* Kp, const void* Vp, const void* k_tilde,
                          const void* v_tilde, const float* cbias, const int32_t* sel, int k,
-                         const int32_t* q_perm, const int32_t* q_offsets, int nqb,
-                         const int32_t* k_offsets, int nkb, int H, int N, int d, void* out,
-                         int out_dtype, uint32_t* err, cudaStream_t s) {
+                         const void* Kc, const void* Vc, int nc, const int32_t* q_perm,
+                         const int32_t* q_offsets, int nqb, const int32_t* k_offsets, int nkb,
+                         int H, int N, int d, void* out, int out_dtype, uint32_t* err,
+                         cudaStream_t s) {
   AttendMaps maps;
   if (!encode_rows_map(&maps.q, Qp, H, N, d) || !encode_rows_map(&maps.k, Kp, H, N, d) ||
       !encode_rows_map(&maps.v, Vp, H, N, d) || !encode_rows_map(&maps.kt, k_tilde, H, nkb, d) ||
       !encode_rows_map(&maps.vt, v_tilde, H, nkb, d))
     return SPARK_ERR_CUDA;
-  return from_cuda(launch_attend(maps, cbias, sel, k, q_perm, q_offsets, nqb, k_offsets, nkb, H,
-                                 N, d, out, out_dtype, err, s));
+  if (nc > 0) {
+    if (!encode_rows_map(&maps.kc, Kc, H, nc, d) || !encode_rows_map(&maps.vc, Vc, H, nc, d))
+      return SPARK_ERR_CUDA;
+  } else {
+    maps.kc = maps.k;                            // never loaded: the kernel has no context tile
+    maps.vc = maps.v;
+  }
+  return from_cuda(launch_attend(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb, k_offsets, nkb,
+                                 H, N, d, out, out_dtype, err, s));
+}
+
+spark_status check_context(const void* Kc, const void* Vc, int nc) {
+  if (nc < 0 || nc > SPARK_MAX_NC) return SPARK_ERR_INVALID_ARG;
+  if (nc > 0 && (!Kc || !Vc || !aligned(Kc, 16) || !aligned(Vc, 16)))
+    return SPARK_ERR_INVALID_ARG;
+  return SPARK_OK;
+}
+
+// The whole forward pass; nc == 0 runs without context rows.
+spark_status forward_impl(const void* Q, const void* K, const void* V, const void* Kc,
+                          const void* Vc, int nc, int dtype, int H, int N, int d,
+                          const int32_t* q_perm, const int32_t* k_perm,
+                          const int32_t* q_block_offsets, int nqb,
+                          const int32_t* k_block_offsets, int nkb, double topk_ratio, void* out,
+                          void* workspace, size_t workspace_bytes, cudaStream_t s) {
+  if (!Q || !K || !V || !q_perm || !k_perm || !q_block_offsets || !k_block_offsets || !out)
+    return SPARK_ERR_INVALID_ARG;
+  if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  spark_bsa_layout L;
+  spark_status st = layout_of(H, N, d, nqb, nkb, topk_ratio, &L);
+  if (st != SPARK_OK) return st;
+  st = check_context(Kc, Vc, nc);
+  if (st != SPARK_OK) return st;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16))
+    return SPARK_ERR_INVALID_ARG;
+  const size_t cbytes = nc > 0 ? context_bytes(H, nc, d) : 0;
+  if (workspace == nullptr || workspace_bytes < L.total + 2 * cbytes ||
+      !aligned(workspace, kAlign))
+    return SPARK_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* Qp = ws + L.Qp;
+  void* Kp = ws + L.Kp;
+  void* Vp = ws + L.Vp;
+  float* qbar_blocks = reinterpret_cast<float*>(ws + L.qbar_blocks);
+  float* qbar = reinterpret_cast<float*>(ws + L.qbar);
+  float* kbar = reinterpret_cast<float*>(ws + L.kbar);
+  void* kt = ws + L.k_tilde;
+  void* vt = ws + L.v_tilde;
+  float* cbias = reinterpret_cast<float*>(ws + L.cbias);
+  int32_t* sel = reinterpret_cast<int32_t*>(ws + L.sel);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.err);
+  void* Kcb = ws + L.total;
+  void* Vcb = ws + L.total + cbytes;
+
+  if (cudaMemsetAsync(err, 0, sizeof(uint32_t), s) != cudaSuccess) return SPARK_ERR_CUDA;
+  if (launch_gather_q(Q, dtype, H, N, d, q_perm, q_block_offsets, nqb, Qp, qbar_blocks, err, s) !=
+      cudaSuccess)
+    return SPARK_ERR_CUDA;
+  if (launch_anchor(qbar_blocks, q_block_offsets, H, N, d, nqb, qbar, s) != cudaSuccess)
+    return SPARK_ERR_CUDA;
+  if (launch_gather_kv_summary(K, V, dtype, H, N, d, k_perm, k_block_offsets, nkb, qbar, Kp, Vp,
+                               kbar, kt, vt, cbias, err, s) != cudaSuccess)
+    return SPARK_ERR_CUDA;
+  if (launch_route(qbar_blocks, kbar, H, nqb, nkb, d, L.k, sel, err, s) != cudaSuccess)
+    return SPARK_ERR_CUDA;
+  const void* Kca = Kc;                          // bf16 context rows are read in place
+  const void* Vca = Vc;
+  if (nc > 0 && dtype == SPARK_F32) {
+    const size_t n = static_cast<size_t>(H) * nc * d;
+    if (launch_to_bf16(Kc, dtype, n, Kcb, s) != cudaSuccess ||
+        launch_to_bf16(Vc, dtype, n, Vcb, s) != cudaSuccess)
+      return SPARK_ERR_CUDA;
+    Kca = Kcb;
+    Vca = Vcb;
+  }
+  return attend_impl(Qp, Kp, Vp, kt, vt, cbias, sel, L.k, Kca, Vca, nc, q_perm, q_block_offsets,
+                     nqb, k_block_offsets, nkb, H, N, d, out, dtype, err, s);
 }
 
 }  // namespace
@@ -217,8 +298,68 @@ spark_status spark_bsa_attend(const void* Qp, const void* Kp, const void* Vp,
   if (!aligned(Qp, 16) || !aligned(Kp, 16) || !aligned(Vp, 16) || !aligned(k_tilde, 16) ||
       !aligned(v_tilde, 16) || !aligned(out, 16))
     return SPARK_ERR_INVALID_ARG;
-  return attend_impl(Qp, Kp, Vp, k_tilde, v_tilde, cbias, sel, k, q_perm, q_block_offsets, nqb,
-                     k_block_offsets, nkb, H, N, d, out, out_dtype, err, as_stream(stream));
+  return attend_impl(Qp, Kp, Vp, k_tilde, v_tilde, cbias, sel, k, nullptr, nullptr, 0, q_perm,
+                     q_block_offsets, nqb, k_block_offsets, nkb, H, N, d, out, out_dtype, err,
+                     as_stream(stream));
+}
+
+spark_status spark_bsa_attend_ctx(const void* Qp, const void* Kp, const void* Vp,
+                                  const void* k_tilde, const void* v_tilde, const float* cbias,
+                                  const int32_t* sel, int k, const void* Kc, const void* Vc,
+                                  int nc, const int32_t* q_perm, const int32_t* q_block_offsets,
+                                  int nqb, const int32_t* k_block_offsets, int nkb, int H, int N,
+                                  int d, void* out, int out_dtype, uint32_t* err, void* stream) {
+  if (!Qp || !Kp || !Vp || !k_tilde || !v_tilde || !cbias || !sel || !q_perm ||
+      !q_block_offsets || !k_block_offsets || !out)
+    return SPARK_ERR_INVALID_ARG;
+  if (out_dtype != SPARK_BF16 && out_dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  spark_status st = check_sizes(H, N, d, nqb, nkb);
+  if (st != SPARK_OK) return st;
+  st = check_context(Kc, Vc, nc);
+  if (st != SPARK_OK) return st;
+  if (k < 1 || k > nkb) return SPARK_ERR_INVALID_ARG;
+  if (!aligned(Qp, 16) || !aligned(Kp, 16) || !aligned(Vp, 16) || !aligned(k_tilde, 16) ||
+      !aligned(v_tilde, 16) || !aligned(out, 16))
+    return SPARK_ERR_INVALID_ARG;
+  return attend_impl(Qp, Kp, Vp, k_tilde, v_tilde, cbias, sel, k, Kc, Vc, nc, q_perm,
+                     q_block_offsets, nqb, k_block_offsets, nkb, H, N, d, out, out_dtype, err,
+                     as_stream(stream));
+}
+
+spark_status spark_bsa_context_bf16(const void* Kc, const void* Vc, int dtype, int H, int nc,
+                                    int d, void* Kc_bf16, void* Vc_bf16, void* stream) {
+  if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  if (H < 1 || H > 65535) return SPARK_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SPARK_ERR_UNSUPPORTED;
+  spark_status st = check_context(Kc, Vc, nc);
+  if (st != SPARK_OK) return st;
+  if (nc == 0) return SPARK_OK;
+  if (!Kc_bf16 || !Vc_bf16 || !aligned(Kc_bf16, 16) || !aligned(Vc_bf16, 16))
+    return SPARK_ERR_INVALID_ARG;
+  const size_t n = static_cast<size_t>(H) * nc * d;
+  cudaStream_t s = as_stream(stream);
+  if (launch_to_bf16(Kc, dtype, n, Kc_bf16, s) != cudaSuccess) return SPARK_ERR_CUDA;
+  return from_cuda(launch_to_bf16(Vc, dtype, n, Vc_bf16, s));
+}
+
+size_t spark_bsa_workspace_size_ctx(int H, int N, int d, int nqb, int nkb, double topk_ratio,
+                                    int nc) {
+  spark_bsa_layout L;
+  if (layout_of(H, N, d, nqb, nkb, topk_ratio, &L) != SPARK_OK) return 0;
+  if (nc < 0 || nc > SPARK_MAX_NC) return 0;
+  return L.total + (nc > 0 ? 2 * context_bytes(H, nc, d) : 0);
+}
+
+spark_status spark_bsa_forward_ctx(const void* Q, const void* K, const void* V, const void* Kc,
+                                   const void* Vc, int nc, int dtype, int H, int N, int d,
+                                   const int32_t* q_perm, const int32_t* k_perm,
+                                   const int32_t* q_block_offsets, int nqb,
+                                   const int32_t* k_block_offsets, int nkb, double topk_ratio,
+                                   void* out, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  return forward_impl(Q, K, V, Kc, Vc, nc, dtype, H, N, d, q_perm, k_perm, q_block_offsets, nqb,
+                      k_block_offsets, nkb, topk_ratio, out, workspace, workspace_bytes,
+                      as_stream(stream));
 }
 
 spark_status spark_bsa_forward(const void* Q, const void* K, const void* V, int dtype, int H,
@@ -227,43 +368,9 @@ spark_status spark_bsa_forward(const void* Q, const void* K, const void* V, int 
                                const int32_t* k_block_offsets, int nkb, double topk_ratio,
                                void* out, void* workspace, size_t workspace_bytes,
                                void* stream) {
-  if (!Q || !K || !V || !q_perm || !k_perm || !q_block_offsets || !k_block_offsets || !out)
-    return SPARK_ERR_INVALID_ARG;
-  if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
-  spark_bsa_layout L;
-  spark_status st = layout_of(H, N, d, nqb, nkb, topk_ratio, &L);
-  if (st != SPARK_OK) return st;
-  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16))
-    return SPARK_ERR_INVALID_ARG;
-  if (workspace == nullptr || workspace_bytes < L.total || !aligned(workspace, kAlign))
-    return SPARK_ERR_WORKSPACE;
-  cudaStream_t s = as_stream(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  void* Qp = ws + L.Qp;
-  void* Kp = ws + L.Kp;
-  void* Vp = ws + L.Vp;
-  float* qbar_blocks = reinterpret_cast<float*>(ws + L.qbar_blocks);
-  float* qbar = reinterpret_cast<float*>(ws + L.qbar);
-  float* kbar = reinterpret_cast<float*>(ws + L.kbar);
-  void* kt = ws + L.k_tilde;
-  void* vt = ws + L.v_tilde;
-  float* cbias = reinterpret_cast<float*>(ws + L.cbias);
-  int32_t* sel = reinterpret_cast<int32_t*>(ws + L.sel);
-  uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.err);
-
-  if (cudaMemsetAsync(err, 0, sizeof(uint32_t), s) != cudaSuccess) return SPARK_ERR_CUDA;
-  if (launch_gather_q(Q, dtype, H, N, d, q_perm, q_block_offsets, nqb, Qp, qbar_blocks, err, s) !=
-      cudaSuccess)
-    return SPARK_ERR_CUDA;
-  if (launch_anchor(qbar_blocks, q_block_offsets, H, N, d, nqb, qbar, s) != cudaSuccess)
-    return SPARK_ERR_CUDA;
-  if (launch_gather_kv_summary(K, V, dtype, H, N, d, k_perm, k_block_offsets, nkb, qbar, Kp, Vp,
-                               kbar, kt, vt, cbias, err, s) != cudaSuccess)
-    return SPARK_ERR_CUDA;
-  if (launch_route(qbar_blocks, kbar, H, nqb, nkb, d, L.k, sel, err, s) != cudaSuccess)
-    return SPARK_ERR_CUDA;
-  return attend_impl(Qp, Kp, Vp, kt, vt, cbias, sel, L.k, q_perm, q_block_offsets, nqb,
-                     k_block_offsets, nkb, H, N, d, out, dtype, err, s);
+  return forward_impl(Q, K, V, nullptr, nullptr, 0, dtype, H, N, d, q_perm, k_perm,
+                      q_block_offsets, nqb, k_block_offsets, nkb, topk_ratio, out, workspace,
+                      workspace_bytes, as_stream(stream));
 }
 
 }  // extern "C"

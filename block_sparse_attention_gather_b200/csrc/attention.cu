@@ -27,8 +27,10 @@
 //              tile t+2 may rescale O_{t%2} once it sees S(t+2).
 //
 // Tile list of a CTA: the k selected blocks in ascending order (a 128-row TMA box starting at
-// the block's first row; rows past the block are masked), then ceil(nkb/128) tiles of the
-// summary rows (rows past nkb are zero-filled by TMA and masked, selected blocks masked).
+// the block's first row; rows past the block are masked), then ceil(nc/128) tiles of the
+// head's context tokens (same blog section: context/sink tokens stay exact, outside the Top-K
+// budget; rows past nc masked), then ceil(nkb/128) tiles of the summary rows (rows past nkb
+// are zero-filled by TMA and masked, selected blocks masked).
 //
 // TMEM columns (512 allocated, one CTA per SM): S/P buffer 0 [0,128), buffer 1 [128,256),
 // O_even [256,256+D), O_odd [384,384+D).
@@ -68,15 +70,20 @@ __device__ __forceinline__ bool wait_bounded_ignore_abort(uint64_t* bar, uint32_
   return true;
 }
 
-// Row range of key tile t and how many of its 128 rows are valid.
+// Row range of key tile t, its source and how many of its 128 rows are valid.
+enum TileSrc : int { kSrcVideo = 0, kSrcContext = 1, kSrcSummary = 2 };
+
 struct TileInfo {
-  int y;          // first row (in Kp/Vp for exact tiles, in k~/v~ for summary tiles)
-  int nvalid;     // exact tiles: block size (rows >= nvalid are masked)
-  bool exact;
+  int y;          // first row (in Kp/Vp, in the context rows, or in k~/v~)
+  int nvalid;     // exact tiles: valid rows (rows >= nvalid are masked)
+  int src;        // TileSrc
+  bool exact;     // video or context rows (no summary offset)
 };
 
-__device__ __forceinline__ TileInfo tile_info(int t, int k, const int32_t* sel_row,
-                                              const int32_t* k_offsets, int nkb, int N) {
+// Tiles 0..k-1: selected video blocks; then nxt context tiles; then the summary tiles.
+__device__ __forceinline__ TileInfo tile_info(int t, int k, int nxt, int nc,
+                                              const int32_t* sel_row, const int32_t* k_offsets,
+                                              int nkb, int N) {
   TileInfo ti;
   if (t < k) {
     const int B = min(max(sel_row[t], 0), nkb - 1);
@@ -84,10 +91,17 @@ __device__ __forceinline__ TileInfo tile_info(int t, int k, const int32_t* sel_r
     const int hi = min(max(k_offsets[B + 1], lo), N);
     ti.y = lo;
     ti.nvalid = min(hi - lo, kMaxBlock);
+    ti.src = kSrcVideo;
+    ti.exact = true;
+  } else if (t < k + nxt) {
+    ti.y = (t - k) * 128;
+    ti.nvalid = min(nc - ti.y, 128);
+    ti.src = kSrcContext;
     ti.exact = true;
   } else {
-    ti.y = (t - k) * 128;
+    ti.y = (t - k - nxt) * 128;
     ti.nvalid = 128;
+    ti.src = kSrcSummary;
     ti.exact = false;
   }
   return ti;
@@ -178,7 +192,8 @@ template <int D, bool kBiasSmem>
 __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kt,
-    const __grid_constant__ CUtensorMap map_vt, const float* __restrict__ cbias,
+    const __grid_constant__ CUtensorMap map_vt, const __grid_constant__ CUtensorMap map_kc,
+    const __grid_constant__ CUtensorMap map_vc, int nc, const float* __restrict__ cbias,
     const int32_t* __restrict__ sel, int k, const int32_t* __restrict__ q_perm,
     const int32_t* __restrict__ q_offsets, int nqb, const int32_t* __restrict__ k_offsets,
     int nkb, int N, void* __restrict__ out, int out_dtype, uint32_t* err) {
@@ -207,7 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   __syncthreads();
   if (s_skip) return;                                      // uniform: no work, nothing held
   const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
-  const int T = k + nct;
+  const int nxt = (nc + 127) / 128;                 // context tiles
+  const int T = k + nxt + nct;
   const int32_t* sel_row = sel + (static_cast<size_t>(h) * nqb + A) * k;
   const int nwords = (nkb + 31) / 32;
   const float* cb = cbias + static_cast<size_t>(h) * nkb;
@@ -263,9 +279,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       uint64_t* full = is_k ? bars->kfull : bars->vfull;
       uint64_t* empty = is_k ? bars->kempty : bars->vempty;
       const CUtensorMap* mx = is_k ? &map_k : &map_v;
+      const CUtensorMap* mc = is_k ? &map_kc : &map_vc;
       const CUtensorMap* ms = is_k ? &map_kt : &map_vt;
       tma_prefetch_desc(mx);
       tma_prefetch_desc(ms);
+      if (nxt > 0) tma_prefetch_desc(mc);
       if (is_k) {
         tma_prefetch_desc(&map_q);
         mbar_arrive_expect_tx(&bars->qfull, TILE_BYTES);
@@ -274,17 +292,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           tma_load_3d(qst + a * 16384, &map_q, &bars->qfull, a * 64, qrow, h);
       }
       int issued = 0;
-      TileInfo next = tile_info(0, k, sel_row, k_offsets, nkb, N);
+      TileInfo next = tile_info(0, k, nxt, nc, sel_row, k_offsets, nkb, N);
       for (int t = 0; t < T; ++t) {
         const int s = t % stages;
         const TileInfo ti = next;
         if (t >= stages && !mbar_wait(&empty[s], ((t / stages) - 1) & 1, abort_flag, err)) break;
         mbar_arrive_expect_tx(&full[s], TILE_BYTES);
+        const CUtensorMap* map = ti.src == kSrcVideo ? mx : (ti.src == kSrcContext ? mc : ms);
         for (int a = 0; a < NATOM; ++a)
-          tma_load_3d(ring + s * TILE_BYTES + a * 16384, ti.exact ? mx : ms, &full[s], a * 64,
-                      ti.y, h);
+          tma_load_3d(ring + s * TILE_BYTES + a * 16384, map, &full[s], a * 64, ti.y, h);
         issued = t + 1;
-        if (t + 1 < T) next = tile_info(t + 1, k, sel_row, k_offsets, nkb, N);
+        if (t + 1 < T) next = tile_info(t + 1, k, nxt, nc, sel_row, k_offsets, nkb, N);
       }
       if (*abort_flag) {
         // drain: wait for every load still in flight (the last round of each stage)
@@ -348,13 +366,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     const float scale_log2 = kLog2e * rsqrtf(static_cast<float>(D));
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true, first = true;
-    TileInfo next = tile_info(par, k, sel_row, k_offsets, nkb, N);
+    TileInfo next = tile_info(par, k, nxt, nc, sel_row, k_offsets, nkb, N);
     for (int t = par; t < T; t += 2) {
       const TileInfo ti = next;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->sfull[par], (t >> 1) & 1, abort_flag, err));
       if (!ok) break;
       tc_fence_after_sync();
-      if (t + 2 < T) next = tile_info(t + 2, k, sel_row, k_offsets, nkb, N);
+      if (t + 2 < T) next = tile_info(t + 2, k, nxt, nc, sel_row, k_offsets, nkb, N);
       const float c = ti.exact ? scale_log2 : 1.f;
       // pass 1: the tile's row maximum (log2 units)
       float x[64];
@@ -487,8 +505,9 @@ static size_t attend_smem_bytes(int d, int nkb, int k) {
 }
 
 template <int D, bool kBiasSmem>
-static cudaError_t launch_attend_t(const AttendMaps& m, const float* cbias, const int32_t* sel,
-                                   int k, const int32_t* q_perm, const int32_t* q_offsets,
+static cudaError_t launch_attend_t(const AttendMaps& m, int nc, const float* cbias,
+                                   const int32_t* sel, int k, const int32_t* q_perm,
+                                   const int32_t* q_offsets,
                                    int nqb, const int32_t* k_offsets, int nkb, int H, int N,
                                    void* out, int out_dtype, uint32_t* err, cudaStream_t s) {
   const size_t smem = attend_smem_bytes(D, nkb, k);
@@ -498,25 +517,26 @@ static cudaError_t launch_attend_t(const AttendMaps& m, const float* cbias, cons
   if (e != cudaSuccess) return e;
   dim3 grid(nqb, H);
   attend_kernel<D, kBiasSmem><<<grid, kThreads, smem, s>>>(
-      m.q, m.k, m.v, m.kt, m.vt, cbias, sel, k, q_perm, q_offsets, nqb, k_offsets, nkb, N, out,
-      out_dtype, err);
+      m.q, m.k, m.v, m.kt, m.vt, m.kc, m.vc, nc, cbias, sel, k, q_perm, q_offsets, nqb,
+      k_offsets, nkb, N, out, out_dtype, err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attend(const AttendMaps& maps, const float* cbias, const int32_t* sel, int k,
-                          const int32_t* q_perm, const int32_t* q_offsets, int nqb,
-                          const int32_t* k_offsets, int nkb, int H, int N, int d, void* out,
-                          int out_dtype, uint32_t* err, cudaStream_t s) {
+cudaError_t launch_attend(const AttendMaps& maps, int nc, const float* cbias,
+                          const int32_t* sel, int k, const int32_t* q_perm,
+                          const int32_t* q_offsets, int nqb, const int32_t* k_offsets, int nkb,
+                          int H, int N, int d, void* out, int out_dtype, uint32_t* err,
+                          cudaStream_t s) {
   const bool bs = bias_in_smem(nkb, k);
   if (d == 128)
-    return bs ? launch_attend_t<128, true>(maps, cbias, sel, k, q_perm, q_offsets, nqb,
+    return bs ? launch_attend_t<128, true>(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb,
                                            k_offsets, nkb, H, N, out, out_dtype, err, s)
-              : launch_attend_t<128, false>(maps, cbias, sel, k, q_perm, q_offsets, nqb,
+              : launch_attend_t<128, false>(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb,
                                             k_offsets, nkb, H, N, out, out_dtype, err, s);
-  return bs ? launch_attend_t<64, true>(maps, cbias, sel, k, q_perm, q_offsets, nqb, k_offsets,
-                                        nkb, H, N, out, out_dtype, err, s)
-            : launch_attend_t<64, false>(maps, cbias, sel, k, q_perm, q_offsets, nqb, k_offsets,
-                                         nkb, H, N, out, out_dtype, err, s);
+  return bs ? launch_attend_t<64, true>(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb,
+                                        k_offsets, nkb, H, N, out, out_dtype, err, s)
+            : launch_attend_t<64, false>(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb,
+                                         k_offsets, nkb, H, N, out, out_dtype, err, s);
 }
 
 }  // namespace spark

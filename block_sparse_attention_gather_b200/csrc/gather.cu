@@ -374,4 +374,28 @@ cudaError_t launch_gather_kv_summary(const void* K, const void* V, int dtype, in
                                       k_tilde, v_tilde, cbias, err, s);
 }
 
+// Context rows to bf16 (round to nearest even), four elements per thread and iteration.
+__global__ void __launch_bounds__(256) to_bf16_kernel(const float4* __restrict__ src, size_t n4,
+                                                     uint2* __restrict__ dst) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 v = src[i];
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+    dst[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
+                        *reinterpret_cast<const uint32_t*>(&hi));
+  }
+}
+
+cudaError_t launch_to_bf16(const void* src, int dtype, size_t n, void* dst, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  if (dtype == 0) return cudaMemcpyAsync(dst, src, n * 2, cudaMemcpyDeviceToDevice, s);
+  const size_t n4 = n / 4;                       // n is a multiple of d (64 or 128)
+  const size_t blocks = (n4 + 255) / 256;
+  const unsigned grid = static_cast<unsigned>(blocks < 148 * 16 ? blocks : 148 * 16);
+  to_bf16_kernel<<<grid, 256, 0, s>>>(static_cast<const float4*>(src), n4,
+                                      static_cast<uint2*>(dst));
+  return cudaGetLastError();
+}
+
 }  // namespace spark

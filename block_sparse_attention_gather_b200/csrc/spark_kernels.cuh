@@ -24,15 +24,21 @@ cudaError_t launch_gather_kv_summary(const void* K, const void* V, int dtype, in
 cudaError_t launch_route(const float* qbar_blocks, const float* kbar, int H, int nqb, int nkb,
                          int d, int k, int32_t* sel, uint32_t* err, cudaStream_t s);
 
+// Context rows converted to bf16: dst[i] = bf16(src[i]) for n elements (a plain copy for
+// bf16 sources).
+cudaError_t launch_to_bf16(const void* src, int dtype, size_t n, void* dst, cudaStream_t s);
+
 // Operands of the attention kernel: TMA descriptors (encoded on the host by api.cu) of the
-// reblocked Q, K, V ([H,N,d] bf16) and of the summaries k~, v~ ([H,nkb,d] bf16).
+// reblocked Q, K, V ([H,N,d] bf16), of the summaries k~, v~ ([H,nkb,d] bf16) and of the
+// context rows Kc, Vc ([H,nc,d] bf16; unused when nc == 0).
 struct AttendMaps {
-  CUtensorMap q, k, v, kt, vt;
+  CUtensorMap q, k, v, kt, vt, kc, vc;
 };
 
-cudaError_t launch_attend(const AttendMaps& maps, const float* cbias, const int32_t* sel, int k,
-                          const int32_t* q_perm, const int32_t* q_offsets, int nqb,
-                          const int32_t* k_offsets, int nkb, int H, int N, int d, void* out,
-                          int out_dtype, uint32_t* err, cudaStream_t s);
+cudaError_t launch_attend(const AttendMaps& maps, int nc, const float* cbias,
+                          const int32_t* sel, int k, const int32_t* q_perm,
+                          const int32_t* q_offsets, int nqb, const int32_t* k_offsets, int nkb,
+                          int H, int N, int d, void* out, int out_dtype, uint32_t* err,
+                          cudaStream_t s);
 
 }  // namespace spark

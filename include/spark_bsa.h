@@ -81,6 +81,7 @@ typedef enum { SPARK_BF16 = 0, SPARK_F32 = 1 } spark_dtype;
 /* Library limits (SPARK_ERR_UNSUPPORTED beyond them). */
 #define SPARK_MAX_BLOCK 128        /* tokens per block                                        */
 #define SPARK_MAX_NKB 12800        /* key blocks per head                                     */
+#define SPARK_MAX_NC (1 << 20)     /* context tokens per head                                 */
 
 /* Human-readable name of a status code; never NULL. */
 SPARK_API const char* spark_status_string(int status);
@@ -173,6 +174,56 @@ SPARK_API spark_status spark_bsa_attend(const void* Qp, const void* Kp, const vo
                               const int32_t* q_block_offsets, int nqb,
                               const int32_t* k_block_offsets, int nkb, int H, int N, int d,
                               void* out, int out_dtype, uint32_t* err, void* stream);
+
+/* ---- Context (sink) tokens ----
+ * Spark-H3 blog, section "Spark-Reblock", after the BSA equations: context/sink tokens stay
+ * exact and are not counted against the video-block Top-K budget.  Reading taken here: each
+ * head has nc context tokens with keys Kc[h] and values Vc[h] ([H,nc,d], row-major, same dtype
+ * as Q/K/V).  Every video query attends to all of them exactly, in the same row-wise softmax
+ * as the exact and compressed branches (logit sigma q.kc_j).  They form no block and take no
+ * part in the anchor, the block means, the summaries or the routing; k is still taken over the
+ * nkb video blocks.  Context queries are not part of this operation (the caller attends them
+ * densely).  0 <= nc <= SPARK_MAX_NC; nc == 0 is exactly the call without context. */
+
+/* Workspace bytes spark_bsa_forward_ctx needs: spark_bsa_workspace_size plus two bf16
+ * [H,nc,d] regions (each rounded up to 256 bytes) that receive the converted context rows at
+ * offsets layout.total and layout.total + round256(H*nc*d*2).  0 if the arguments are
+ * invalid. */
+SPARK_API size_t spark_bsa_workspace_size_ctx(int H, int N, int d, int nqb, int nkb,
+                                              double topk_ratio, int nc);
+
+/* spark_bsa_forward with context tokens.  Kc, Vc: device, 16-byte aligned, [H,nc,d] of
+ * `dtype` (may be NULL when nc == 0).  bf16 context rows are read in place; fp32 ones are
+ * first converted to bf16 into the workspace (after the intermediates of
+ * spark_bsa_workspace_layout).  They are attended as extra exact key tiles.  Errors as spark_bsa_forward; SPARK_ERR_INVALID_ARG for nc outside
+ * [0, SPARK_MAX_NC] or missing/misaligned context pointers. */
+SPARK_API spark_status spark_bsa_forward_ctx(const void* Q, const void* K, const void* V,
+                                             const void* Kc, const void* Vc, int nc, int dtype,
+                                             int H, int N, int d, const int32_t* q_perm,
+                                             const int32_t* k_perm,
+                                             const int32_t* q_block_offsets, int nqb,
+                                             const int32_t* k_block_offsets, int nkb,
+                                             double topk_ratio, void* out, void* workspace,
+                                             size_t workspace_bytes, void* stream);
+
+/* Step of the context path: Kc_bf16[i] = bf16(Kc[i]), Vc_bf16[i] = bf16(Vc[i]) (round to
+ * nearest even; a copy for bf16 input), [H,nc,d].  All pointers device, 16-byte aligned. */
+SPARK_API spark_status spark_bsa_context_bf16(const void* Kc, const void* Vc, int dtype, int H,
+                                              int nc, int d, void* Kc_bf16, void* Vc_bf16,
+                                              void* stream);
+
+/* spark_bsa_attend with context rows: Kc, Vc are bf16 [H,nc,d] (16-byte aligned; NULL allowed
+ * when nc == 0).  The tiles of a query block are the selected video blocks, then ceil(nc/128)
+ * context tiles, then the summary tiles. */
+SPARK_API spark_status spark_bsa_attend_ctx(const void* Qp, const void* Kp, const void* Vp,
+                                            const void* k_tilde, const void* v_tilde,
+                                            const float* cbias, const int32_t* sel, int k,
+                                            const void* Kc, const void* Vc, int nc,
+                                            const int32_t* q_perm,
+                                            const int32_t* q_block_offsets, int nqb,
+                                            const int32_t* k_block_offsets, int nkb, int H,
+                                            int N, int d, void* out, int out_dtype,
+                                            uint32_t* err, void* stream);
 
 /* ---- Forward pass without any allocation ----
  * No counterpart in the pages: this entry point exists for callers that cannot allocate

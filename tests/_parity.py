@@ -35,18 +35,24 @@ def bf16_64(t: torch.Tensor) -> np.ndarray:
 
 
 def head_inputs(x: dict, h: int) -> dict:
-    """CPU float64 copies of one head's inputs, rounded to bf16 as the library does."""
-    return dict(Q=bf16_64(x["Q"][h]), K=bf16_64(x["K"][h]), V=bf16_64(x["V"][h]),
-                q_perm=x["q_perm"][h].cpu().numpy().astype(np.int64),
-                k_perm=x["k_perm"][h].cpu().numpy().astype(np.int64),
-                q_offsets=x["q_offsets"].cpu().numpy().astype(np.int64),
-                k_offsets=x["k_offsets"].cpu().numpy().astype(np.int64))
+    """CPU float64 copies of one head's inputs (and context rows, if any), rounded to bf16 as
+    the library does."""
+    hi = dict(Q=bf16_64(x["Q"][h]), K=bf16_64(x["K"][h]), V=bf16_64(x["V"][h]),
+              q_perm=x["q_perm"][h].cpu().numpy().astype(np.int64),
+              k_perm=x["k_perm"][h].cpu().numpy().astype(np.int64),
+              q_offsets=x["q_offsets"].cpu().numpy().astype(np.int64),
+              k_offsets=x["k_offsets"].cpu().numpy().astype(np.int64),
+              Kc=None, Vc=None)
+    if x.get("Kc") is not None:
+        hi["Kc"], hi["Vc"] = bf16_64(x["Kc"][h]), bf16_64(x["Vc"][h])
+    return hi
 
 
 def oracle_head(x: dict, h: int, ratio: float, blocks=None, sel=None, hi=None):
     hi = head_inputs(x, h) if hi is None else hi
     return O.forward_head(hi["Q"], hi["K"], hi["V"], hi["q_perm"], hi["k_perm"],
-                          hi["q_offsets"], hi["k_offsets"], ratio, blocks=blocks, sel=sel)
+                          hi["q_offsets"], hi["k_offsets"], ratio, blocks=blocks, sel=sel,
+                          Kc=hi["Kc"], Vc=hi["Vc"])
 
 
 def compare_sel(gpu_sel: np.ndarray, ref_sel: np.ndarray, scores: np.ndarray, k: int):

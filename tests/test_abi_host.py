@@ -124,6 +124,37 @@ def test_step_entry_points_reject_bad_arguments(L):
     assert L.spark_bsa_read_error(None, None, ctypes.byref(flags)) == INVALID
 
 
+def test_context_entry_points_reject_bad_arguments(L):
+    from block_sparse_attention_gather_b200 import (spark_bsa_workspace_layout,
+                                                    spark_bsa_workspace_size_ctx)
+    H, N, d, nqb, nkb = 24, 241920, 128, 1890, 1890
+    lay = spark_bsa_workspace_layout(H, N, d, nqb, nkb, 0.1)
+    cbytes = (H * 512 * d * 2 + 255) // 256 * 256
+    assert spark_bsa_workspace_size_ctx(H, N, d, nqb, nkb, 0.1, 0) == lay.total
+    assert spark_bsa_workspace_size_ctx(H, N, d, nqb, nkb, 0.1, 512) == lay.total + 2 * cbytes
+    assert spark_bsa_workspace_size_ctx(H, N, d, nqb, nkb, 0.1, -1) == 0
+    assert spark_bsa_workspace_size_ctx(H, N, d, nqb, nkb, 0.1, (1 << 20) + 1) == 0
+
+    p = ctypes.c_void_p(0x100000)
+    def fwd(Kc=p, Vc=p, nc=16, ws_bytes=1 << 40):
+        return L.spark_bsa_forward_ctx(p, p, p, Kc, Vc, nc, 0, 2, 1000, 128, p, p, p, 10, p, 10,
+                                       0.2, p, p, ws_bytes, None)
+    assert fwd(nc=-1) == INVALID
+    assert fwd(nc=(1 << 20) + 1) == INVALID
+    assert fwd(Kc=None) == INVALID
+    assert fwd(Vc=ctypes.c_void_p(0x100008)) == INVALID          # not 16-byte aligned
+    small = L.spark_bsa_workspace_size(2, 1000, 128, 10, 10, ctypes.c_double(0.2))
+    assert fwd(ws_bytes=small) == WORKSPACE                       # no room for the context rows
+    assert L.spark_bsa_context_bf16(p, p, 3, 2, 16, 128, p, p, None) == INVALID    # dtype
+    assert L.spark_bsa_context_bf16(p, p, 0, 2, 16, 96, p, p, None) == UNSUPPORTED
+    assert L.spark_bsa_context_bf16(p, None, 0, 2, 16, 128, p, p, None) == INVALID
+    assert L.spark_bsa_context_bf16(None, None, 0, 2, 0, 128, None, None, None) == 0  # no rows
+    assert L.spark_bsa_attend_ctx(p, p, p, p, p, p, p, 1, None, p, 5, p, p, 1, p, 1, 1, 10, 128,
+                                  p, 0, None, None) == INVALID   # Kc NULL with nc > 0
+    assert L.spark_bsa_attend_ctx(p, p, p, p, p, p, p, 1, p, p, -3, p, p, 1, p, 1, 1, 10, 128,
+                                  p, 0, None, None) == INVALID   # nc < 0
+
+
 def test_missing_library_fails_loudly(tmp_path):
     code = ("import block_sparse_attention_gather_b200._native as n;"
             f"n.LIB_PATH = {str(tmp_path / 'nope.so')!r};"
