@@ -52,6 +52,9 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=["attention", "reblock"], default="attention",
+                    help="attention: the two-branch forward (default); reblock: the "
+                         "Spark-Reblock partitioner on the same workload's Q and K")
     return ap.parse_args()
 
 
@@ -339,9 +342,122 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+REBLOCK_METRIC = "ms/call of the Spark-Reblock partitioner (q_reuse_k), 768p shape"
+
+
+def reblock_bytes_flops(H, N, d, levels, e_in, power_iters=4):
+    """Algorithmic work of one partitioner call: fp32 FMAs of the second moment and of the
+    whitening (2 H N d^2 flops each), and HBM bytes of the per-level passes over the bf16
+    unit rows (power_iters + 1 reads of X with the perm index per level) plus the keys,
+    histogram and scatter passes (4 + 4 + 4 + 8 bytes per token and level)."""
+    flops = 2 * 2.0 * H * N * d * d
+    prep_bytes = 2.0 * H * N * d * e_in + H * N * d * 2
+    level_bytes = levels * H * N * ((power_iters + 1) * (2 * d + 4) + 4 + 3 * 4 + 4 + 8)
+    return flops, prep_bytes, level_bytes
+
+
+def run_reblock(args, world, rank, local):
+    from block_sparse_attention_gather_b200 import (lib, spark_reblock_workspace_layout)
+    from block_sparse_attention_gather_b200.workloads import WORKLOADS, make_inputs
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w, device=device)
+    Q, K = x["Q"], x["K"]
+    del x
+    H, N, d = Q.shape
+    block = w.block
+    L = lib()
+    lay = spark_reblock_workspace_layout(H, N, d, block)
+    ws = torch.empty(lay.total, dtype=torch.uint8, device=device)
+    qp = torch.empty(H, N, dtype=torch.int32, device=device)
+    kp = torch.empty_like(qp)
+    offs = torch.empty(lay.nb + 1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+    s = ctypes.c_void_p(stream.cuda_stream)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    code = 0 if Q.dtype == torch.bfloat16 else 1
+
+    def call():
+        st = L.spark_reblock(p(Q), p(K), code, H, N, d, block, 0, p(qp), p(kp), p(offs), p(ws),
+                             ws.numel(), s)
+        if st != 0:
+            raise RuntimeError(f"spark_reblock failed with status {st}")
+
+    def prep():
+        st = L.spark_reblock_whiten(p(Q), p(K), code, H, N, d, block, p(ws), ws.numel(), s)
+        if st != 0:
+            raise RuntimeError(f"spark_reblock_whiten failed with status {st}")
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    peaks, peak_kind = load_peaks()
+    clocks = ClockSampler(device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(args.steps):
+        call()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    total_ms = ev[0].elapsed_time(ev[1])
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([total_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms = total_ms / args.steps
+    # the whitening steps alone (same kernels as inside the call)
+    pe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    pe[0].record(stream)
+    for _ in range(args.steps):
+        prep()
+    pe[1].record(stream)
+    torch.cuda.synchronize()
+    prep_ms = pe[0].elapsed_time(pe[1]) / args.steps
+    part_ms = ms - prep_ms
+    flops, prep_bytes, level_bytes = reblock_bytes_flops(H, N, d, lay.levels, Q.element_size())
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    gbs = level_bytes / (part_ms / 1e3) / 1e9
+    line = {
+        "impl": "ours", "op": "reblock", "metric": REBLOCK_METRIC, "value": ms, "unit": "ms",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "H": H, "N": N, "d": d, "block": block,
+                   "levels": lay.levels, "mode": "q_reuse_k", "power_iters": 4,
+                   "l2": "inputs larger than L2, no flush"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": gbs / hbm, "traffic": None,
+                     "kernel": "per-level passes (power, project, select, scatter)",
+                     "algorithmic_bytes_per_call": level_bytes},
+        "kernels": {"whiten (second moment, M^1/2, unit rows)": {
+                        "ms": prep_ms, "fp32_tflops": flops / (prep_ms / 1e3) / 1e12,
+                        "flops": flops, "bytes": prep_bytes},
+                    "levels": {"ms": part_ms, "GB/s": gbs, "bytes": level_bytes}},
+        # per call: 4 whitening kernels, the identity order, 19 kernels per level, offsets
+        "gpu_launches": (6 + 19 * lay.levels) * args.steps,
+        "clocks": clock_info,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     world, rank, local = init_dist()
+    if args.op == "reblock" and args.impl == "ours":
+        run_reblock(args, world, rank, local)
+        return
     if args.impl == "reference":
         run_reference(args, world, rank)
         if world > 1:

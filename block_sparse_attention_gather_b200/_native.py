@@ -21,7 +21,9 @@ __all__ = [
     "spark_bsa_gather_q", "spark_bsa_anchor", "spark_bsa_gather_kv_summarize",
     "spark_bsa_route", "spark_bsa_attend", "workspace_views", "spark_bsa_forward_noalloc",
     "spark_bsa_workspace_size_ctx", "spark_bsa_forward_ctx", "spark_bsa_context_bf16",
-    "spark_bsa_attend_ctx",
+    "spark_bsa_attend_ctx", "ReblockLayout", "spark_reblock_workspace_layout",
+    "spark_reblock_workspace_size", "spark_reblock_levels", "spark_reblock",
+    "spark_reblock_whiten", "spark_reblock_level", "reblock_views",
 ]
 
 SPARK_BF16, SPARK_F32 = 0, 1
@@ -32,8 +34,10 @@ EXPORTED = [
     "spark_bsa_gather_q", "spark_bsa_anchor", "spark_bsa_gather_kv_summarize",
     "spark_bsa_route", "spark_bsa_attend", "spark_bsa_forward_noalloc",
     "spark_bsa_workspace_size_ctx", "spark_bsa_forward_ctx", "spark_bsa_context_bf16",
-    "spark_bsa_attend_ctx",
+    "spark_bsa_attend_ctx", "spark_reblock_workspace_layout", "spark_reblock_workspace_size",
+    "spark_reblock_levels", "spark_reblock", "spark_reblock_whiten", "spark_reblock_level",
 ]
+REBLOCK_MODES = {"q_reuse_k": 0, "separate": 1}
 
 
 class SparkError(RuntimeError):
@@ -46,6 +50,11 @@ class Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "Qp", "Kp", "Vp", "qbar_blocks", "qbar", "kbar", "k_tilde", "v_tilde", "cbias", "sel",
         "err", "total")] + [("k", ctypes.c_int)]
+
+
+class ReblockLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("M", "W", "X", "total")] + \
+        [("levels", ctypes.c_int), ("nb", ctypes.c_int)]
 
 
 _LIB = None
@@ -88,6 +97,12 @@ def lib():
         "spark_bsa_context_bf16": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
         "spark_bsa_attend_ctx": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _I,
                                       _P, _I, _I, _I, _I, _P, _I, _P, _P]),
+        "spark_reblock_workspace_layout": (_I, [_I, _I, _I, _I, ctypes.POINTER(ReblockLayout)]),
+        "spark_reblock_workspace_size": (_SZ, [_I, _I, _I, _I]),
+        "spark_reblock_levels": (_I, [_I, _I]),
+        "spark_reblock": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+        "spark_reblock_whiten": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P]),
+        "spark_reblock_level": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -426,3 +441,78 @@ def spark_bsa_attend_ctx(Qp, Kp, Vp, k_tilde, v_tilde, cbias, sel, Kc, Vc, q_per
                                     _stream(stream))
     _check("spark_bsa_attend_ctx", st)
     return out
+
+
+# ------------------------------------------------------------ Spark-Reblock partitioner
+
+def spark_reblock_workspace_layout(H, N, d, block) -> ReblockLayout:
+    L = ReblockLayout()
+    _check("spark_reblock_workspace_layout",
+           lib().spark_reblock_workspace_layout(H, N, d, block, ctypes.byref(L)))
+    return L
+
+
+def spark_reblock_workspace_size(H, N, d, block) -> int:
+    return int(lib().spark_reblock_workspace_size(H, N, d, block))
+
+
+def spark_reblock_levels(N, block) -> int:
+    return int(lib().spark_reblock_levels(N, block))
+
+
+def reblock_views(workspace: torch.Tensor, layout: ReblockLayout, H, N, d) -> dict:
+    """Typed views of M, W (fp32 [H,d,d]) and X (bf16 [H,N,d]) in a reblock workspace."""
+    def view(off, count, dt):
+        nbytes = count * torch.empty(0, dtype=dt).element_size()
+        return workspace[off:off + nbytes].view(dt)
+    return {"M": view(layout.M, H * d * d, torch.float32).view(H, d, d),
+            "W": view(layout.W, H * d * d, torch.float32).view(H, d, d),
+            "X": view(layout.X, H * N * d, torch.bfloat16).view(H, N, d)}
+
+
+def spark_reblock(Q, K, block, mode="q_reuse_k", workspace=None, stream=None):
+    """Spark-Reblock partition of Q, K [H, N, d]; returns (q_perm, k_perm, offsets)."""
+    _need(Q, "Q", (torch.bfloat16, torch.float32))
+    _need(K, "K", Q.dtype, Q.device)
+    H, N, d = Q.shape
+    if K.shape != Q.shape:
+        raise ValueError("Q and K must share the shape [H, N, d]")
+    layout = spark_reblock_workspace_layout(H, N, d, block)
+    if workspace is None:
+        workspace = torch.empty(layout.total, dtype=torch.uint8, device=Q.device)
+    _need(workspace, "workspace", torch.uint8, Q.device)
+    q_perm = torch.empty(H, N, dtype=torch.int32, device=Q.device)
+    k_perm = torch.empty_like(q_perm)
+    offsets = torch.empty(layout.nb + 1, dtype=torch.int32, device=Q.device)
+    st = lib().spark_reblock(_ptr(Q), _ptr(K), _code(Q.dtype), H, N, d, int(block),
+                             REBLOCK_MODES[mode], _ptr(q_perm), _ptr(k_perm), _ptr(offsets),
+                             _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("spark_reblock", st)
+    return q_perm, k_perm, offsets
+
+
+def spark_reblock_whiten(X, Y, block, workspace=None, stream=None):
+    """Step: second moment of Y, its square root W, unit rows of W x into the workspace;
+    returns (workspace, layout, views)."""
+    _need(X, "X", (torch.bfloat16, torch.float32))
+    _need(Y, "Y", X.dtype, X.device)
+    H, N, d = X.shape
+    layout = spark_reblock_workspace_layout(H, N, d, block)
+    if workspace is None:
+        workspace = torch.empty(layout.total, dtype=torch.uint8, device=X.device)
+    st = lib().spark_reblock_whiten(_ptr(X), _ptr(Y), _code(X.dtype), H, N, d, int(block),
+                                    _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("spark_reblock_whiten", st)
+    return workspace, layout, reblock_views(workspace, layout, H, N, d)
+
+
+def spark_reblock_level(H, N, d, block, level, perm_in, workspace, perm_out=None, stream=None):
+    """Step: the splits of one tree level over the workspace's X rows; returns perm_out."""
+    _need(perm_in, "perm_in", torch.int32)
+    if perm_out is None:
+        perm_out = torch.empty_like(perm_in)
+    st = lib().spark_reblock_level(H, N, d, int(block), int(level), _ptr(perm_in),
+                                   _ptr(perm_out), _ptr(workspace), workspace.numel(),
+                                   _stream(stream))
+    _check("spark_reblock_level", st)
+    return perm_out

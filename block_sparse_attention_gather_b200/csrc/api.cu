@@ -373,4 +373,93 @@ spark_status spark_bsa_forward(const void* Q, const void* K, const void* V, int 
                       workspace_bytes, as_stream(stream));
 }
 
+// ---------------------------------------------------------------- Spark-Reblock
+
+int spark_reblock_levels(int N, int block) {
+  if (N < 1 || block < 1 || block > SPARK_MAX_BLOCK) return -1;
+  return static_cast<int>(reblock_levels(N, block));
+}
+
+spark_status spark_reblock_workspace_layout(int H, int N, int d, int block,
+                                            spark_reblock_layout* layout) {
+  if (layout == nullptr || H < 1 || N < 1 || block < 1 || block > SPARK_MAX_BLOCK)
+    return SPARK_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SPARK_ERR_UNSUPPORTED;
+  if (H > 65535 || (N + block - 1) / block > kMaxNkb) return SPARK_ERR_UNSUPPORTED;
+  const ReblockLayout L = reblock_layout(H, N, d, block);
+  layout->M = L.M;
+  layout->W = L.W;
+  layout->X = L.X;
+  layout->total = L.total;
+  layout->levels = L.levels;
+  layout->nb = L.nb;
+  return SPARK_OK;
+}
+
+size_t spark_reblock_workspace_size(int H, int N, int d, int block) {
+  spark_reblock_layout L;
+  return spark_reblock_workspace_layout(H, N, d, block, &L) == SPARK_OK ? L.total : 0;
+}
+
+spark_status spark_reblock_whiten(const void* X, const void* Y, int dtype, int H, int N, int d,
+                                  int block, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  if (!X || !Y) return SPARK_ERR_INVALID_ARG;
+  if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  spark_reblock_layout pub;
+  spark_status st = spark_reblock_workspace_layout(H, N, d, block, &pub);
+  if (st != SPARK_OK) return st;
+  if (!aligned(X, 16) || !aligned(Y, 16)) return SPARK_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pub.total || !aligned(workspace, kAlign))
+    return SPARK_ERR_WORKSPACE;
+  const ReblockLayout L = reblock_layout(H, N, d, block);
+  return from_cuda(launch_reblock_whiten(X, Y, dtype, H, N, d, workspace, L, as_stream(stream)));
+}
+
+spark_status spark_reblock_level(int H, int N, int d, int block, int level,
+                                 const int32_t* perm_in, int32_t* perm_out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (!perm_in || !perm_out || perm_in == perm_out) return SPARK_ERR_INVALID_ARG;
+  spark_reblock_layout pub;
+  spark_status st = spark_reblock_workspace_layout(H, N, d, block, &pub);
+  if (st != SPARK_OK) return st;
+  if (level < 0 || level >= pub.levels) return SPARK_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pub.total || !aligned(workspace, kAlign))
+    return SPARK_ERR_WORKSPACE;
+  const ReblockLayout L = reblock_layout(H, N, d, block);
+  cudaStream_t s = as_stream(stream);
+  if (upload_reblock_plan(N, block, workspace, L, s) != cudaSuccess) return SPARK_ERR_CUDA;
+  return from_cuda(launch_reblock_level(H, N, d, block, level, perm_in, perm_out, workspace, L, s));
+}
+
+spark_status spark_reblock(const void* Q, const void* K, int dtype, int H, int N, int d,
+                           int block, int mode, int32_t* q_perm, int32_t* k_perm,
+                           int32_t* offsets, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (!Q || !K || !q_perm || !k_perm || !offsets) return SPARK_ERR_INVALID_ARG;
+  if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  if (mode != SPARK_REBLOCK_Q_REUSE_K && mode != SPARK_REBLOCK_SEPARATE)
+    return SPARK_ERR_INVALID_ARG;
+  spark_reblock_layout pub;
+  spark_status st = spark_reblock_workspace_layout(H, N, d, block, &pub);
+  if (st != SPARK_OK) return st;
+  if (!aligned(Q, 16) || !aligned(K, 16)) return SPARK_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pub.total || !aligned(workspace, kAlign))
+    return SPARK_ERR_WORKSPACE;
+  const ReblockLayout L = reblock_layout(H, N, d, block);
+  cudaStream_t s = as_stream(stream);
+  if (launch_reblock_whiten(Q, K, dtype, H, N, d, workspace, L, s) != cudaSuccess ||
+      launch_reblock_partition(H, N, d, block, q_perm, workspace, L, s) != cudaSuccess)
+    return SPARK_ERR_CUDA;
+  if (mode == SPARK_REBLOCK_SEPARATE) {
+    if (launch_reblock_whiten(K, Q, dtype, H, N, d, workspace, L, s) != cudaSuccess ||
+        launch_reblock_partition(H, N, d, block, k_perm, workspace, L, s) != cudaSuccess)
+      return SPARK_ERR_CUDA;
+  } else if (cudaMemcpyAsync(k_perm, q_perm, static_cast<size_t>(H) * N * 4,
+                             cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
+    return SPARK_ERR_CUDA;
+  }
+  return from_cuda(launch_reblock_offsets(offsets, L.nb, N, block, s));
+}
+
 }  // extern "C"

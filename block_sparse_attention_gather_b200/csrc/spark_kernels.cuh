@@ -41,4 +41,30 @@ cudaError_t launch_attend(const AttendMaps& maps, int nc, const float* cbias,
                           int H, int N, int d, void* out, int out_dtype, uint32_t* err,
                           cudaStream_t s);
 
+// ---- Spark-Reblock partitioner (reblock.cu)
+// Byte offsets of its workspace regions (256-byte aligned).
+struct ReblockLayout {
+  size_t mpart, M, W, X, perm0, perm1, keys, meta, part, mu, v, hist, state, cnt, base, total;
+  int levels, nb;
+};
+
+ReblockLayout reblock_layout(int H, int N, int d, int block);
+size_t reblock_levels(int N, int block);
+
+// M = second moment of Yin's rows, W = M^{1/2}, workspace X = bf16 unit rows of W Xin.
+cudaError_t launch_reblock_whiten(const void* Xin, const void* Yin, int dtype, int H, int N,
+                                  int d, void* workspace, const ReblockLayout& L,
+                                  cudaStream_t s);
+// Copies the block tree's node / chunk tables into the workspace.
+cudaError_t upload_reblock_plan(int N, int block, void* workspace, const ReblockLayout& L,
+                                cudaStream_t s);
+// One level of splits of the workspace's X rows: perm_in -> perm_out ([H,N] positions).
+cudaError_t launch_reblock_level(int H, int N, int d, int block, int level,
+                                 const int32_t* perm_in, int32_t* perm_out, void* workspace,
+                                 const ReblockLayout& L, cudaStream_t s);
+// All levels from the identity order; the final permutation goes to perm_out.
+cudaError_t launch_reblock_partition(int H, int N, int d, int block, int32_t* perm_out,
+                                     void* workspace, const ReblockLayout& L, cudaStream_t s);
+cudaError_t launch_reblock_offsets(int32_t* offsets, int nb, int N, int block, cudaStream_t s);
+
 }  // namespace spark

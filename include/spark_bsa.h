@@ -225,6 +225,65 @@ SPARK_API spark_status spark_bsa_attend_ctx(const void* Qp, const void* Kp, cons
                                             int N, int d, void* out, int out_dtype,
                                             uint32_t* err, void* stream);
 
+/* ---- Spark-Reblock token partitioner ----
+ * Spark-H3 blog, section "Spark-Reblock": queries are grouped under the Mahalanobis cosine
+ * distance d_Q(q_i,q_j) = 1 - cos(M_K^{1/2} q_i, M_K^{1/2} q_j), M_K = E[k k^T] (keys
+ * symmetrically with M_Q), by a hierarchical partitioner that splits every group level by
+ * level into children of assigned capacities until every leaf is one block.  The blog does
+ * not spell out the split; the reading implemented here:
+ *   - fixed-size blocks of `block` tokens (the last takes the remainder), offsets shared by
+ *     all heads; a binary tree over the block range, the left child of an m-block node
+ *     holding ceil(m/2) blocks; a child's capacity is the tokens of its blocks;
+ *   - unit vectors x_i = W q_i / |W q_i| with W = M_K^{1/2} (symmetric square root; computed
+ *     by a fixed number of Newton-Schulz iterations in fp32; x stored as bf16);
+ *   - a node splits along its principal direction (4 power iterations of the node covariance
+ *     from (1,...,1)/sqrt(d)): its capacity-largest projections go left, equal projections to
+ *     the token earlier in the node's current order, both children keep the current order;
+ *   - the root order is 0..N-1; leaves in block order give the permutation.
+ * Mode SPARK_REBLOCK_Q_REUSE_K: keys reuse the query partition (the pages' released
+ * reblock_layout=q_reuse_k); SPARK_REBLOCK_SEPARATE: keys are partitioned the same way with
+ * Q and K swapped.  Deterministic (fixed-order sums, integer histograms). */
+#define SPARK_REBLOCK_Q_REUSE_K 0
+#define SPARK_REBLOCK_SEPARATE 1
+
+/* Workspace regions a caller may inspect after spark_reblock_whiten (byte offsets):
+ * M fp32 [H,d,d] second moment of the other side, W fp32 [H,d,d] = M^{1/2},
+ * X bf16 [H,N,d] unit rows; `levels` = depth of the block tree; `nb` = number of blocks. */
+typedef struct {
+  size_t M, W, X, total;
+  int levels, nb;
+} spark_reblock_layout;
+
+/* Fills *layout (pure host arithmetic).  1 <= block <= SPARK_MAX_BLOCK, d in {64,128},
+ * ceil(N/block) <= SPARK_MAX_NKB. */
+SPARK_API spark_status spark_reblock_workspace_layout(int H, int N, int d, int block,
+                                                      spark_reblock_layout* layout);
+SPARK_API size_t spark_reblock_workspace_size(int H, int N, int d, int block);
+/* Depth of the block tree (levels of splits) for N tokens, or -1 for invalid arguments. */
+SPARK_API int spark_reblock_levels(int N, int block);
+
+/* The partitioner.  Q, K: device [H,N,d] of `dtype`, 16-byte aligned.  Outputs (device):
+ * q_perm, k_perm [H,N] int32 (reblocked row i of head h is token perm[h,i]) and offsets
+ * [nb+1] int32 (fixed-size blocks), ready for spark_bsa_forward.  `workspace`: device,
+ * 256-byte aligned, spark_reblock_workspace_size bytes.  Asynchronous on `stream`. */
+SPARK_API spark_status spark_reblock(const void* Q, const void* K, int dtype, int H, int N, int d,
+                                     int block, int mode, int32_t* q_perm, int32_t* k_perm,
+                                     int32_t* offsets, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+/* Step: M = second moment of Y's rows, W = M^{1/2}, X = unit rows of W x_i into the
+ * workspace (offsets of spark_reblock_layout). */
+SPARK_API spark_status spark_reblock_whiten(const void* X, const void* Y, int dtype, int H, int N,
+                                            int d, int block, void* workspace,
+                                            size_t workspace_bytes, void* stream);
+
+/* Step: the splits of tree level `level` (0 = root) of the workspace's X rows: perm_in ->
+ * perm_out ([H,N] int32 device, distinct buffers; tokens of nodes that do not split at this
+ * level are copied). */
+SPARK_API spark_status spark_reblock_level(int H, int N, int d, int block, int level,
+                                           const int32_t* perm_in, int32_t* perm_out,
+                                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- Forward pass without any allocation ----
  * No counterpart in the pages: this entry point exists for callers that cannot allocate
  * device memory while they run (a memory budget owned by a host framework, work recorded into
