@@ -155,6 +155,30 @@ def test_context_entry_points_reject_bad_arguments(L):
                                   p, 0, None, None) == INVALID   # nc < 0
 
 
+def test_reblock_entry_points_reject_bad_arguments(L):
+    from block_sparse_attention_gather_b200 import (spark_reblock_levels,
+                                                    spark_reblock_workspace_layout,
+                                                    spark_reblock_workspace_size)
+    lay = spark_reblock_workspace_layout(24, 241920, 128, 128)
+    assert lay.nb == 1890 and lay.levels == 11
+    assert lay.X % 256 == 0 and lay.total >= lay.X + 24 * 241920 * 128 * 2
+    assert spark_reblock_levels(241920, 128) == 11
+    assert spark_reblock_levels(1, 64) == 0
+    assert spark_reblock_levels(0, 64) == -1
+    assert spark_reblock_workspace_size(2, 1000, 96, 64) == 0         # d unsupported
+    assert spark_reblock_workspace_size(2, 1000, 128, 129) == 0       # block > 128
+    p = ctypes.c_void_p(0x100000)
+    big = ctypes.c_size_t(1 << 40)
+    assert L.spark_reblock(p, p, 0, 2, 1000, 128, 64, 2, p, p, p, p, big, None) == INVALID   # mode
+    assert L.spark_reblock(p, p, 5, 2, 1000, 128, 64, 0, p, p, p, p, big, None) == INVALID   # dtype
+    assert L.spark_reblock(None, p, 0, 2, 1000, 128, 64, 0, p, p, p, p, big, None) == INVALID
+    assert L.spark_reblock(p, p, 0, 2, 1000, 128, 64, 0, p, p, p, p, 1024, None) == WORKSPACE
+    assert L.spark_reblock_level(2, 1000, 128, 64, 4, p, p, p, big, None) == INVALID    # in == out
+    q = ctypes.c_void_p(0x200000)
+    assert L.spark_reblock_level(2, 1000, 128, 64, 99, p, q, p, big, None) == INVALID   # level
+    assert L.spark_reblock_whiten(p, p, 0, 2, 1000, 64, 64, p, 16, None) == WORKSPACE
+
+
 def test_missing_library_fails_loudly(tmp_path):
     code = ("import block_sparse_attention_gather_b200._native as n;"
             f"n.LIB_PATH = {str(tmp_path / 'nope.so')!r};"
