@@ -40,6 +40,7 @@ constexpr int kChunk = 1024;        // tokens of one node handled by one CTA
 constexpr int kPowerIters = 4;
 constexpr int kNsIters = 40;        // Newton-Schulz iterations (fixed)
 constexpr int kMomentParts = 16;    // row partitions of the second-moment sum per head
+constexpr int kRowsInFlight = 8;    // unit rows a warp loads before using them
 
 __device__ __forceinline__ uint32_t rb_order_key(float f) {
   const uint32_t u = __float_as_uint(f);
@@ -53,20 +54,6 @@ __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
-}
-
-// R = D/32 consecutive bf16 of a unit-vector row, as fp32.
-template <int R>
-__device__ __forceinline__ void load_row_part(const __nv_bfloat16* p, float (&x)[R]) {
-  if constexpr (R == 4) {
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
-    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
-    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
-    x[0] = __low2float(a); x[1] = __high2float(a); x[2] = __low2float(b); x[3] = __high2float(b);
-  } else {
-    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(p);
-    x[0] = __low2float(a); x[1] = __high2float(a);
-  }
 }
 
 }  // namespace
@@ -292,45 +279,97 @@ __global__ void __launch_bounds__(kRbThreads) rb_whiten_kernel(const T* __restri
 // positions, with one sentinel node whose chunk0 is the level's chunk count; chunks[c] =
 // (node, start, end, 0).
 
-// Pass over a chunk: sum of (x.v) x (and of x on the first pass), per warp in position order,
-// then over the warps in order.
+// Lanes per token in the level passes: lane group g of a warp handles one token, lane s of
+// the group the DPL = D / 8 dimensions [s*DPL, (s+1)*DPL) of it (two or one 16-byte loads).
+constexpr int kLanesPerTok = 8;
+constexpr int kTokPerWarp = 32 / kLanesPerTok;
+
+template <int DPL>
+__device__ __forceinline__ void load_dims(const __nv_bfloat16* p, uint32_t (&w)[DPL / 2]) {
+#pragma unroll
+  for (int q = 0; q < DPL / 8; ++q)
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w[4 * q]), "=r"(w[4 * q + 1]), "=r"(w[4 * q + 2]), "=r"(w[4 * q + 3])
+                 : "l"(p + 8 * q));
+}
+
+template <int DPL>
+__device__ __forceinline__ float group_dot(const uint32_t (&w)[DPL / 2], const float (&v)[DPL],
+                                           float (&x)[DPL]) {
+  float y = 0.f;
+#pragma unroll
+  for (int i = 0; i < DPL / 2; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    y = fmaf(x[2 * i], v[2 * i], y);
+    y = fmaf(x[2 * i + 1], v[2 * i + 1], y);
+  }
+#pragma unroll
+  for (int o = 1; o < kLanesPerTok; o <<= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
+  return y;
+}
+
+// Pass over a chunk: sum of (x.v) x (and of x on the first pass).  Tokens are taken in a
+// fixed order (warp, step, group) and the partial sums are reduced over groups and then
+// warps in a fixed order.
 template <int D, bool kFirst>
 __global__ void __launch_bounds__(kRbThreads) rb_power_kernel(
     const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm, int N,
     const int4* __restrict__ chunks, int nch, const float* __restrict__ vnode, int nnodes,
     float* __restrict__ part) {
-  constexpr int R = D / 32;
+  constexpr int DPL = D / kLanesPerTok;
+  constexpr int U = kRowsInFlight / 2;                     // steps of 4 tokens in flight
   __shared__ float red[kRbWarps][2 * D];
+  __shared__ int toks[kChunk];                             // the chunk's token ids, staged once
   const int c = blockIdx.x, h = blockIdx.y, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int grp = lane / kLanesPerTok, sub = lane % kLanesPerTok;
   const int4 ch = chunks[c];
-  float v[R];
+  for (int i = threadIdx.x; i < ch.z - ch.y; i += kRbThreads)
+    toks[i] = min(max(perm[static_cast<size_t>(h) * N + ch.y + i], 0), N - 1);
+  float v[DPL];
 #pragma unroll
-  for (int j = 0; j < R; ++j)
+  for (int j = 0; j < DPL; ++j)
     v[j] = kFirst ? rsqrtf(static_cast<float>(D))
-                  : vnode[(static_cast<size_t>(h) * nnodes + ch.x) * D + lane * R + j];
-  float sxv[R], sx[R];
+                  : vnode[(static_cast<size_t>(h) * nnodes + ch.x) * D + sub * DPL + j];
+  __syncthreads();
+  float sxv[DPL], sx[DPL];
 #pragma unroll
-  for (int j = 0; j < R; ++j) sxv[j] = sx[j] = 0.f;
-  const int32_t* ph = perm + static_cast<size_t>(h) * N;
-  const __nv_bfloat16* Xh = X + static_cast<size_t>(h) * N * D;
-  for (int pos = ch.y + warp; pos < ch.z; pos += kRbWarps) {
-    const int tok = min(max(ph[pos], 0), N - 1);
-    float x[R];
-    load_row_part<R>(Xh + static_cast<size_t>(tok) * D + lane * R, x);
-    float y = 0.f;
+  for (int j = 0; j < DPL; ++j) sxv[j] = sx[j] = 0.f;
+  const __nv_bfloat16* Xh = X + static_cast<size_t>(h) * N * D + sub * DPL;
+  for (int p0 = ch.y + warp * kTokPerWarp * U; p0 < ch.z; p0 += kRbWarps * kTokPerWarp * U) {
+    uint32_t raw[U][DPL / 2];
 #pragma unroll
-    for (int j = 0; j < R; ++j) y = fmaf(x[j], v[j], y);
-    y = warp_sum(y);
+    for (int u = 0; u < U; ++u) {                          // U x 4 row loads in flight
+      const int pos = min(p0 + u * kTokPerWarp + grp, ch.z - 1);
+      load_dims<DPL>(Xh + static_cast<size_t>(toks[pos - ch.y]) * D, raw[u]);
+    }
 #pragma unroll
-    for (int j = 0; j < R; ++j) {
-      sxv[j] = fmaf(y, x[j], sxv[j]);
-      if (kFirst) sx[j] += x[j];
+    for (int u = 0; u < U; ++u) {
+      float x[DPL];
+      const float y = group_dot<DPL>(raw[u], v, x);
+      if (p0 + u * kTokPerWarp + grp < ch.z) {
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) {
+          sxv[j] = fmaf(y, x[j], sxv[j]);
+          if (kFirst) sx[j] += x[j];
+        }
+      }
     }
   }
+  // groups -> lanes 0..7 of the warp, in a fixed order
 #pragma unroll
-  for (int j = 0; j < R; ++j) {
-    red[warp][lane * R + j] = sxv[j];
-    red[warp][D + lane * R + j] = sx[j];
+  for (int o = kLanesPerTok; o < 32; o <<= 1)
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) {
+      sxv[j] += __shfl_xor_sync(0xffffffffu, sxv[j], o);
+      if (kFirst) sx[j] += __shfl_xor_sync(0xffffffffu, sx[j], o);
+    }
+  if (grp == 0) {
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) {
+      red[warp][sub * DPL + j] = sxv[j];
+      red[warp][D + sub * DPL + j] = sx[j];
+    }
   }
   __syncthreads();
   for (int t = threadIdx.x; t < (kFirst ? 2 * D : D); t += kRbThreads) {
@@ -388,29 +427,39 @@ __global__ void __launch_bounds__(kRbThreads) rb_project_kernel(
     const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm, int N,
     const int4* __restrict__ chunks, const float* __restrict__ vnode, int nnodes,
     uint32_t* __restrict__ keys, uint32_t* __restrict__ hist) {
-  constexpr int R = D / 32;
+  constexpr int DPL = D / kLanesPerTok;
+  constexpr int U = kRowsInFlight / 2;
   __shared__ uint32_t sh[256];
+  __shared__ int toks[kChunk];
   const int c = blockIdx.x, h = blockIdx.y, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int grp = lane / kLanesPerTok, sub = lane % kLanesPerTok;
   const int4 ch = chunks[c];
   sh[threadIdx.x] = 0u;
-  float v[R];
+  for (int i = threadIdx.x; i < ch.z - ch.y; i += kRbThreads)
+    toks[i] = min(max(perm[static_cast<size_t>(h) * N + ch.y + i], 0), N - 1);
+  float v[DPL];
 #pragma unroll
-  for (int j = 0; j < R; ++j) v[j] = vnode[(static_cast<size_t>(h) * nnodes + ch.x) * D + lane * R + j];
+  for (int j = 0; j < DPL; ++j)
+    v[j] = vnode[(static_cast<size_t>(h) * nnodes + ch.x) * D + sub * DPL + j];
   __syncthreads();
-  const int32_t* ph = perm + static_cast<size_t>(h) * N;
-  const __nv_bfloat16* Xh = X + static_cast<size_t>(h) * N * D;
-  for (int pos = ch.y + warp; pos < ch.z; pos += kRbWarps) {
-    const int tok = min(max(ph[pos], 0), N - 1);
-    float x[R];
-    load_row_part<R>(Xh + static_cast<size_t>(tok) * D + lane * R, x);
-    float y = 0.f;
+  const __nv_bfloat16* Xh = X + static_cast<size_t>(h) * N * D + sub * DPL;
+  for (int p0 = ch.y + warp * kTokPerWarp * U; p0 < ch.z; p0 += kRbWarps * kTokPerWarp * U) {
+    uint32_t raw[U][DPL / 2];
 #pragma unroll
-    for (int j = 0; j < R; ++j) y = fmaf(x[j], v[j], y);
-    y = warp_sum(y);
-    if (lane == 0) {
-      const uint32_t key = rb_order_key(y);
-      keys[static_cast<size_t>(h) * N + pos] = key;
-      atomicAdd(&sh[key >> 24], 1u);
+    for (int u = 0; u < U; ++u) {
+      const int pos = min(p0 + u * kTokPerWarp + grp, ch.z - 1);
+      load_dims<DPL>(Xh + static_cast<size_t>(toks[pos - ch.y]) * D, raw[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float x[DPL];
+      const float y = group_dot<DPL>(raw[u], v, x);
+      const int pos = p0 + u * kTokPerWarp + grp;
+      if (sub == 0 && pos < ch.z) {
+        const uint32_t key = rb_order_key(y);
+        keys[static_cast<size_t>(h) * N + pos] = key;
+        atomicAdd(&sh[key >> 24], 1u);
+      }
     }
   }
   __syncthreads();
