@@ -346,10 +346,11 @@ REBLOCK_METRIC = "ms/call of the Spark-Reblock partitioner (q_reuse_k), 768p sha
 
 
 def reblock_bytes_flops(H, N, d, levels, e_in, power_iters=4):
-    """Algorithmic work of one partitioner call: fp32 FMAs of the second moment and of the
-    whitening (2 H N d^2 flops each), and HBM bytes of the per-level passes over the bf16
-    unit rows (power_iters + 1 reads of X with the perm index per level) plus the keys,
-    histogram and scatter passes (4 + 4 + 4 + 8 bytes per token and level)."""
+    """Algorithmic work of one partitioner call: the flops of the second moment and of the
+    whitening (2 H N d^2 each; bf16 tensor-core MMAs for bf16 inputs), the HBM bytes of the
+    whitening (read Q and K, write the bf16 unit rows), and the HBM bytes of the per-level
+    passes over the unit rows (power_iters + 1 reads with the token index per level) plus the
+    keys, histogram and scatter passes (4 + 4 + 4 + 8 bytes per token and level)."""
     flops = 2 * 2.0 * H * N * d * d
     prep_bytes = 2.0 * H * N * d * e_in + H * N * d * 2
     level_bytes = levels * H * N * ((power_iters + 1) * (2 * d + 4) + 4 + 3 * 4 + 4 + 8)
@@ -427,8 +428,8 @@ def run_reblock(args, world, rank, local):
     line = {
         "impl": "ours", "op": "reblock", "metric": REBLOCK_METRIC, "value": ms, "unit": "ms",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic",
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if Q.dtype == torch.bfloat16 else "f32", "data": "synthetic",
         "config": {"workload": w.name, "H": H, "N": N, "d": d, "block": block,
                    "levels": lay.levels, "mode": "q_reuse_k", "power_iters": 4,
                    "l2": "inputs larger than L2, no flush"},
@@ -437,11 +438,14 @@ def run_reblock(args, world, rank, local):
                      "kernel": "per-level passes (power, project, select, scatter)",
                      "algorithmic_bytes_per_call": level_bytes},
         "kernels": {"whiten (second moment, M^1/2, unit rows)": {
-                        "ms": prep_ms, "fp32_tflops": flops / (prep_ms / 1e3) / 1e12,
-                        "flops": flops, "bytes": prep_bytes},
+                        "ms": prep_ms, "TFLOP/s": flops / (prep_ms / 1e3) / 1e12,
+                        "flops": flops, "bytes": prep_bytes,
+                        "GB/s": prep_bytes / (prep_ms / 1e3) / 1e9,
+                        "units": ("tcgen05 bf16 MMAs, fp32 accumulation" if
+                                  Q.dtype == torch.bfloat16 and d == 128 else "fp32 CUDA cores")},
                     "levels": {"ms": part_ms, "GB/s": gbs, "bytes": level_bytes}},
         # per call: 4 whitening kernels, the identity order, 19 kernels per level, offsets
-        "gpu_launches": (6 + 19 * lay.levels) * args.steps,
+        "gpu_launches": (6 + 19 * lay.levels) * args.steps,  # + 0: same count on either path
         "clocks": clock_info,
     }
     if rank == 0:

@@ -10,33 +10,7 @@
 
 using namespace spark;
 
-namespace {
-
-constexpr size_t kAlign = 256;
-
-size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
-
-bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
-cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
-
-int topk_count(int nkb, double ratio) {
-  if (nkb < 1 || !(ratio > 0.0) || !(ratio <= 1.0)) return -1;
-  double kk = std::ceil(ratio * static_cast<double>(nkb) - 1e-9);
-  int k = static_cast<int>(kk);
-  if (k < 1) k = 1;
-  if (k > nkb) k = nkb;
-  return k;
-}
-
-spark_status check_sizes(int H, int N, int d, int nqb, int nkb) {
-  if (H < 1 || N < 1 || nqb < 1 || nkb < 1 || nqb > N || nkb > N) return SPARK_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return SPARK_ERR_UNSUPPORTED;
-  if (H > 65535 || nkb > kMaxNkb) return SPARK_ERR_UNSUPPORTED;
-  return SPARK_OK;
-}
-
-spark_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA; }
+namespace spark {
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -67,6 +41,36 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int H, int rows, int d) {
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+}  // namespace spark
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+int topk_count(int nkb, double ratio) {
+  if (nkb < 1 || !(ratio > 0.0) || !(ratio <= 1.0)) return -1;
+  double kk = std::ceil(ratio * static_cast<double>(nkb) - 1e-9);
+  int k = static_cast<int>(kk);
+  if (k < 1) k = 1;
+  if (k > nkb) k = nkb;
+  return k;
+}
+
+spark_status check_sizes(int H, int N, int d, int nqb, int nkb) {
+  if (H < 1 || N < 1 || nqb < 1 || nkb < 1 || nqb > N || nkb > N) return SPARK_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SPARK_ERR_UNSUPPORTED;
+  if (H > 65535 || nkb > kMaxNkb) return SPARK_ERR_UNSUPPORTED;
+  return SPARK_OK;
+}
+
+spark_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA; }
 
 spark_status layout_of(int H, int N, int d, int nqb, int nkb, double ratio,
                        spark_bsa_layout* L) {

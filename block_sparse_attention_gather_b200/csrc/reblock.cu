@@ -26,6 +26,7 @@
 //             rb_count, rb_scan, rb_scatter            stable two-way partition of perm
 // Everything is deterministic: sums run in a fixed order, histograms are integer counts.
 #include <cmath>
+#include <type_traits>
 #include <vector>
 
 #include "spark_kernels.cuh"
@@ -38,7 +39,8 @@ constexpr int kRbThreads = 256;
 constexpr int kRbWarps = kRbThreads / 32;
 constexpr int kChunk = 1024;        // tokens of one node handled by one CTA
 constexpr int kPowerIters = 4;
-constexpr int kNsIters = 40;        // Newton-Schulz iterations (fixed)
+constexpr int kNsIters = 40;        // Newton-Schulz iterations at most
+constexpr float kNsTol = 1e-5f;     // stop once max |Z Y - I| is below this
 constexpr int kMomentParts = 16;    // row partitions of the second-moment sum per head
 constexpr int kRowsInFlight = 8;    // unit rows a warp loads before using them
 
@@ -122,32 +124,46 @@ __global__ void __launch_bounds__(kRbThreads) rb_moment_reduce_kernel(const floa
 }
 
 // ------------------------------------------------------------------ W = M^{1/2}
-// Coupled Newton-Schulz iteration (stable form): with c = trace(M) (>= the largest eigenvalue
+// Coupled Newton-Schulz iteration (stable form): with c = |M|_F (>= the largest eigenvalue
 // of a PSD M), Y0 = M/c, Z0 = I, T = (3I - Z Y)/2, Y <- Y T, Z <- T Z; Y converges to
-// (M/c)^{1/2} and W = sqrt(c) Y.  Zero eigenvalues stay zero.  One CTA per head, the three
-// D x D matrices in shared memory; thread (rg, cg) owns a RT x CT tile of every product.
+// (M/c)^{1/2} and W = sqrt(c) Y.  Zero eigenvalues stay zero.  The loop stops once
+// max |Z Y - I| < kNsTol (a block-wide decision, so the count depends only on M) or after
+// kNsIters steps.  One CTA per head, the three D x D matrices in shared memory; thread
+// (rg, cg) owns a RT x CT tile of every product.
 template <int D>
 __global__ void __launch_bounds__(512) rb_sqrt_kernel(const float* __restrict__ M,
-                                                      float* __restrict__ W) {
+                                                      float* __restrict__ W,
+                                                      __nv_bfloat16* __restrict__ Wb) {
   constexpr int RT = D / 32, CT = D / 16;                 // 4 x 8 (D=128) or 2 x 4 (D=64)
   extern __shared__ __align__(16) float rb_sm[];
   float* Ys = rb_sm;
   float* Zs = Ys + D * D;
   float* Ts = Zs + D * D;
   __shared__ float s_c;
+  __shared__ float s_red[16];
   const int h = blockIdx.x, tid = threadIdx.x;
   const float* Mh = M + static_cast<size_t>(h) * D * D;
   float* Wh = W + static_cast<size_t>(h) * D * D;
-  if (tid < 32) {
+  {
     float t = 0.f;
-    for (int i = tid; i < D; i += 32) t += Mh[i * D + i];
+    for (int i = tid; i < D * D; i += 512) t = fmaf(Mh[i], Mh[i], t);
     t = warp_sum(t);
-    if (tid == 0) s_c = t;
+    if (tid % 32 == 0) s_red[tid / 32] = t;
+    __syncthreads();
+    if (tid == 0) {
+      float a = 0.f;
+      for (int w = 0; w < 16; ++w) a += s_red[w];
+      s_c = sqrtf(a);
+    }
   }
   __syncthreads();
   const float c = s_c;
+  __nv_bfloat16* Wbh = Wb + static_cast<size_t>(h) * D * D;
   if (!(c > 0.f) || !isfinite(c)) {
-    for (int idx = tid; idx < D * D; idx += 512) Wh[idx] = 0.f;
+    for (int idx = tid; idx < D * D; idx += 512) {
+      Wh[idx] = 0.f;
+      Wbh[idx] = __float2bfloat16_rn(0.f);
+    }
     return;
   }
   const float invc = 1.f / c;
@@ -181,12 +197,23 @@ __global__ void __launch_bounds__(512) rb_sqrt_kernel(const float* __restrict__ 
   float acc[RT][CT], acc2[RT][CT];
   for (int it = 0; it < kNsIters; ++it) {
     mm(Zs, Ys, acc);                                         // T = (3I - Z Y) / 2
+    float dev = 0.f;
 #pragma unroll
     for (int i = 0; i < RT; ++i)
 #pragma unroll
-      for (int j = 0; j < CT; ++j)
-        Ts[(r0 + i) * D + c0 + j] = 0.5f * (((r0 + i) == (c0 + j) ? 3.f : 0.f) - acc[i][j]);
+      for (int j = 0; j < CT; ++j) {
+        const float id = (r0 + i) == (c0 + j) ? 1.f : 0.f;
+        dev = fmaxf(dev, fabsf(acc[i][j] - id));
+        Ts[(r0 + i) * D + c0 + j] = 0.5f * (3.f * id - acc[i][j]);
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, o));
+    if (tid % 32 == 0) s_red[tid / 32] = dev;
     __syncthreads();
+    float mx = 0.f;
+    for (int w = 0; w < 16; ++w) mx = fmaxf(mx, s_red[w]);
+    if (mx < kNsTol) break;                                  // uniform: every thread sees mx
+    __syncthreads();                                         // s_red is rewritten next step
     mm(Ys, Ts, acc);                                         // Y T
     mm(Ts, Zs, acc2);                                        // T Z
     __syncthreads();
@@ -200,7 +227,252 @@ __global__ void __launch_bounds__(512) rb_sqrt_kernel(const float* __restrict__ 
     __syncthreads();
   }
   const float sc = sqrtf(c);
-  for (int idx = tid; idx < D * D; idx += 512) Wh[idx] = Ys[idx] * sc;
+  for (int idx = tid; idx < D * D; idx += 512) {
+    Wh[idx] = Ys[idx] * sc;
+    Wbh[idx] = __float2bfloat16_rn(Ys[idx] * sc);
+  }
+}
+
+// ------------------------------------------------------------------ tensor-core whitening
+// bf16 inputs with d = 128 take these two tcgen05 kernels instead of the CUDA-core ones.
+// Tiles are 128 tokens x 128 dims, loaded by TMA with 128-byte swizzle (two 64-column atoms).
+
+constexpr int kTcTile = 128 * 128 * 2;          // bytes of one bf16 tile
+constexpr int kMomStages = 4;
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) &
+                                    ~static_cast<uintptr_t>(1023));
+}
+
+__device__ __forceinline__ bool rb_wait_quiet(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_test(bar, parity))
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  return true;
+}
+
+// part[h][p] = sum over the CTA's token tiles of Y^T Y: A = tile^T and B = tile, both read
+// MN-major from the same shared-memory tile; the 128 x 128 fp32 sum stays in TMEM.
+__global__ void __launch_bounds__(128) rb_moment_tc_kernel(const __grid_constant__ CUtensorMap map_y,
+                                                           int tiles, float* __restrict__ part,
+                                                           uint32_t* __restrict__ err) {
+  extern __shared__ uint8_t rb_tc_raw[];
+  uint8_t* st = align1024(rb_tc_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(st + kMomStages * kTcTile);
+  uint64_t* empty = full + kMomStages;
+  uint64_t* done = empty + kMomStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int p = blockIdx.x, P = gridDim.x, h = blockIdx.y, tid = threadIdx.x, warp = tid / 32;
+  const int t0 = static_cast<int>(static_cast<long long>(tiles) * p / P);
+  const int T = static_cast<int>(static_cast<long long>(tiles) * (p + 1) / P) - t0;
+  if (tid == 0) {
+    for (int s = 0; s < kMomStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tbase = *tmem_slot;
+  if (tid == 0) {
+    constexpr uint32_t idM = idesc_bf16(128, 128, true, true);
+    tma_prefetch_desc(&map_y);
+    int issued = 0;
+    auto load = [&](int t) {
+      const int s = t % kMomStages;
+      mbar_arrive_expect_tx(&full[s], kTcTile);
+      for (int a = 0; a < 2; ++a)
+        tma_load_3d(st + s * kTcTile + a * 16384, &map_y, &full[s], a * 64, (t0 + t) * 128, h);
+      issued = t + 1;
+    };
+    for (int t = 0; t < min(T, kMomStages); ++t) load(t);
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int s = t % kMomStages;
+      if (!mbar_wait(&full[s], (t / kMomStages) & 1, abort_flag, err)) { ok = false; break; }
+      tc_fence_after_sync();
+      const uint64_t d0 = sdesc_sw128(smem_u32(st + s * kTcTile), 16384, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t dk = d0 + static_cast<uint64_t>((kk * 2048) >> 4);
+        mma_ss(tbase, dk, dk, idM, (t > 0 || kk > 0) ? 1u : 0u);
+      }
+      tc_commit(&empty[s]);
+      if (t + kMomStages < T) {
+        if (!mbar_wait(&empty[s], (t / kMomStages) & 1, abort_flag, err)) { ok = false; break; }
+        load(t + kMomStages);
+      }
+    }
+    if (!ok)                                               // drain the loads still in flight
+      for (int t = max(0, issued - kMomStages); t < issued; ++t)
+        rb_wait_quiet(&full[t % kMomStages], (t / kMomStages) & 1);
+    tc_commit(done);
+    rb_wait_quiet(done, 0);
+  }
+  __syncthreads();
+  const bool fine = !*abort_flag;
+  tc_fence_after_sync();
+  float* out = part + (static_cast<size_t>(h) * P + p) * 128 * 128;
+  const int row = warp * 32 + (tid % 32);
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t r[32];
+    if (T > 0 && fine) {
+      tmem_ld32(tbase + (static_cast<uint32_t>(warp * 32) << 16) + cc * 32, r);
+    } else {
+      for (int j = 0; j < 32; ++j) r[j] = 0u;
+    }
+    float4* dst = reinterpret_cast<float4*>(out + row * 128 + cc * 32);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                           __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tbase, 128);
+  }
+}
+
+// X rows = bf16(unit(W y)) for the CTA's token tiles: A = Y tile and B = W (both K-major), two
+// TMEM accumulators; warps 0-3 normalise and store one row per thread while warp 4 (one
+// thread) loads and issues the next tile.
+__global__ void __launch_bounds__(160) rb_whiten_tc_kernel(const __grid_constant__ CUtensorMap map_y,
+                                                           const __grid_constant__ CUtensorMap map_w,
+                                                           int N, int tiles,
+                                                           __nv_bfloat16* __restrict__ X,
+                                                           uint32_t* __restrict__ err) {
+  extern __shared__ uint8_t rb_tc_raw[];
+  uint8_t* wst = align1024(rb_tc_raw);
+  uint8_t* yst = wst + kTcTile;                          // 2 stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(yst + 2 * kTcTile);
+  uint64_t* wfull = bars;
+  uint64_t* yfull = bars + 1;                            // [2]
+  uint64_t* yempty = bars + 3;                           // [2]
+  uint64_t* accfull = bars + 5;                          // [2]
+  uint64_t* accempty = bars + 7;                         // [2], count 128
+  uint64_t* done = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int h = blockIdx.y, tid = threadIdx.x, warp = tid / 32;
+  const int t0 = static_cast<int>(static_cast<long long>(tiles) * blockIdx.x / gridDim.x);
+  const int T = static_cast<int>(static_cast<long long>(tiles) * (blockIdx.x + 1) / gridDim.x) - t0;
+  if (tid == 0) {
+    mbar_init(wfull, 1);
+    mbar_init(done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&yfull[b], 1);
+      mbar_init(&yempty[b], 1);
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 128);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tbase = *tmem_slot;
+  if (warp == 4) {
+    if ((tid % 32) == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
+      tma_prefetch_desc(&map_y);
+      tma_prefetch_desc(&map_w);
+      mbar_arrive_expect_tx(wfull, kTcTile);
+      for (int a = 0; a < 2; ++a) tma_load_3d(wst + a * 16384, &map_w, wfull, a * 64, 0, h);
+      int issued = 0;
+      auto load = [&](int t) {
+        const int s = t & 1;
+        mbar_arrive_expect_tx(&yfull[s], kTcTile);
+        for (int a = 0; a < 2; ++a)
+          tma_load_3d(yst + s * kTcTile + a * 16384, &map_y, &yfull[s], a * 64, (t0 + t) * 128, h);
+        issued = t + 1;
+      };
+      for (int t = 0; t < min(T, 2); ++t) load(t);
+      bool ok = mbar_wait(wfull, 0, abort_flag, err);
+      const uint64_t wd = sdesc_sw128(smem_u32(wst), 16, 1024);
+      for (int t = 0; ok && t < T; ++t) {
+        const int s = t & 1;
+        if (!mbar_wait(&yfull[s], (t >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (t >= 2 && !mbar_wait(&accempty[s], ((t >> 1) - 1) & 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint64_t yd = sdesc_sw128(smem_u32(yst + s * kTcTile), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) / 16;
+          mma_ss(tbase + s * 128, yd + off, wd + off, idS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&accfull[s]);
+        tc_commit(&yempty[s]);
+        if (t + 2 < T) {
+          if (!mbar_wait(&yempty[s], (t >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          load(t + 2);
+        }
+      }
+      if (!ok) {
+        for (int t = max(0, issued - 2); t < issued; ++t) rb_wait_quiet(&yfull[t & 1], (t >> 1) & 1);
+        rb_wait_quiet(wfull, 0);
+      }
+      tc_commit(done);                                     // no MMA left in flight before TMEM
+      rb_wait_quiet(done, 0);                              // is freed
+    }
+  } else {
+    const int row = tid;                                 // TMEM lane = token row of the tile
+    for (int t = 0; t < T; ++t) {
+      const int b = t & 1;
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&accfull[b], (t >> 1) & 1, abort_flag, err));
+      if (!got) break;
+      tc_fence_after_sync();
+      float v[128];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tbase + (static_cast<uint32_t>(warp * 32) << 16) + b * 128 + cc * 32, r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[cc * 32 + j] = __uint_as_float(r[j]);
+      }
+      tc_fence_before_sync();
+      mbar_arrive(&accempty[b]);                         // accumulator b may be reused
+      float ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < 128; ++j) ss = fmaf(v[j], v[j], ss);
+      const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+      const int tok = (t0 + t) * 128 + row;
+      if (tok < N) {
+        uint4* dst = reinterpret_cast<uint4*>(X + (static_cast<size_t>(h) * N + tok) * 128);
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          dst[q] = make_uint4(pack_bf16(v[8 * q] * inv, v[8 * q + 1] * inv),
+                              pack_bf16(v[8 * q + 2] * inv, v[8 * q + 3] * inv),
+                              pack_bf16(v[8 * q + 4] * inv, v[8 * q + 5] * inv),
+                              pack_bf16(v[8 * q + 6] * inv, v[8 * q + 7] * inv));
+      }
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tbase, 256);
+  }
 }
 
 // ------------------------------------------------------------------ whitening
@@ -726,6 +998,7 @@ ReblockLayout reblock_layout(int H, int N, int d, int block) {
   L.mpart = take(static_cast<size_t>(H) * kMomentParts * dd * 4);
   L.M = take(static_cast<size_t>(H) * dd * 4);
   L.W = take(static_cast<size_t>(H) * dd * 4);
+  L.Wb = take(static_cast<size_t>(H) * dd * 2);
   L.X = take(static_cast<size_t>(H) * N * d * 2);
   L.perm0 = take(static_cast<size_t>(H) * N * 4);
   L.perm1 = take(static_cast<size_t>(H) * N * 4);
@@ -739,11 +1012,15 @@ ReblockLayout reblock_layout(int H, int N, int d, int block) {
   L.state = take(static_cast<size_t>(H) * mn * 2 * 4);
   L.cnt = take(static_cast<size_t>(H) * mc * 2 * 4);
   L.base = take(static_cast<size_t>(H) * mc * 3 * 4);
+  L.err = take(4);
   L.total = off;
   L.levels = static_cast<int>(P.levels.size());
   L.nb = P.nb;
   return L;
 }
+
+constexpr int kMomentTcParts = 6;     // token-tile partitions per head on the tensor cores
+constexpr int kWhitenTcTiles = 16;    // token tiles per CTA of the tensor-core whitening
 
 template <int D, typename T>
 static cudaError_t whiten_t(const void* Xin, const void* Yin, int H, int N, uint8_t* ws,
@@ -751,23 +1028,52 @@ static cudaError_t whiten_t(const void* Xin, const void* Yin, int H, int N, uint
   float* part = reinterpret_cast<float*>(ws + L.mpart);
   float* M = reinterpret_cast<float*>(ws + L.M);
   float* W = reinterpret_cast<float*>(ws + L.W);
+  auto* Wb = reinterpret_cast<__nv_bfloat16*>(ws + L.Wb);
   auto* X = reinterpret_cast<__nv_bfloat16*>(ws + L.X);
-  rb_moment_partial_kernel<D, T><<<dim3(kMomentParts, H), kRbThreads, 0, s>>>(
-      static_cast<const T*>(Yin), N, part);
-  rb_moment_reduce_kernel<D><<<H, kRbThreads, 0, s>>>(part, kMomentParts, N, M);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.err);
+  constexpr bool kTc = (D == 128) && std::is_same<T, __nv_bfloat16>::value;
+  const int tiles = (N + 127) / 128;
+  CUtensorMap map_x, map_y, map_w;
+  if constexpr (kTc) {
+    if (!encode_rows_map(&map_x, Xin, H, N, D) || !encode_rows_map(&map_y, Yin, H, N, D) ||
+        !encode_rows_map(&map_w, Wb, H, D, D))
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaMemsetAsync(err, 0, 4, s);
+  if (e != cudaSuccess) return e;
+  if constexpr (kTc) {
+    const size_t smem = 1024 + kMomStages * kTcTile + 2 * kMomStages * 8 + 8 + 16;
+    e = cudaFuncSetAttribute(rb_moment_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    rb_moment_tc_kernel<<<dim3(kMomentTcParts, H), 128, smem, s>>>(map_y, tiles, part, err);
+    rb_moment_reduce_kernel<D><<<H, kRbThreads, 0, s>>>(part, kMomentTcParts, N, M);
+  } else {
+    rb_moment_partial_kernel<D, T><<<dim3(kMomentParts, H), kRbThreads, 0, s>>>(
+        static_cast<const T*>(Yin), N, part);
+    rb_moment_reduce_kernel<D><<<H, kRbThreads, 0, s>>>(part, kMomentParts, N, M);
+  }
   const size_t sq_smem = 3 * D * D * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(rb_sqrt_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(sq_smem));
+  e = cudaFuncSetAttribute(rb_sqrt_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sq_smem));
   if (e != cudaSuccess) return e;
-  rb_sqrt_kernel<D><<<H, 512, sq_smem, s>>>(M, W);
-  const size_t wh_smem = (D * D + kRbWarps * 8 * D) * sizeof(float);
-  e = cudaFuncSetAttribute(rb_whiten_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(wh_smem));
-  if (e != cudaSuccess) return e;
-  const int tok_per_cta = kRbWarps * 8 * 4;
-  rb_whiten_kernel<D, T><<<dim3((N + tok_per_cta - 1) / tok_per_cta, H), kRbThreads, wh_smem, s>>>(
-      static_cast<const T*>(Xin), W, N, X);
+  rb_sqrt_kernel<D><<<H, 512, sq_smem, s>>>(M, W, Wb);
+  if constexpr (kTc) {
+    const size_t smem = 1024 + 3 * kTcTile + 11 * 8 + 16;
+    e = cudaFuncSetAttribute(rb_whiten_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int ctas = (tiles + kWhitenTcTiles - 1) / kWhitenTcTiles;
+    rb_whiten_tc_kernel<<<dim3(ctas, H), 160, smem, s>>>(map_x, map_w, N, tiles, X, err);
+  } else {
+    const size_t wh_smem = (D * D + kRbWarps * 8 * D) * sizeof(float);
+    e = cudaFuncSetAttribute(rb_whiten_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(wh_smem));
+    if (e != cudaSuccess) return e;
+    const int tok_per_cta = kRbWarps * 8 * 4;
+    rb_whiten_kernel<D, T><<<dim3((N + tok_per_cta - 1) / tok_per_cta, H), kRbThreads, wh_smem,
+                             s>>>(static_cast<const T*>(Xin), W, N, X);
+  }
   return cudaGetLastError();
 }
 

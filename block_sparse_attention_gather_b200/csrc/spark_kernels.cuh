@@ -41,10 +41,14 @@ cudaError_t launch_attend(const AttendMaps& maps, int nc, const float* cbias,
                           int H, int N, int d, void* out, int out_dtype, uint32_t* err,
                           cudaStream_t s);
 
+// 3-D bf16 tensor map [H][rows][d], box 64 columns x 128 rows, 128-byte swizzle (api.cu).
+bool encode_rows_map(CUtensorMap* m, const void* base, int H, int rows, int d);
+
 // ---- Spark-Reblock partitioner (reblock.cu)
 // Byte offsets of its workspace regions (256-byte aligned).
 struct ReblockLayout {
-  size_t mpart, M, W, X, perm0, perm1, keys, meta, part, mu, v, hist, state, cnt, base, total;
+  size_t mpart, M, W, Wb, X, perm0, perm1, keys, meta, part, mu, v, hist, state, cnt, base, err,
+      total;
   int levels, nb;
 };
 
