@@ -540,18 +540,37 @@ def main():
     # ---- end to end through the public call with host buffers (pinned), copies timed
     e2e = None
     if args.e2e_steps > 0:
-        from block_sparse_attention_gather_b200 import spark_bsa_forward, spark_bsa_forward_ctx
+        from block_sparse_attention_gather_b200 import (spark_bsa_forward, spark_bsa_forward_ctx,
+                                                        spark_bsa_forward_host,
+                                                        spark_bsa_host_staging_size,
+                                                        spark_bsa_workspace_size)
         names = ["Q", "K", "V", "q_perm", "k_perm", "q_offsets", "k_offsets"]
         if hp.nc:
             names += ["Kc", "Vc"]
         host = {n: x[n].to("cpu").pin_memory() for n in names}
-        dev_in = {n: torch.empty_like(x[n]) for n in host}
+        dev_in = {n: torch.empty_like(x[n]) for n in host} if hp.nc else {}
         out_host = torch.empty(hp.out.shape, dtype=hp.out.dtype).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = out_host.numel() * out_host.element_size()
         s = torch.cuda.current_stream(device)
+        # without context tokens: the host-buffer entry point, pipelined by chunks of 4 heads
+        hpc = 4
+        if not hp.nc:
+            staging = torch.empty(spark_bsa_host_staging_size(hp.H, hp.N, hp.d, hp.out.dtype,
+                                                              hp.nqb, hp.nkb, hpc),
+                                  dtype=torch.uint8, device=device)
+            chunk_ws = torch.empty(spark_bsa_workspace_size(min(hpc, hp.H), hp.N, hp.d, hp.nqb,
+                                                            hp.nkb, w.ratio),
+                                   dtype=torch.uint8, device=device)
+            pipe = (s, torch.cuda.Stream(device), torch.cuda.Stream(device))
 
         def e2e_step():
+            if not hp.nc:
+                spark_bsa_forward_host(host["Q"], host["K"], host["V"], host["q_perm"],
+                                       host["k_perm"], host["q_offsets"], host["k_offsets"],
+                                       w.ratio, out=out_host, heads_per_chunk=hpc,
+                                       staging=staging, workspace=chunk_ws, streams=pipe)
+                return
             for n in host:
                 dev_in[n].copy_(host[n], non_blocking=True)
             if hp.nc:
@@ -586,7 +605,10 @@ def main():
             e_ms = float(tt.item())
         e2e = {"value": world * dflops * args.e2e_steps / (e_ms / 1e3) / 1e12, "unit": UNIT,
                "ms_per_call": e_ms / args.e2e_steps, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "call": ("spark_bsa_forward_ctx after host-to-device copies" if hp.nc else
+                        f"spark_bsa_forward_host (host buffers, chunks of {hpc} heads, copies "
+                        "overlapped with computation on three streams)")}
         del host, dev_in, out_host
 
     traffic = profiled_traffic(hp)

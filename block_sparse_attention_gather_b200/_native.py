@@ -24,6 +24,7 @@ __all__ = [
     "spark_bsa_attend_ctx", "ReblockLayout", "spark_reblock_workspace_layout",
     "spark_reblock_workspace_size", "spark_reblock_levels", "spark_reblock",
     "spark_reblock_whiten", "spark_reblock_level", "reblock_views",
+    "spark_bsa_host_staging_size", "spark_bsa_forward_host",
 ]
 
 SPARK_BF16, SPARK_F32 = 0, 1
@@ -36,6 +37,7 @@ EXPORTED = [
     "spark_bsa_workspace_size_ctx", "spark_bsa_forward_ctx", "spark_bsa_context_bf16",
     "spark_bsa_attend_ctx", "spark_reblock_workspace_layout", "spark_reblock_workspace_size",
     "spark_reblock_levels", "spark_reblock", "spark_reblock_whiten", "spark_reblock_level",
+    "spark_bsa_host_staging_size", "spark_bsa_forward_host",
 ]
 REBLOCK_MODES = {"q_reuse_k": 0, "separate": 1}
 
@@ -103,6 +105,9 @@ def lib():
         "spark_reblock": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
         "spark_reblock_whiten": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P]),
         "spark_reblock_level": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+        "spark_bsa_host_staging_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+        "spark_bsa_forward_host": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _I, _D,
+                                        _P, _I, _P, _SZ, _P, _SZ, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -516,3 +521,58 @@ def spark_reblock_level(H, N, d, block, level, perm_in, workspace, perm_out=None
                                    _stream(stream))
     _check("spark_reblock_level", st)
     return perm_out
+
+
+# ------------------------------------------------ host buffers, pipelined by head chunks
+
+def spark_bsa_host_staging_size(H, N, d, dtype, nqb, nkb, heads_per_chunk) -> int:
+    return int(lib().spark_bsa_host_staging_size(H, N, d, _code(dtype), nqb, nkb,
+                                                  heads_per_chunk))
+
+
+def _need_host(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def spark_bsa_forward_host(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, topk_ratio, out=None,
+                           heads_per_chunk=4, device=None, staging=None, workspace=None,
+                           streams=None):
+    """The forward pass on HOST tensors (page-locked for overlap), pipelined by head chunks
+    over three CUDA streams; returns `out` (host) once the work is enqueued on the compute
+    stream (synchronise that stream, or the device, before reading it)."""
+    _need_host(Q, "Q", (torch.bfloat16, torch.float32))
+    for n, t in (("K", K), ("V", V)):
+        _need_host(t, n, Q.dtype)
+    for n, t in (("q_perm", q_perm), ("k_perm", k_perm), ("q_offsets", q_offsets),
+                 ("k_offsets", k_offsets)):
+        _need_host(t, n, torch.int32)
+    H, N, d = Q.shape
+    nqb, nkb = q_offsets.numel() - 1, k_offsets.numel() - 1
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    hpc = max(1, min(int(heads_per_chunk), H))
+    if out is None:
+        out = torch.empty_like(Q).pin_memory()
+    _need_host(out, "out", Q.dtype)
+    if staging is None:
+        staging = torch.empty(spark_bsa_host_staging_size(H, N, d, Q.dtype, nqb, nkb, hpc),
+                              dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = torch.empty(spark_bsa_workspace_size(hpc, N, d, nqb, nkb, topk_ratio),
+                                dtype=torch.uint8, device=dev)
+    if streams is None:
+        streams = (torch.cuda.current_stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    sc, sh, sd = (ctypes.c_void_p(s.cuda_stream) for s in streams)
+    st = lib().spark_bsa_forward_host(_ptr(Q), _ptr(K), _ptr(V), _code(Q.dtype), H, N, d,
+                                      _ptr(q_perm), _ptr(k_perm), _ptr(q_offsets), nqb,
+                                      _ptr(k_offsets), nkb, float(topk_ratio), _ptr(out), hpc,
+                                      _ptr(staging), staging.numel(), _ptr(workspace),
+                                      workspace.numel(), sc, sh, sd)
+    _check("spark_bsa_forward_host", st)
+    return out

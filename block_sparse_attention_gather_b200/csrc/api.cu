@@ -377,6 +377,153 @@ spark_status spark_bsa_forward(const void* Q, const void* K, const void* V, int 
                       workspace_bytes, as_stream(stream));
 }
 
+// ------------------------------------------------- host buffers, pipelined by head chunks
+
+namespace {
+
+struct HostStaging {
+  size_t Q, K, V, qp, kp, out, slot, qo, ko, total;
+};
+
+HostStaging staging_layout(int hpc, int N, int d, int esize, int nqb, int nkb) {
+  HostStaging L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  const size_t rows = static_cast<size_t>(hpc) * N;
+  L.Q = take(rows * d * esize);
+  L.K = take(rows * d * esize);
+  L.V = take(rows * d * esize);
+  L.qp = take(rows * 4);
+  L.kp = take(rows * 4);
+  L.out = take(rows * d * esize);
+  L.slot = off;                                  // one slot; the second follows at +slot
+  off = 2 * L.slot;
+  L.qo = take(static_cast<size_t>(nqb + 1) * 4);
+  L.ko = take(static_cast<size_t>(nkb + 1) * 4);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+size_t spark_bsa_host_staging_size(int H, int N, int d, int dtype, int nqb, int nkb,
+                                   int heads_per_chunk) {
+  if (check_sizes(H, N, d, nqb, nkb) != SPARK_OK || heads_per_chunk < 1) return 0;
+  if (dtype != SPARK_BF16 && dtype != SPARK_F32) return 0;
+  const int hpc = heads_per_chunk < H ? heads_per_chunk : H;
+  return staging_layout(hpc, N, d, dtype == SPARK_BF16 ? 2 : 4, nqb, nkb).total;
+}
+
+spark_status spark_bsa_forward_host(const void* Q, const void* K, const void* V, int dtype,
+                                    int H, int N, int d, const int32_t* q_perm,
+                                    const int32_t* k_perm, const int32_t* q_block_offsets,
+                                    int nqb, const int32_t* k_block_offsets, int nkb,
+                                    double topk_ratio, void* out, int heads_per_chunk,
+                                    void* staging, size_t staging_bytes, void* workspace,
+                                    size_t workspace_bytes, void* compute_stream,
+                                    void* h2d_stream, void* d2h_stream) {
+  if (!Q || !K || !V || !q_perm || !k_perm || !q_block_offsets || !k_block_offsets || !out)
+    return SPARK_ERR_INVALID_ARG;
+  if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  if (heads_per_chunk < 1) return SPARK_ERR_INVALID_ARG;
+  spark_bsa_layout whole;
+  spark_status st = layout_of(H, N, d, nqb, nkb, topk_ratio, &whole);
+  if (st != SPARK_OK) return st;
+  const int hpc = heads_per_chunk < H ? heads_per_chunk : H;
+  spark_bsa_layout chunk_layout;
+  st = layout_of(hpc, N, d, nqb, nkb, topk_ratio, &chunk_layout);
+  if (st != SPARK_OK) return st;
+  const int esize = dtype == SPARK_BF16 ? 2 : 4;
+  const HostStaging S = staging_layout(hpc, N, d, esize, nqb, nkb);
+  if (!staging || staging_bytes < S.total || !aligned(staging, kAlign)) return SPARK_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < chunk_layout.total || !aligned(workspace, kAlign))
+    return SPARK_ERR_WORKSPACE;
+  cudaStream_t sc = as_stream(compute_stream), sh = as_stream(h2d_stream),
+               sd = as_stream(d2h_stream);
+  uint8_t* stg = static_cast<uint8_t*>(staging);
+  cudaEvent_t ev[7] = {};
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      for (auto& f : ev)
+        if (f) cudaEventDestroy(f);
+      return SPARK_ERR_CUDA;
+    }
+  cudaEvent_t* h2d_done = ev;        // [2]
+  cudaEvent_t* comp_done = ev + 2;   // [2]
+  cudaEvent_t* d2h_done = ev + 4;    // [2]
+  cudaEvent_t start = ev[6];
+  auto fail = [&]() {
+    for (auto& e : ev) cudaEventDestroy(e);
+    return SPARK_ERR_CUDA;
+  };
+  // the copy streams start after everything already queued on the compute stream (e.g. an
+  // earlier call that still reads the staging slots)
+  if (cudaEventRecord(start, sc) != cudaSuccess || cudaStreamWaitEvent(sh, start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(sd, start, 0) != cudaSuccess)
+    return fail();
+  const size_t row_bytes = static_cast<size_t>(N) * d * esize;
+  const size_t perm_bytes = static_cast<size_t>(N) * 4;
+  int32_t* qo = reinterpret_cast<int32_t*>(stg + S.qo);
+  int32_t* ko = reinterpret_cast<int32_t*>(stg + S.ko);
+  if (cudaMemcpyAsync(qo, q_block_offsets, (nqb + 1) * 4, cudaMemcpyHostToDevice, sh) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(ko, k_block_offsets, (nkb + 1) * 4, cudaMemcpyHostToDevice, sh) !=
+          cudaSuccess)
+    return fail();
+  const int nchunks = (H + hpc - 1) / hpc;
+  const auto* q8 = static_cast<const uint8_t*>(Q);
+  const auto* k8 = static_cast<const uint8_t*>(K);
+  const auto* v8 = static_cast<const uint8_t*>(V);
+  auto* o8 = static_cast<uint8_t*>(out);
+  for (int c = 0; c < nchunks; ++c) {
+    const int slot = c & 1;
+    const int h0 = c * hpc;
+    const int hc = (H - h0) < hpc ? (H - h0) : hpc;
+    uint8_t* base = stg + slot * S.slot;
+    // inputs of chunk c into the slot, once chunk c-2 no longer reads it
+    if (c >= 2 && cudaStreamWaitEvent(sh, comp_done[slot], 0) != cudaSuccess) return fail();
+    if (cudaMemcpyAsync(base + S.Q, q8 + h0 * row_bytes, hc * row_bytes, cudaMemcpyHostToDevice,
+                        sh) != cudaSuccess ||
+        cudaMemcpyAsync(base + S.K, k8 + h0 * row_bytes, hc * row_bytes, cudaMemcpyHostToDevice,
+                        sh) != cudaSuccess ||
+        cudaMemcpyAsync(base + S.V, v8 + h0 * row_bytes, hc * row_bytes, cudaMemcpyHostToDevice,
+                        sh) != cudaSuccess ||
+        cudaMemcpyAsync(base + S.qp, q_perm + static_cast<size_t>(h0) * N, hc * perm_bytes,
+                        cudaMemcpyHostToDevice, sh) != cudaSuccess ||
+        cudaMemcpyAsync(base + S.kp, k_perm + static_cast<size_t>(h0) * N, hc * perm_bytes,
+                        cudaMemcpyHostToDevice, sh) != cudaSuccess ||
+        cudaEventRecord(h2d_done[slot], sh) != cudaSuccess)
+      return fail();
+    // the forward pass of the chunk, once its inputs are in and the slot's output is read out
+    if (cudaStreamWaitEvent(sc, h2d_done[slot], 0) != cudaSuccess) return fail();
+    if (c >= 2 && cudaStreamWaitEvent(sc, d2h_done[slot], 0) != cudaSuccess) return fail();
+    st = forward_impl(base + S.Q, base + S.K, base + S.V, nullptr, nullptr, 0, dtype, hc, N, d,
+                      reinterpret_cast<const int32_t*>(base + S.qp),
+                      reinterpret_cast<const int32_t*>(base + S.kp), qo, nqb, ko, nkb,
+                      topk_ratio, base + S.out, workspace, workspace_bytes, sc);
+    if (st != SPARK_OK) {
+      for (auto& e : ev) cudaEventDestroy(e);
+      return st;
+    }
+    if (cudaEventRecord(comp_done[slot], sc) != cudaSuccess) return fail();
+    // the chunk's output back to the host
+    if (cudaStreamWaitEvent(sd, comp_done[slot], 0) != cudaSuccess ||
+        cudaMemcpyAsync(o8 + h0 * row_bytes, base + S.out, hc * row_bytes,
+                        cudaMemcpyDeviceToHost, sd) != cudaSuccess ||
+        cudaEventRecord(d2h_done[slot], sd) != cudaSuccess)
+      return fail();
+  }
+  // the compute stream completes only after every copy back
+  for (int slot = 0; slot < 2 && slot < nchunks; ++slot)
+    if (cudaStreamWaitEvent(sc, d2h_done[slot], 0) != cudaSuccess) return fail();
+  for (auto& e : ev) cudaEventDestroy(e);   // released once the pending work completes
+  return SPARK_OK;
+}
+
 // ---------------------------------------------------------------- Spark-Reblock
 
 int spark_reblock_levels(int N, int block) {

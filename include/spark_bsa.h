@@ -225,6 +225,37 @@ SPARK_API spark_status spark_bsa_attend_ctx(const void* Qp, const void* Kp, cons
                                             int N, int d, void* out, int out_dtype,
                                             uint32_t* err, void* stream);
 
+/* ---- Host buffers, pipelined by head chunks ----
+ * No counterpart in the pages: the forward pass for inputs and output in host memory.  The
+ * heads are processed in chunks of `heads_per_chunk`; the copies of chunk c+1 in and of
+ * chunk c-1 out run on `h2d_stream` / `d2h_stream` while chunk c is computed on
+ * `compute_stream`, through two device staging slots.  The result equals spark_bsa_forward
+ * on the same inputs bit for bit (heads are independent).
+ *   - Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister); pageable memory
+ *     works but the copies then do not overlap the computation.
+ *   - `staging`: device, 256-byte aligned, spark_bsa_host_staging_size bytes;
+ *     `workspace`: device, 256-byte aligned, spark_bsa_workspace_size(min(heads_per_chunk, H),
+ *     ...) bytes, reused by every chunk.
+ *   - The call only enqueues work; `compute_stream` completes after the last copy back, so
+ *     synchronising it is enough.  The three streams must be distinct.
+ *   - The workspace's error word describes the last chunk only.
+ *   - The copy streams first wait for the work already queued on `compute_stream`, so
+ *     back-to-back calls sharing staging buffers are ordered.
+ *   - The call creates and releases seven CUDA events; it allocates no device memory. */
+SPARK_API size_t spark_bsa_host_staging_size(int H, int N, int d, int dtype, int nqb, int nkb,
+                                             int heads_per_chunk);
+
+SPARK_API spark_status spark_bsa_forward_host(const void* Q, const void* K, const void* V,
+                                              int dtype, int H, int N, int d,
+                                              const int32_t* q_perm, const int32_t* k_perm,
+                                              const int32_t* q_block_offsets, int nqb,
+                                              const int32_t* k_block_offsets, int nkb,
+                                              double topk_ratio, void* out, int heads_per_chunk,
+                                              void* staging, size_t staging_bytes,
+                                              void* workspace, size_t workspace_bytes,
+                                              void* compute_stream, void* h2d_stream,
+                                              void* d2h_stream);
+
 /* ---- Spark-Reblock token partitioner ----
  * Spark-H3 blog, section "Spark-Reblock": queries are grouped under the Mahalanobis cosine
  * distance d_Q(q_i,q_j) = 1 - cos(M_K^{1/2} q_i, M_K^{1/2} q_j), M_K = E[k k^T] (keys

@@ -179,6 +179,27 @@ def test_reblock_entry_points_reject_bad_arguments(L):
     assert L.spark_reblock_whiten(p, p, 0, 2, 1000, 64, 64, p, 16, None) == WORKSPACE
 
 
+def test_host_pipeline_rejects_bad_arguments(L):
+    from block_sparse_attention_gather_b200 import spark_bsa_host_staging_size
+    import torch
+    assert spark_bsa_host_staging_size(24, 241920, 128, torch.bfloat16, 1890, 1890, 4) > 0
+    assert spark_bsa_host_staging_size(24, 241920, 128, torch.bfloat16, 1890, 1890, 0) == 0
+    four = spark_bsa_host_staging_size(24, 241920, 128, torch.bfloat16, 1890, 1890, 4)
+    eight = spark_bsa_host_staging_size(24, 241920, 128, torch.bfloat16, 1890, 1890, 8)
+    assert eight > four                                  # two slots of the chunk size
+    p = ctypes.c_void_p(0x100000)
+    big = ctypes.c_size_t(1 << 40)
+
+    def call(hpc=2, staging_bytes=big, ws_bytes=big, out=p):
+        return L.spark_bsa_forward_host(p, p, p, 0, 4, 1000, 128, p, p, p, 10, p, 10,
+                                        ctypes.c_double(0.2), out, hpc, p, staging_bytes, p,
+                                        ws_bytes, None, None, None)
+    assert call(hpc=0) == INVALID
+    assert call(out=None) == INVALID
+    assert call(staging_bytes=16) == WORKSPACE
+    assert call(ws_bytes=16) == WORKSPACE
+
+
 def test_missing_library_fails_loudly(tmp_path):
     code = ("import block_sparse_attention_gather_b200._native as n;"
             f"n.LIB_PATH = {str(tmp_path / 'nope.so')!r};"
