@@ -152,6 +152,16 @@ def test_edge_cases(case):
         check_forward(x, 0.9)
 
 
+@pytest.mark.parametrize("nkb", [7000, 12800])
+def test_many_key_blocks(nkb):
+    """Unit-size blocks: 7000 key blocks take the routing kernel's 4-row variant and the
+    attention kernel's path that reads summary offsets from global memory (they no longer fit
+    its shared-memory row); 12800 is the largest block count the library accepts."""
+    x = custom_inputs(27 + nkb, H=1, N=nkb, d=128, dtype="bf16", lo=1, hi=1)
+    assert x["k_offsets"].numel() - 1 == nkb
+    check_forward(x, 0.01, blocks_per_head=6, seed=nkb, check_inter=False)
+
+
 # ------------------------------------------------------------------- step entry points
 
 @pytest.mark.parametrize("d", [64, 128])
