@@ -585,7 +585,7 @@ __device__ __forceinline__ float group_dot(const uint32_t (&w)[DPL / 2], const f
 // fixed order (warp, step, group) and the partial sums are reduced over groups and then
 // warps in a fixed order.
 template <int D, bool kFirst>
-__global__ void __launch_bounds__(kRbThreads) rb_power_kernel(
+__global__ void __launch_bounds__(kRbThreads, 3) rb_power_kernel(
     const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm, int N,
     const int4* __restrict__ chunks, int nch, const float* __restrict__ vnode, int nnodes,
     float* __restrict__ part) {
@@ -695,7 +695,7 @@ __global__ void __launch_bounds__(D) rb_node_reduce_kernel(const float* __restri
 
 // keys[pos] = order key of x.v (the order of (x - mu).v), and the histogram of the top byte.
 template <int D>
-__global__ void __launch_bounds__(kRbThreads) rb_project_kernel(
+__global__ void __launch_bounds__(kRbThreads, 3) rb_project_kernel(
     const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm, int N,
     const int4* __restrict__ chunks, const float* __restrict__ vnode, int nnodes,
     uint32_t* __restrict__ keys, uint32_t* __restrict__ hist) {
