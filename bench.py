@@ -345,15 +345,38 @@ def run_reference(args, world, rank):
 REBLOCK_METRIC = "ms/call of the Spark-Reblock partitioner (q_reuse_k), 768p shape"
 
 
-def reblock_bytes_flops(H, N, d, levels, e_in, power_iters=4):
+def reblock_level_min_nodes(N, block):
+    """Smallest node (in tokens) of every level of the partitioner's block tree: an m-block
+    node gives ceil(m/2) blocks to its left child; the last block takes the remainder."""
+    nb = -(-N // block)
+    off = lambda b: N if b >= nb else b * block
+    out, frontier = [], [(0, nb)]
+    while frontier:
+        sizes, nxt = [], []
+        for lo, hi in frontier:
+            if hi - lo >= 2:
+                mid = lo + (hi - lo + 1) // 2
+                sizes.append(off(hi) - off(lo))
+                nxt += [(lo, mid), (mid, hi)]
+        if sizes:
+            out.append(min(sizes))
+        frontier = nxt
+    return out
+
+
+def reblock_bytes_flops(H, N, d, block, e_in, power_iters=4, moment_min_node=2048):
     """Algorithmic work of one partitioner call: the flops of the second moment and of the
     whitening (2 H N d^2 each; bf16 tensor-core MMAs for bf16 inputs), the HBM bytes of the
     whitening (read Q and K, write the bf16 unit rows), and the HBM bytes of the per-level
-    passes over the unit rows (power_iters + 1 reads with the token index per level) plus the
-    keys, histogram and scatter passes (4 + 4 + 4 + 8 bytes per token and level)."""
+    passes over the unit rows with the token index: 2 passes (node moments, projection) on
+    levels whose nodes hold >= moment_min_node tokens when d = 128, power_iters + 1 passes
+    otherwise, plus the keys, histogram and scatter passes (4 + 4 + 4 + 8 bytes per token)."""
     flops = 2 * 2.0 * H * N * d * d
     prep_bytes = 2.0 * H * N * d * e_in + H * N * d * 2
-    level_bytes = levels * H * N * ((power_iters + 1) * (2 * d + 4) + 4 + 3 * 4 + 4 + 8)
+    level_bytes = 0.0
+    for m in reblock_level_min_nodes(N, block):
+        passes = 2 if (d == 128 and m >= moment_min_node) else power_iters + 1
+        level_bytes += H * N * (passes * (2 * d + 4) + 4 + 3 * 4 + 4 + 8)
     return flops, prep_bytes, level_bytes
 
 
@@ -422,7 +445,7 @@ def run_reblock(args, world, rank, local):
     torch.cuda.synchronize()
     prep_ms = pe[0].elapsed_time(pe[1]) / args.steps
     part_ms = ms - prep_ms
-    flops, prep_bytes, level_bytes = reblock_bytes_flops(H, N, d, lay.levels, Q.element_size())
+    flops, prep_bytes, level_bytes = reblock_bytes_flops(H, N, d, block, Q.element_size())
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     gbs = level_bytes / (part_ms / 1e3) / 1e9
     line = {
@@ -444,8 +467,10 @@ def run_reblock(args, world, rank, local):
                         "units": ("tcgen05 bf16 MMAs, fp32 accumulation" if
                                   Q.dtype == torch.bfloat16 and d == 128 else "fp32 CUDA cores")},
                     "levels": {"ms": part_ms, "GB/s": gbs, "bytes": level_bytes}},
-        # per call: 4 whitening kernels, the identity order, 19 kernels per level, offsets
-        "gpu_launches": (6 + 19 * lay.levels) * args.steps,  # + 0: same count on either path
+        # per call: 4 whitening kernels, the identity order, offsets, and per level 11
+        # selection/scatter kernels plus 8 power-pass kernels or 2 node-moment kernels
+        "gpu_launches": (6 + sum(11 + (2 if (d == 128 and m >= 2048) else 8)
+                                 for m in reblock_level_min_nodes(N, block))) * args.steps,
         "clocks": clock_info,
     }
     if rank == 0:

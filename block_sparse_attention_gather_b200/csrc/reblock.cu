@@ -933,6 +933,218 @@ __global__ void __launch_bounds__(kRbThreads) rb_scatter_kernel(
   }
 }
 
+// ------------------------------------------------------------------ tensor-core node moments
+// Levels whose nodes hold at least kCovMinNode tokens (d = 128): instead of kPowerIters passes
+// over the rows, one pass gathers each chunk's rows (by the permutation) into shared memory
+// and sums x x^T on the tensor cores (both operands the MN-major tile, as in rb_moment_tc),
+// plus the sum of x; rb_cov_node then runs the power iterations on the node's 128 x 128
+// matrix: v <- (S/n - mu mu^T) v, the same update as the row passes.
+
+constexpr int kCovChunk = 16384;      // tokens per CTA of the moment pass
+constexpr int kCovMinNode = 2048;     // smallest node size that takes this path
+constexpr int kCovStride = 128 * 128 + 128;   // floats per partial: x x^T, then sum x
+
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// One chunk of a node: rows gathered by the permutation into 128-token tiles (cp.async, each
+// 16-byte piece written to its place in the 128-byte swizzled layout, zero past the chunk
+// end), the next tile in flight while the tensor core consumes the current one.
+__global__ void __launch_bounds__(128) rb_cov_tc_kernel(const __nv_bfloat16* __restrict__ X,
+                                                        const int32_t* __restrict__ perm, int N,
+                                                        const int4* __restrict__ cchunks,
+                                                        int ncch, float* __restrict__ cpart,
+                                                        uint32_t* __restrict__ err) {
+  extern __shared__ uint8_t rb_tc_raw[];
+  uint8_t* st = align1024(rb_tc_raw);                    // 2 stages x 32 KB
+  uint64_t* mdone = reinterpret_cast<uint64_t*>(st + 2 * kTcTile);   // [2]
+  uint64_t* done = mdone + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* toks = reinterpret_cast<int*>(tmem_slot + 4);     // [2][128] token ids of a tile
+  float* red = reinterpret_cast<float*>(toks + 256);     // [128][8] column sums
+  const int c = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, warp = tid / 32;
+  const int4 ch = cchunks[c];
+  const int T = (ch.z - ch.y + 127) / 128;
+  const int cidx = tid % 16;                             // this thread's 16-byte column chunk
+  if (tid == 0) {
+    mbar_init(&mdone[0], 1);
+    mbar_init(&mdone[1], 1);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  const int32_t* ph = perm + static_cast<size_t>(h) * N;
+  const __nv_bfloat16* Xh = X + static_cast<size_t>(h) * N * 128;
+  auto stage_toks = [&](int t) {                         // thread tid: row tid of tile t
+    const int pos = ch.y + t * 128 + tid;
+    toks[(t & 1) * 128 + tid] = pos < ch.z ? min(max(ph[pos], 0), N - 1) : -1;
+  };
+  auto issue_tile = [&](int t) {                         // after toks of tile t are visible
+    uint8_t* tile = st + (t & 1) * kTcTile;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int r = (tid + 128 * i) >> 4;
+      const int tok = toks[(t & 1) * 128 + r];
+      cp_async16_zfill(tile + (cidx / 8) * 16384 + r * 128 + (((cidx % 8) ^ (r & 7)) * 16),
+                       Xh + static_cast<size_t>(tok < 0 ? 0 : tok) * 128 + cidx * 8, tok >= 0);
+    }
+    cp_async_commit();
+  };
+  if (T > 0) stage_toks(0);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tbase = *tmem_slot;
+  constexpr uint32_t idM = idesc_bf16(128, 128, true, true);
+  float sx[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) sx[j] = 0.f;
+  if (T > 0) issue_tile(0);
+  bool ok = true;
+  for (int t = 0; t < T; ++t) {
+    const int s = t & 1;
+    if (t + 1 < T) stage_toks(t + 1);                    // its latency overlaps the wait below
+    cp_async_wait_all();                                 // this thread's pieces of tile t
+    fence_proxy_async_smem();                            // visible to the tensor core
+    __syncthreads();                                     // everyone's pieces, and toks(t+1)
+    const uint8_t* tile = st + s * kTcTile;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int r = (tid + 128 * i) >> 4;
+      const uint4 u = *reinterpret_cast<const uint4*>(
+          tile + (cidx / 8) * 16384 + r * 128 + (((cidx % 8) ^ (r & 7)) * 16));
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        sx[2 * q] += __uint_as_float(w[q] << 16);
+        sx[2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+      }
+    }
+    if (tid == 0) {
+      tc_fence_after_sync();
+      const uint64_t d0 = sdesc_sw128(smem_u32(tile), 16384, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t dk = d0 + static_cast<uint64_t>((kk * 2048) >> 4);
+        mma_ss(tbase, dk, dk, idM, (t > 0 || kk > 0) ? 1u : 0u);
+      }
+      tc_commit(&mdone[s]);
+    }
+    if (t + 1 < T) {
+      // stage s^1 held tile t-1: its MMAs must be done before it is overwritten
+      if (t >= 1)
+        ok = __syncthreads_and(mbar_wait(&mdone[s ^ 1], ((t - 1) >> 1) & 1, abort_flag, err));
+      if (!ok) break;
+      issue_tile(t + 1);
+    }
+  }
+  cp_async_wait_all();                                   // nothing of ours left in flight
+  if (tid == 0) {
+    tc_commit(done);                                     // every MMA issued has completed
+    rb_wait_quiet(done, 0);
+  }
+  __syncthreads();
+  const bool fine = ok && !*abort_flag;
+  tc_fence_after_sync();
+  float* out = cpart + (static_cast<size_t>(h) * ncch + c) * kCovStride;
+  const int row = warp * 32 + (tid % 32);
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t r[32];
+    if (fine) {
+      tmem_ld32(tbase + (static_cast<uint32_t>(warp * 32) << 16) + cc * 32, r);
+    } else {
+      for (int j = 0; j < 32; ++j) r[j] = 0u;
+    }
+    float4* dst = reinterpret_cast<float4*>(out + row * 128 + cc * 32);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                           __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+  }
+  // column sums: the 8 threads with the same chunk index, in thread order
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[tid * 8 + j] = sx[j];
+  __syncthreads();
+  {
+    const int dim = tid, cc = dim / 8, j = dim % 8;
+    float a = 0.f;
+    for (int g = 0; g < 8; ++g) a += red[(g * 16 + cc) * 8 + j];
+    out[128 * 128 + dim] = fine ? a : 0.f;
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tbase, 128);
+  }
+}
+
+// Per node: S = sum of the chunk partials (in order), mu = sum x / n, then kPowerIters steps
+// v <- w / |w|, w = S v / n - (mu . v) mu, from v0 = (1,...,1)/sqrt(d).
+__global__ void __launch_bounds__(128) rb_cov_node_kernel(const float* __restrict__ cpart,
+                                                          int ncch,
+                                                          const int4* __restrict__ cnodes,
+                                                          const int4* __restrict__ nodes,
+                                                          int nnodes, float* __restrict__ mu,
+                                                          float* __restrict__ vnode) {
+  extern __shared__ __align__(16) float Ssm[];           // [128][128]
+  __shared__ float vs[128];
+  __shared__ float red[4];
+  __shared__ float s_val;
+  const int g = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
+  const int4 cn = cnodes[g];
+  const int4 nd = nodes[g];
+  const float n = static_cast<float>(nd.z - nd.x);
+  for (int row0 = 0; row0 < 128; row0 += 8) {
+    float a[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) a[r] = 0.f;
+    for (int c = cn.x; c < cn.y; ++c) {
+      const float* pc = cpart + (static_cast<size_t>(h) * ncch + c) * kCovStride + t;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) a[r] += pc[(row0 + r) * 128];   // 8 rows in flight
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) Ssm[(row0 + r) * 128 + t] = a[r];
+  }
+  float sxv = 0.f;
+  for (int c = cn.x; c < cn.y; ++c) sxv += cpart[(static_cast<size_t>(h) * ncch + c) * kCovStride + 128 * 128 + t];
+  const float m = sxv / n;
+  float v = rsqrtf(128.f);
+  auto block_sum = [&](float x) {
+    x = warp_sum(x);
+    __syncthreads();
+    if (t % 32 == 0) red[t / 32] = x;
+    __syncthreads();
+    if (t == 0) s_val = red[0] + red[1] + red[2] + red[3];
+    __syncthreads();
+    return s_val;
+  };
+  for (int it = 0; it < kPowerIters; ++it) {
+    vs[t] = v;
+    __syncthreads();
+    float sv = 0.f;
+    for (int j = 0; j < 128; ++j) sv = fmaf(Ssm[j * 128 + t], vs[j], sv);   // S symmetric
+    const float muv = block_sum(m * v);
+    const float w = sv / n - muv * m;
+    const float nrm2 = block_sum(w * w);
+    v = nrm2 > 0.f ? w * rsqrtf(nrm2) : v;
+  }
+  const size_t at = (static_cast<size_t>(h) * nnodes + g) * 128 + t;
+  mu[at] = m;
+  vnode[at] = v;
+}
+
 // ------------------------------------------------------------------ host side
 
 namespace {
@@ -940,13 +1152,15 @@ namespace {
 struct LevelMeta {
   int node_off, nnodes;      // into the int4 node array (nnodes + 1 entries incl. sentinel)
   int chunk_off, nch;        // into the int4 chunk array
+  bool cov;                  // every node >= kCovMinNode tokens: tensor-core moments
+  int cnode_off, cchunk_off, ncch;   // per node (first, end) moment chunk; moment chunks
 };
 
 struct Plan {
   int nb = 0;
   std::vector<LevelMeta> levels;
-  std::vector<int4> nodes, chunks;
-  int max_nodes = 0, max_chunks = 0;
+  std::vector<int4> nodes, chunks, cnodes, cchunks;
+  int max_nodes = 0, max_chunks = 0, max_cchunks = 0;
 };
 
 Plan make_plan(int N, int block) {
@@ -956,7 +1170,8 @@ Plan make_plan(int N, int block) {
   std::vector<std::pair<int, int>> frontier{{0, P.nb}};
   while (!frontier.empty()) {
     std::vector<std::pair<int, int>> next;
-    LevelMeta L{static_cast<int>(P.nodes.size()), 0, static_cast<int>(P.chunks.size()), 0};
+    LevelMeta L{static_cast<int>(P.nodes.size()), 0, static_cast<int>(P.chunks.size()), 0,
+                true, static_cast<int>(P.cnodes.size()), static_cast<int>(P.cchunks.size()), 0};
     for (auto [lo, hi] : frontier) {
       if (hi - lo < 2) continue;
       const int mid = lo + (hi - lo + 1) / 2;
@@ -966,6 +1181,13 @@ Plan make_plan(int N, int block) {
         P.chunks.push_back(make_int4(L.nnodes, s, std::min(e, s + kChunk), 0));
         ++L.nch;
       }
+      if (e - a < kCovMinNode) L.cov = false;
+      const int c0 = L.ncch;
+      for (int s = a; s < e; s += kCovChunk) {
+        P.cchunks.push_back(make_int4(L.nnodes, s, std::min(e, s + kCovChunk), 0));
+        ++L.ncch;
+      }
+      P.cnodes.push_back(make_int4(c0, L.ncch, 0, 0));
       ++L.nnodes;
       next.push_back({lo, mid});
       next.push_back({mid, hi});
@@ -975,6 +1197,7 @@ Plan make_plan(int N, int block) {
       P.levels.push_back(L);
       P.max_nodes = std::max(P.max_nodes, L.nnodes);
       P.max_chunks = std::max(P.max_chunks, L.nch);
+      if (L.cov) P.max_cchunks = std::max(P.max_cchunks, L.ncch);
     }
     frontier.swap(next);
   }
@@ -1003,9 +1226,12 @@ ReblockLayout reblock_layout(int H, int N, int d, int block) {
   L.perm0 = take(static_cast<size_t>(H) * N * 4);
   L.perm1 = take(static_cast<size_t>(H) * N * 4);
   L.keys = take(static_cast<size_t>(H) * N * 4);
-  L.meta = take((P.nodes.size() + P.chunks.size()) * sizeof(int4));
+  L.meta = take((P.nodes.size() + P.chunks.size() + P.cnodes.size() + P.cchunks.size()) *
+                sizeof(int4));
   const size_t mn = std::max(P.max_nodes, 1), mc = std::max(P.max_chunks, 1);
   L.part = take(static_cast<size_t>(H) * mc * 2 * d * 4);
+  L.cpart = take(d == 128 ? static_cast<size_t>(H) * std::max(P.max_cchunks, 1) * kCovStride * 4
+                          : 256);
   L.mu = take(static_cast<size_t>(H) * mn * d * 4);
   L.v = take(static_cast<size_t>(H) * mn * d * 4);
   L.hist = take(static_cast<size_t>(H) * mn * 256 * 4);
@@ -1093,6 +1319,8 @@ cudaError_t upload_reblock_plan(int N, int block, void* workspace, const Reblock
   const Plan P = make_plan(N, block);
   std::vector<int4> meta(P.nodes);
   meta.insert(meta.end(), P.chunks.begin(), P.chunks.end());
+  meta.insert(meta.end(), P.cnodes.begin(), P.cnodes.end());
+  meta.insert(meta.end(), P.cchunks.begin(), P.cchunks.end());
   if (meta.empty()) return cudaSuccess;
   // pageable source: the copy is staged before the call returns
   return cudaMemcpyAsync(static_cast<uint8_t*>(workspace) + L.meta, meta.data(),
@@ -1121,11 +1349,29 @@ static cudaError_t level_t(int H, int N, int block, int level, const int32_t* pe
   const dim3 gc(nc, H), gn(nn, H);
   cudaError_t e = cudaMemsetAsync(hist, 0, static_cast<size_t>(H) * nn * 256 * 4, s);
   if (e != cudaSuccess) return e;
-  rb_power_kernel<D, true><<<gc, kRbThreads, 0, s>>>(X, perm_in, N, chunks, nc, v, nn, part);
-  rb_node_reduce_kernel<D, true><<<gn, D, 0, s>>>(part, nc, nodes, nn, mu, v);
-  for (int it = 1; it < kPowerIters; ++it) {
-    rb_power_kernel<D, false><<<gc, kRbThreads, 0, s>>>(X, perm_in, N, chunks, nc, v, nn, part);
-    rb_node_reduce_kernel<D, false><<<gn, D, 0, s>>>(part, nc, nodes, nn, mu, v);
+  if (D == 128 && lm.cov) {
+    const int4* cnodes = meta + P.nodes.size() + P.chunks.size() + lm.cnode_off;
+    const int4* cchunks = meta + P.nodes.size() + P.chunks.size() + P.cnodes.size() + lm.cchunk_off;
+    float* cpart = reinterpret_cast<float*>(ws + L.cpart);
+    uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.err);
+    const size_t smem = 1024 + 2 * kTcTile + 3 * 8 + 16 + 256 * 4 + 128 * 8 * 4;
+    e = cudaFuncSetAttribute(rb_cov_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    rb_cov_tc_kernel<<<dim3(lm.ncch, H), 128, smem, s>>>(X, perm_in, N, cchunks, lm.ncch, cpart,
+                                                         err);
+    const size_t nsmem = 128 * 128 * 4;
+    e = cudaFuncSetAttribute(rb_cov_node_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(nsmem));
+    if (e != cudaSuccess) return e;
+    rb_cov_node_kernel<<<gn, 128, nsmem, s>>>(cpart, lm.ncch, cnodes, nodes, nn, mu, v);
+  } else {
+    rb_power_kernel<D, true><<<gc, kRbThreads, 0, s>>>(X, perm_in, N, chunks, nc, v, nn, part);
+    rb_node_reduce_kernel<D, true><<<gn, D, 0, s>>>(part, nc, nodes, nn, mu, v);
+    for (int it = 1; it < kPowerIters; ++it) {
+      rb_power_kernel<D, false><<<gc, kRbThreads, 0, s>>>(X, perm_in, N, chunks, nc, v, nn, part);
+      rb_node_reduce_kernel<D, false><<<gn, D, 0, s>>>(part, nc, nodes, nn, mu, v);
+    }
   }
   rb_project_kernel<D><<<gc, kRbThreads, 0, s>>>(X, perm_in, N, chunks, v, nn, keys, hist);
   for (int shift = 24; shift >= 0; shift -= 8) {

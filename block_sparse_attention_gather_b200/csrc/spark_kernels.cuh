@@ -47,8 +47,8 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int H, int rows, int d);
 // ---- Spark-Reblock partitioner (reblock.cu)
 // Byte offsets of its workspace regions (256-byte aligned).
 struct ReblockLayout {
-  size_t mpart, M, W, Wb, X, perm0, perm1, keys, meta, part, mu, v, hist, state, cnt, base, err,
-      total;
+  size_t mpart, M, W, Wb, X, perm0, perm1, keys, meta, part, cpart, mu, v, hist, state, cnt, base,
+      err, total;
   int levels, nb;
 };
 
