@@ -364,7 +364,7 @@ def reblock_level_min_nodes(N, block):
     return out
 
 
-def reblock_bytes_flops(H, N, d, block, e_in, power_iters=4, moment_min_node=2048):
+def reblock_bytes_flops(H, N, d, block, e_in, power_iters=4, moment_min_node=256):
     """Algorithmic work of one partitioner call: the flops of the second moment and of the
     whitening (2 H N d^2 each; bf16 tensor-core MMAs for bf16 inputs), the HBM bytes of the
     whitening (read Q and K, write the bf16 unit rows), and the HBM bytes of the per-level
@@ -469,7 +469,7 @@ def run_reblock(args, world, rank, local):
                     "levels": {"ms": part_ms, "GB/s": gbs, "bytes": level_bytes}},
         # per call: 4 whitening kernels, the identity order, offsets, and per level 11
         # selection/scatter kernels plus 8 power-pass kernels or 2 node-moment kernels
-        "gpu_launches": (6 + sum(11 + (2 if (d == 128 and m >= 2048) else 8)
+        "gpu_launches": (6 + sum(11 + (2 if (d == 128 and m >= 256) else 8)
                                  for m in reblock_level_min_nodes(N, block))) * args.steps,
         "clocks": clock_info,
     }

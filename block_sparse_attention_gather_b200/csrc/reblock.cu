@@ -941,7 +941,7 @@ __global__ void __launch_bounds__(kRbThreads) rb_scatter_kernel(
 // matrix: v <- (S/n - mu mu^T) v, the same update as the row passes.
 
 constexpr int kCovChunk = 16384;      // tokens per CTA of the moment pass
-constexpr int kCovMinNode = 2048;     // smallest node size that takes this path
+constexpr int kCovMinNode = 256;     // smallest node size that takes this path
 constexpr int kCovStride = 128 * 128 + 128;   // floats per partial: x x^T, then sum x
 
 __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
