@@ -304,6 +304,22 @@ def dense_flops(w):
 
 # --------------------------------------------------------------------------------- main
 
+def max_over_ranks(x, world, device=None):
+    """The largest of every rank's value (the job's time is its slowest rank's); one
+    all-reduce on the default process group when world > 1."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, work_per_step, steps, total_ms):
+    """Whole-job throughput in TFLOP/s: every rank's work over the slowest rank's time."""
+    return world * work_per_step * steps / (total_ms / 1e3) / 1e12
+
+
 def init_dist():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -429,12 +445,7 @@ def run_reblock(args, world, rank, local):
     ev[1].record(stream)
     torch.cuda.synchronize()
     clock_info = clocks.stop()
-    total_ms = ev[0].elapsed_time(ev[1])
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([total_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[1]), world, device)
     ms = total_ms / args.steps
     # the whitening steps alone (same kernels as inside the call)
     pe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -532,15 +543,10 @@ def main():
         for j, n in enumerate(KERNELS):
             per_kernel[n].append(e[j].elapsed_time(e[j + 1]))
         totals.append(e[0].elapsed_time(e[5]))
-    total_ms = sum(totals)
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([total_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(totals), world, device)
     ms_per_step = total_ms / args.steps
     dflops = dense_flops(w)
-    value = world * dflops * args.steps / (total_ms / 1e3) / 1e12
+    value = whole_job_rate(world, dflops, args.steps, total_ms)
     flags = int(hp.v["err"].item())
     if flags:
         raise RuntimeError(f"device error word {flags:#x} after the timed region")
@@ -622,13 +628,8 @@ def main():
         e1.record(s)
         torch.cuda.synchronize()
         barrier()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            import torch.distributed as dist
-            tt = torch.tensor([e_ms], device=device, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
-        e2e = {"value": world * dflops * args.e2e_steps / (e_ms / 1e3) / 1e12, "unit": UNIT,
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+        e2e = {"value": whole_job_rate(world, dflops, args.e2e_steps, e_ms), "unit": UNIT,
                "ms_per_call": e_ms / args.e2e_steps, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "call": ("spark_bsa_forward_ctx after host-to-device copies" if hp.nc else
