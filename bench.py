@@ -584,8 +584,8 @@ def main():
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = out_host.numel() * out_host.element_size()
         s = torch.cuda.current_stream(device)
-        # without context tokens: the host-buffer entry point, pipelined by chunks of 4 heads
-        hpc = 4
+        # without context tokens: the host-buffer entry point, pipelined head by head
+        hpc = 1
         if not hp.nc:
             staging = torch.empty(spark_bsa_host_staging_size(hp.H, hp.N, hp.d, hp.out.dtype,
                                                               hp.nqb, hp.nkb, hpc),

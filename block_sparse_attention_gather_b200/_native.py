@@ -542,7 +542,7 @@ def _need_host(t, name, dtype=None):
 
 
 def spark_bsa_forward_host(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, topk_ratio, out=None,
-                           heads_per_chunk=4, device=None, staging=None, workspace=None,
+                           heads_per_chunk=1, device=None, staging=None, workspace=None,
                            streams=None):
     """The forward pass on HOST tensors (page-locked for overlap), pipelined by head chunks
     over three CUDA streams; returns `out` (host) once the work is enqueued on the compute
