@@ -6,25 +6,27 @@
 // a single row-wise softmax normalises both branches.
 //
 // One CTA per (query block A, head h); 11 warps with fixed roles:
-//   warps 0-3  softmax of the EVEN key tiles, warps 4-7 softmax of the ODD key tiles; warp w
-//              owns TMEM lanes 32*(w%4).. (query rows) and all 128 columns of its tiles.
-//              Each parity keeps its own online softmax (running max, running sum and O
-//              accumulator in TMEM) over its half of the tiles, so the two warps of an SMSP
-//              never wait for each other and drift out of phase: one is in its exponentials
-//              while the other waits for data.  The two partial results are merged once in
-//              the epilogue (max-shifted sums), which is exact.  Per tile: read the S row from
-//              TMEM twice (row max, then exponentials), apply the scale, the column mask or
-//              the summary offsets, rescale lazily (the max used for the exponentials only
-//              moves when a tile's max exceeds it by more than 8 in log2 units, and only then
-//              is the O row rescaled), and write P (bf16) over the S tile it came from.
+//   warps 0-3  softmax of the even key tiles, warps 4-7 of the odd key tiles (two groups);
+//              warp w owns TMEM lanes 32*(w%4).. (query rows).  Both groups exponentiate
+//              against one fixed reference per row, the larger of the two groups' first-tile
+//              row maxima, so no tile ever rescales anything: P(t) = 2^(s*scale - ref) is
+//              written (bf16) over the S columns it came from, each group sums its p, and the
+//              epilogue divides the single O accumulator by the two sums.  The exponentials
+//              are those of the exact softmax up to the common factor 2^(max - ref), which
+//              cancels in the division, so no accuracy is lost as long as every p stays in
+//              floating-point range.  A row whose sum leaves [2^-60, 2^60] (a maximum far above
+//              the reference, e.g. a sink or context key 50 nats above the first blocks)
+//              makes its CTA repeat all tiles with that row's true maximum as the reference
+//              (a second pass over the same pipeline; each chunk whose sum is out of range
+//              records its maximum, which is within a few units of the row's).
 //   warp 8     TMA producer: the Q tile once, then K tiles (3-stage ring).
 //   warp 9     TMA producer of V tiles (2-stage ring).
 //   warp 10    MMA issuer (one thread): S(t) = Q K^T (both from shared memory) into TMEM
-//              buffer t%2, O_{t%2} += P(t) V(t) (P read from TMEM, V an MN-major shared-memory
-//              operand).  Issue order S(0), S(1), PV(0), S(2), PV(1), S(3), ...: MMAs of one
-//              thread execute in order, so S(t+2) overwrites the buffer only after PV(t) has
-//              consumed P(t), and the commit of S(t+2) also covers PV(t) - the softmax of
-//              tile t+2 may rescale O_{t%2} once it sees S(t+2).
+//              buffer t%3, O += P(t) V(t) (P read from TMEM, V an MN-major shared-memory
+//              operand).  Issue order S(0), S(1), S(2), PV(0), S(3), PV(1), S(4), ...: MMAs
+//              of one thread execute in order, so S(t+3) overwrites its buffer only after
+//              PV(t) has consumed P(t).  With three buffers the next S of a group is ready
+//              while the group still works on its current tile.
 //
 // Tile list of a CTA: the k selected blocks in ascending order (a 128-row TMA box starting at
 // the block's first row; rows past the block are masked), then ceil(nc/128) tiles of the
@@ -32,8 +34,8 @@
 // budget; rows past nc masked), then ceil(nkb/128) tiles of the summary rows (rows past nkb
 // are zero-filled by TMA and masked, selected blocks masked).
 //
-// TMEM columns (512 allocated, one CTA per SM): S/P buffer 0 [0,128), buffer 1 [128,256),
-// O_even [256,256+D), O_odd [384,384+D).
+// TMEM columns (512 allocated, one CTA per SM): S/P buffers [0,128), [128,256), [256,384),
+// O [384,384+D).
 //
 // Every wait is bounded (spark_ptx.cuh); on expiry the kernel flags kErrTimeout, stops every
 // role, drains the copies and MMAs it issued, frees TMEM and returns.
@@ -47,21 +49,14 @@ constexpr int kKStages = 3;
 constexpr int kVStages = 2;
 constexpr int kWarpK = 8, kWarpV = 9, kWarpMma = 10;
 constexpr int kThreads = 352;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
+constexpr uint32_t kColO = 384;             // S/P buffer b at column 128*b (b < 3)
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr int kMaxSmemBias = 6144;          // summary offsets kept in shared memory (floats)
-
-// Which of a thread's exponential pairs go to the polynomial (FMA pipe) instead of MUFU.
-// Measured at 768p (attention ms, A/B in one run): none 77.1, a quarter 78.7, half 83.1 - the
-// softmax here is bound by latency and issue slots, not by MUFU throughput, so all pairs take
-// ex2.approx.  The polynomial path stays available (and tested) for kernels where it pays.
-__device__ __forceinline__ constexpr bool poly_pair(int) { return false; }
 
 struct __align__(8) Barriers {
   uint64_t qfull;
   uint64_t kfull[kKStages], kempty[kKStages], vfull[kVStages], vempty[kVStages];
-  uint64_t sfull[2], pready[2], done;
+  uint64_t sfull[3], pready[3], done;
 };
 
 __device__ __forceinline__ bool wait_bounded_ignore_abort(uint64_t* bar, uint32_t parity) {
@@ -162,29 +157,23 @@ __device__ __forceinline__ float max64(const float (&x)[64]) {
   return fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
 }
 
-// p = 2^(x*c - m) for 64 columns, packed to bf16 pairs; returns the sum of the p.
-__device__ __forceinline__ float exp64(const float (&x)[64], float c, float m,
-                                       uint32_t (&pk)[32]) {
+// p = 2^(x*c - m) for the 32 columns x[j0 .. j0+31], packed to bf16 pairs; returns their sum.
+__device__ __forceinline__ float exp32_at(const float (&x)[64], int j0, float c, float m,
+                                          uint32_t (&pk)[16]) {
   const uint64_t c2 = f2_splat(c);
   const uint64_t nm2 = f2_splat(-m);
-  uint64_t sum2[4] = {0, 0, 0, 0};
+  uint64_t sum2[2] = {0, 0};
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const uint64_t a2 = f2_fma(f2_pack(x[2 * j], x[2 * j + 1]), c2, nm2);
-    float p0, p1;
-    if (poly_pair(j)) {
-      exp2_poly2(a2, p0, p1);
-    } else {
-      float a0, a1;
-      f2_unpack(a2, a0, a1);
-      p0 = ex2_approx(a0);
-      p1 = ex2_approx(a1);
-    }
-    sum2[j & 3] = f2_add(sum2[j & 3], f2_pack(p0, p1));
+  for (int j = 0; j < 16; ++j) {
+    const uint64_t a2 = f2_fma(f2_pack(x[j0 + 2 * j], x[j0 + 2 * j + 1]), c2, nm2);
+    float a0, a1;
+    f2_unpack(a2, a0, a1);
+    const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+    sum2[j & 1] = f2_add(sum2[j & 1], f2_pack(p0, p1));
     pk[j] = pack_bf16(p0, p1);
   }
   float s0, s1;
-  f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
+  f2_unpack(f2_add(sum2[0], sum2[1]), s0, s1);
   return s0 + s1;
 }
 
@@ -218,9 +207,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
 
   const int A = blockIdx.x, h = blockIdx.y;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  __shared__ int s_skip;
-  __shared__ float ex_m[2][128], ex_l[2][128];   // [parity][row] for the epilogue merge
-  if (tid == 0) s_skip = launch_timed_out(err) ? 1 : 0;   // an earlier CTA gave up
+  __shared__ int s_skip, s_rerun;
+  // [group][row]: first-tile maxima (the reference), then sums and maxima for the epilogue
+  __shared__ float ex_m[2][128], ex_l[2][128], ex_mt[2][128];
+  if (tid == 0) {
+    s_skip = launch_timed_out(err) ? 1 : 0;                // an earlier CTA gave up
+    s_rerun = 0;
+  }
   __syncthreads();
   if (s_skip) return;                                      // uniform: no work, nothing held
   const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
@@ -241,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       mbar_init(&bars->vfull[s], 1);
       mbar_init(&bars->vempty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
       mbar_init(&bars->sfull[b], 1);
       mbar_init(&bars->pready[b], 4 * 32);
     }
@@ -272,218 +265,236 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   __syncthreads();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == kWarpK || warp == kWarpV) {
-    // ------------------------------------------------------------- TMA producers
-    if (lane == 0) {
-      const bool is_k = (warp == kWarpK);
-      const int stages = is_k ? kKStages : kVStages;
-      uint8_t* ring = is_k ? kst : vst;
-      uint64_t* full = is_k ? bars->kfull : bars->vfull;
-      uint64_t* empty = is_k ? bars->kempty : bars->vempty;
-      const CUtensorMap* mx = is_k ? &map_k : &map_v;
-      const CUtensorMap* mc = is_k ? &map_kc : &map_vc;
-      const CUtensorMap* ms = is_k ? &map_kt : &map_vt;
-      tma_prefetch_desc(mx);
-      tma_prefetch_desc(ms);
-      if (nxt > 0) tma_prefetch_desc(mc);
-      if (is_k) {
-        tma_prefetch_desc(&map_q);
-        mbar_arrive_expect_tx(&bars->qfull, TILE_BYTES);
-        const int qrow = min(max(qlo, 0), N - 1);   // rows past the block are never stored
-        for (int a = 0; a < NATOM; ++a)
-          tma_load_3d(qst + a * 16384, &map_q, &bars->qfull, a * 64, qrow, h);
-      }
-      int issued = 0;
-      TileInfo next = tile_info(0, k, nxt, nc, sel_row, k_offsets, nkb, N);
-      for (int t = 0; t < T; ++t) {
-        const int s = t % stages;
-        const TileInfo ti = next;
-        if (t >= stages && !mbar_wait(&empty[s], ((t / stages) - 1) & 1, abort_flag, err)) break;
-        mbar_arrive_expect_tx(&full[s], TILE_BYTES);
-        const CUtensorMap* map = ti.src == kSrcVideo ? mx : (ti.src == kSrcContext ? mc : ms);
-        for (int a = 0; a < NATOM; ++a)
-          tma_load_3d(ring + s * TILE_BYTES + a * 16384, map, &full[s], a * 64, ti.y, h);
-        issued = t + 1;
-        if (t + 1 < T) next = tile_info(t + 1, k, nxt, nc, sel_row, k_offsets, nkb, N);
-      }
-      if (*abort_flag) {
-        // drain: wait for every load still in flight (the last round of each stage)
-        for (int t = max(0, issued - stages); t < issued; ++t)
-          wait_bounded_ignore_abort(&full[t % stages], (t / stages) & 1);
-        if (is_k) wait_bounded_ignore_abort(&bars->qfull, 0);
-      }
-    }
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idO = idesc_bf16(128, D, false, true);
-      // descriptors built once; per MMA only a compile-time offset (16-byte units) changes
-      const uint64_t qd = sdesc_sw128(smem_u32(qst), 16, 1024);
-      const uint64_t kdesc0 = sdesc_sw128(smem_u32(kst), 16, 1024);
-      const uint64_t vdesc0 = sdesc_sw128(smem_u32(vst), 16384, 1024);
-      bool ok = mbar_wait(&bars->qfull, 0, abort_flag, err);
-      auto issue_s = [&](int t) -> bool {
-        const int s = t % kKStages;
-        if (!mbar_wait(&bars->kfull[s], (t / kKStages) & 1, abort_flag, err)) return false;
-        const uint32_t dcol = tbase + ((t & 1) ? kColS1 : kColS0);
-        const uint64_t kd = kdesc0 + static_cast<uint64_t>(s * (TILE_BYTES >> 4));
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) / 16;
-          mma_ss(dcol, qd + off, kd + off, idS, kk > 0 ? 1u : 0u);
+  // Pass 0 exponentiates every tile against a fixed reference per row (the larger of the two
+  // groups' first-tile maxima) and tracks the true row maximum.  A CTA with a row whose sum
+  // leaves [2^-60, 2^60] (a maximum far above the reference) runs pass 1 over the same tiles
+  // with the true maximum as the reference.  Barrier phases count tiles over both passes.
+  float m_true = -INFINITY;                        // softmax threads: row maximum (log2 units)
+  int issued = 0;                                  // producers: loads issued over both passes
+  for (int pass = 0; pass < 2; ++pass) {
+    const int tg0 = pass * T;                      // tile counter of this pass's first tile
+    if (warp == kWarpK || warp == kWarpV) {
+      // ----------------------------------------------------------- TMA producers
+      if (lane == 0) {
+        const bool is_k = (warp == kWarpK);
+        const int stages = is_k ? kKStages : kVStages;
+        uint8_t* ring = is_k ? kst : vst;
+        uint64_t* full = is_k ? bars->kfull : bars->vfull;
+        uint64_t* empty = is_k ? bars->kempty : bars->vempty;
+        const CUtensorMap* mx = is_k ? &map_k : &map_v;
+        const CUtensorMap* mc = is_k ? &map_kc : &map_vc;
+        const CUtensorMap* ms = is_k ? &map_kt : &map_vt;
+        if (pass == 0) {
+          tma_prefetch_desc(mx);
+          tma_prefetch_desc(ms);
+          if (nxt > 0) tma_prefetch_desc(mc);
+          if (is_k) {
+            tma_prefetch_desc(&map_q);
+            mbar_arrive_expect_tx(&bars->qfull, TILE_BYTES);
+            const int qrow = min(max(qlo, 0), N - 1);   // rows past the block are never stored
+            for (int a = 0; a < NATOM; ++a)
+              tma_load_3d(qst + a * 16384, &map_q, &bars->qfull, a * 64, qrow, h);
+          }
         }
-        tc_commit(&bars->sfull[t & 1]);
-        tc_commit(&bars->kempty[s]);
-        return true;
-      };
-      if (ok && T > 0) ok = issue_s(0);
-      if (ok && T > 1) ok = issue_s(1);
-      for (int t = 0; ok && t < T; ++t) {
-        if (!mbar_wait(&bars->pready[t & 1], (t >> 1) & 1, abort_flag, err)) break;
-        tc_fence_after_sync();
-        const int s = t % kVStages;
-        if (!mbar_wait(&bars->vfull[s], (t / kVStages) & 1, abort_flag, err)) break;
-        const uint64_t vd = vdesc0 + static_cast<uint64_t>(s * (TILE_BYTES >> 4));
-        const uint32_t pcol = tbase + ((t & 1) ? kColS1 : kColS0);   // P(t) over S(t)
-        const uint32_t ocol = tbase + ((t & 1) ? kColO1 : kColO0);
-        const uint32_t acc0 = t >= 2 ? 1u : 0u;                       // first tile of a parity
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(ocol, pcol + kk * 8, vd + (kk * 2048) / 16, idO, kk > 0 ? 1u : acc0);
-        tc_commit(&bars->vempty[s]);
-        if (t + 2 < T && !(ok = issue_s(t + 2))) break;
+        TileInfo next = tile_info(0, k, nxt, nc, sel_row, k_offsets, nkb, N);
+        for (int t = 0; t < T; ++t) {
+          const int tg = tg0 + t;
+          const int s = tg % stages;
+          const TileInfo ti = next;
+          if (tg >= stages && !mbar_wait(&empty[s], ((tg / stages) - 1) & 1, abort_flag, err))
+            break;
+          mbar_arrive_expect_tx(&full[s], TILE_BYTES);
+          const CUtensorMap* map = ti.src == kSrcVideo ? mx : (ti.src == kSrcContext ? mc : ms);
+          for (int a = 0; a < NATOM; ++a)
+            tma_load_3d(ring + s * TILE_BYTES + a * 16384, map, &full[s], a * 64, ti.y, h);
+          issued = tg + 1;
+          if (t + 1 < T) next = tile_info(t + 1, k, nxt, nc, sel_row, k_offsets, nkb, N);
+        }
+        if (*abort_flag) {
+          // drain: wait for every load still in flight (the last round of each stage)
+          for (int tg = max(0, issued - stages); tg < issued; ++tg)
+            wait_bounded_ignore_abort(&full[tg % stages], (tg / stages) & 1);
+          if (is_k) wait_bounded_ignore_abort(&bars->qfull, 0);
+        }
       }
-      // every MMA complete: the softmax epilogue reads O, and TMEM is freed afterwards
-      tc_commit(&bars->done);
-      wait_bounded_ignore_abort(&bars->done, 0);
-    }
-  } else {
-    // ------------------------------------------------------------------ softmax rows
-    const int q4 = warp & 3, par = warp >> 2;            // row quarter, tile parity
-    const int row = q4 * 32 + lane;                      // 0..127 == TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    const uint32_t sbuf = tbase + lane_off + (par ? kColS1 : kColS0);
-    const uint32_t obuf = tbase + lane_off + (par ? kColO1 : kColO0);
-    const float scale_log2 = kLog2e * rsqrtf(static_cast<float>(D));
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true, first = true;
-    TileInfo next = tile_info(par, k, nxt, nc, sel_row, k_offsets, nkb, N);
-    for (int t = par; t < T; t += 2) {
-      const TileInfo ti = next;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->sfull[par], (t >> 1) & 1, abort_flag, err));
-      if (!ok) break;
-      tc_fence_after_sync();
-      if (t + 2 < T) next = tile_info(t + 2, k, nxt, nc, sel_row, k_offsets, nkb, N);
-      const float c = ti.exact ? scale_log2 : 1.f;
-      // pass 1: the tile's row maximum (log2 units)
+    } else if (warp == kWarpMma) {
+      // ---------------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
+        constexpr uint32_t idO = idesc_bf16(128, D, false, true);
+        // descriptors built once; per MMA only a compile-time offset (16-byte units) changes
+        const uint64_t qd = sdesc_sw128(smem_u32(qst), 16, 1024);
+        const uint64_t kdesc0 = sdesc_sw128(smem_u32(kst), 16, 1024);
+        const uint64_t vdesc0 = sdesc_sw128(smem_u32(vst), 16384, 1024);
+        bool ok = pass > 0 || mbar_wait(&bars->qfull, 0, abort_flag, err);
+        // S(t) of this pass into buffer (tg0 + t) % 3
+        auto issue_s = [&](int t) -> bool {
+          const int tg = tg0 + t;
+          const int s = tg % kKStages;
+          if (!mbar_wait(&bars->kfull[s], (tg / kKStages) & 1, abort_flag, err)) return false;
+          const uint32_t dcol = tbase + (tg % 3) * 128;
+          const uint64_t kd = kdesc0 + static_cast<uint64_t>(s * (TILE_BYTES >> 4));
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) / 16;
+            mma_ss(dcol, qd + off, kd + off, idS, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bars->sfull[tg % 3]);
+          tc_commit(&bars->kempty[s]);
+          return true;
+        };
+        for (int t = 0; ok && t < min(T, 3); ++t) ok = issue_s(t);
+        for (int t = 0; ok && t < T; ++t) {
+          const int tg = tg0 + t;
+          if (!mbar_wait(&bars->pready[tg % 3], (tg / 3) & 1, abort_flag, err)) break;
+          tc_fence_after_sync();
+          const int s = tg % kVStages;
+          if (!mbar_wait(&bars->vfull[s], (tg / kVStages) & 1, abort_flag, err)) break;
+          const uint64_t vd = vdesc0 + static_cast<uint64_t>(s * (TILE_BYTES >> 4));
+          const uint32_t pcol = tbase + (tg % 3) * 128;               // P(t) over S(t)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tbase + kColO, pcol + kk * 8, vd + (kk * 2048) / 16, idO,
+                   (kk > 0 || t > 0) ? 1u : 0u);
+          tc_commit(&bars->vempty[s]);
+          // S(t+3) reuses the columns of P(t): issued after PV(t), and MMAs of one thread
+          // execute in order
+          if (t + 3 < T && !(ok = issue_s(t + 3))) break;
+        }
+        // every MMA complete: the softmax epilogue reads O, and TMEM is reused or freed after
+        tc_commit(&bars->done);
+        wait_bounded_ignore_abort(&bars->done, pass);
+      }
+    } else {
+      // ---------------------------------------------------------------- softmax rows
+      const int q4 = warp & 3, grp = warp >> 2;          // row quarter, tile group
+      const int row = q4 * 32 + lane;                    // 0..127 == TMEM lane
+      const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+      const float scale_log2 = kLog2e * rsqrtf(static_cast<float>(D));
+      float l_run = 0.f;
+      bool ok = true;
       float x[64];
-      load_logits<kBiasSmem>(sbuf, 0, ti, scale_log2, biasrow, cb, selmask, nkb, x);
-      float mt = max64(x);
-      load_logits<kBiasSmem>(sbuf + 64, 64, ti, scale_log2, biasrow, cb, selmask, nkb, x);
-      mt = fmaxf(mt, max64(x));
-      if (ti.exact) mt *= scale_log2;                    // -inf stays -inf
-      bool need = false;
-      float m_new = m_run;
-      if (first) {
-        m_new = mt;
-      } else if (mt > m_run + kRescaleThreshold) {
-        need = true;
-        m_new = mt;
-      }
-      // O of this parity is settled (the commit of S(t) covers PV(t-2)); rescale it if the
-      // max moved
-      if (__any_sync(0xffffffffu, need)) {
-        const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
-        l_run *= alpha;
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t r[32];
-          tmem_ld32(obuf + cc * 32, r);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-          tmem_st32(obuf + cc * 32, r);
+      float m_ref;
+      if (pass == 0) {
+        // reference: the row maximum of the first tile of each group, shared by both
+        float mt = -INFINITY;
+        if (grp < T) {
+          const int tg = tg0 + grp;
+          const TileInfo ti = tile_info(grp, k, nxt, nc, sel_row, k_offsets, nkb, N);
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(&bars->sfull[tg % 3], (tg / 3) & 1, abort_flag, err));
+          if (ok) {
+            tc_fence_after_sync();
+            const uint32_t sbuf = tbase + lane_off + (tg % 3) * 128;
+            load_logits<kBiasSmem>(sbuf, 0, ti, scale_log2, biasrow, cb, selmask, nkb, x);
+            mt = max64(x);
+            load_logits<kBiasSmem>(sbuf + 64, 64, ti, scale_log2, biasrow, cb, selmask, nkb, x);
+            mt = fmaxf(mt, max64(x));
+            if (ti.exact) mt *= scale_log2;
+          }
         }
+        ex_m[grp][row] = mt;
+        named_bar_sync(1 + q4, 64);                      // the two groups of this quarter
+        m_ref = fmaxf(ex_m[0][row], ex_m[1][row]);
+      } else {
+        m_ref = m_true;                                  // both groups' maximum (epilogue)
       }
-      // pass 2: exponentials, P written over the S columns already consumed
-      uint32_t pk[32];
-      load_logits<kBiasSmem>(sbuf, 0, ti, scale_log2, biasrow, cb, selmask, nkb, x);
-      float rowsum = exp64(x, c, m_new, pk);
-      tmem_st32(sbuf, pk);
-      load_logits<kBiasSmem>(sbuf + 64, 64, ti, scale_log2, biasrow, cb, selmask, nkb, x);
-      rowsum += exp64(x, c, m_new, pk);
-      tmem_st32(sbuf + 32, pk);
-      l_run = first ? rowsum : l_run + rowsum;
-      m_run = m_new;
-      first = false;
-      tc_fence_before_sync();
-      mbar_arrive(&bars->pready[par]);
-    }
-    // ---- epilogue: merge the two parities and scatter O / l to the original token order
-    bool fine = ok && T > 0;
-    if (fine) fine = __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, abort_flag, err));
-    ex_m[par][row] = m_run;
-    ex_l[par][row] = l_run;
-    named_bar_sync(1 + q4, 64);                          // the two parities of this quarter
-    if (fine) {
-      tc_fence_after_sync();
-      const float m_o = ex_m[par ^ 1][row], l_o = ex_l[par ^ 1][row];
-      const float M = fmaxf(m_run, m_o);
-      // weights of the two partial results (a parity without tiles has l = 0)
-      const float w_self = l_run > 0.f ? ex2_approx(m_run - M) : 0.f;
-      const float w_oth = l_o > 0.f ? ex2_approx(m_o - M) : 0.f;
-      const float inv = 1.f / (l_run * w_self + l_o * w_oth);
-      const float ws = w_self * inv, wo = w_oth * inv;
-      const int qsize = max(0, min(q_offsets[A + 1] - qlo, kMaxBlock));
-      int tok = -1;
-      if (row < qsize) {
-        tok = q_perm[static_cast<size_t>(h) * N + qlo + row];
-        if (tok < 0 || tok >= N) {
-          if (par == 0) flag_error(err, kErrPerm);
-          tok = -1;
+      if (!(m_ref > -INFINITY)) m_ref = 0.f;
+      TileInfo next = tile_info(grp, k, nxt, nc, sel_row, k_offsets, nkb, N);
+      for (int t = grp; ok && t < T; t += 2) {
+        const TileInfo ti = next;
+        const int tg = tg0 + t;
+        const int b = tg % 3;
+        if (pass > 0 || t >= 2) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars->sfull[b], (tg / 3) & 1, abort_flag, err));
+          if (!ok) break;
+          tc_fence_after_sync();
         }
+        if (t + 2 < T) next = tile_info(t + 2, k, nxt, nc, sel_row, k_offsets, nkb, N);
+        const uint32_t sbuf = tbase + lane_off + b * 128;
+        const float c = ti.exact ? scale_log2 : 1.f;
+        // The row maximum is only needed for a repeat, and only to within a few units: a
+        // chunk whose sum stays in [2^-40, 2^40] has its maximum within 40 of the reference
+        // and cannot drive the row sum out of [2^-60, 2^60] (fewer than 2^16 chunks per row),
+        // so only chunks outside that range (rare) take their maximum.
+        float rowsum = 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          load_logits<kBiasSmem>(sbuf + half * 64, half * 64, ti, scale_log2, biasrow, cb,
+                                 selmask, nkb, x);
+          uint32_t p16[16];
+          float cs = exp32_at(x, 0, c, m_ref, p16);
+          tmem_st16(sbuf + half * 32, p16);
+          cs += exp32_at(x, 32, c, m_ref, p16);
+          tmem_st16(sbuf + half * 32 + 16, p16);
+          if (!(cs >= 0x1p-40f && cs <= 0x1p40f)) {
+            const float mt = max64(x);
+            m_true = fmaxf(m_true, ti.exact ? mt * scale_log2 : mt);
+          }
+          rowsum += cs;
+        }
+        l_run += rowsum;
+        tc_fence_before_sync();
+        mbar_arrive(&bars->pready[b]);
       }
-      // each parity's warp writes half of the d output columns
-      const uint32_t o_self = tbase + lane_off + (par ? kColO1 : kColO0);
-      const uint32_t o_oth = tbase + lane_off + (par ? kColO0 : kColO1);
-      constexpr int HALF = D / 2;
-      // TMEM of a parity that never ran holds garbage: skip it (the weights are 0 there)
-      const bool self_live = __any_sync(0xffffffffu, l_run > 0.f);
-      const bool oth_live = __any_sync(0xffffffffu, l_o > 0.f);
-#pragma unroll
-      for (int cc = 0; cc < HALF / 32; ++cc) {
-        const int col = par * HALF + cc * 32;
-        uint32_t a[32], b[32];
-        if (self_live) tmem_ld32(o_self + col, a);
-        else for (int j = 0; j < 32; ++j) a[j] = 0u;
-        if (oth_live) tmem_ld32(o_oth + col, b);
-        else for (int j = 0; j < 32; ++j) b[j] = 0u;
-        float o[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float av = w_self > 0.f ? __uint_as_float(a[j]) * ws : 0.f;
-          const float bv = w_oth > 0.f ? __uint_as_float(b[j]) * wo : 0.f;
-          o[j] = av + bv;
+      // ---- epilogue: O / (l_0 + l_1), scattered to the original token order
+      bool fine = ok && T > 0;
+      if (fine) fine = __all_sync(0xffffffffu, mbar_wait(&bars->done, pass, abort_flag, err));
+      ex_l[grp][row] = l_run;
+      ex_mt[grp][row] = m_true;
+      named_bar_sync(1 + q4, 64);
+      const float l_tot = ex_l[0][row] + ex_l[1][row];
+      m_true = fmaxf(ex_mt[0][row], ex_mt[1][row]);
+      if (fine) {
+        tc_fence_after_sync();
+        const int qsize = max(0, min(q_offsets[A + 1] - qlo, kMaxBlock));
+        // a sum outside the window means the reference was far from the row maximum
+        if (pass == 0 && row < qsize && !(l_tot >= 0x1p-60f && l_tot <= 0x1p60f))
+          s_rerun = 1;
+        const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+        int tok = -1;
+        if (row < qsize) {
+          tok = q_perm[static_cast<size_t>(h) * N + qlo + row];
+          if (tok < 0 || tok >= N) {
+            if (grp == 0) flag_error(err, kErrPerm);
+            tok = -1;
+          }
         }
-        if (tok >= 0) {
-          const size_t off = (static_cast<size_t>(h) * N + tok) * D + col;
-          if (out_dtype == 0) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + off);
+        // each group's warp writes half of the d output columns
+        constexpr int HALF = D / 2;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(pack_bf16(o[8 * j], o[8 * j + 1]),
-                                  pack_bf16(o[8 * j + 2], o[8 * j + 3]),
-                                  pack_bf16(o[8 * j + 4], o[8 * j + 5]),
-                                  pack_bf16(o[8 * j + 6], o[8 * j + 7]));
-          } else {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + off);
+        for (int cc = 0; cc < HALF / 32; ++cc) {
+          const int col = grp * HALF + cc * 32;
+          uint32_t a[32];
+          tmem_ld32(tbase + lane_off + kColO + col, a);
+          float o[32];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+          for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(a[j]) * inv;
+          if (tok >= 0) {
+            const size_t off = (static_cast<size_t>(h) * N + tok) * D + col;
+            if (out_dtype == 0) {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + off);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dst[j] = make_uint4(pack_bf16(o[8 * j], o[8 * j + 1]),
+                                    pack_bf16(o[8 * j + 2], o[8 * j + 3]),
+                                    pack_bf16(o[8 * j + 4], o[8 * j + 5]),
+                                    pack_bf16(o[8 * j + 6], o[8 * j + 7]));
+            } else {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + off);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+            }
           }
         }
       }
     }
+    // every role is done with this pass (TMEM reads included) before the next one starts
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (pass == 1 || !s_rerun || *abort_flag) break;   // uniform: written before the barrier
   }
   tc_fence_before_sync();
   __syncthreads();

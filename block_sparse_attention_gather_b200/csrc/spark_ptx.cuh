@@ -314,29 +314,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA/ALU pipes (relieves the MUFU pipe, which is as busy as the tensor cores in
-// the attention softmax).  Range reduction x = j + f with j = round(x) (adding 1.5*2^23 makes
-// the FADD round to an integer held in the low mantissa bits) and |f| <= 1/2; 2^f by a
-// degree-3 polynomial whose coefficients are a Lawson-reweighted least-squares fit of the
-// relative error on [-1/2, 1/2] (max relative error 7.5e-5, far below bf16's 2^-9); j is then
-// added to the exponent field.  x is clamped to >= -126 so the exponent cannot wrap, so
-// -inf gives 2^-126 instead of 0.
-constexpr float kExp2C0 = 0.9999280572f;
-constexpr float kExp2C1 = 0.6932609677f;
-constexpr float kExp2C2 = 0.2426111251f;
-constexpr float kExp2C3 = 0.0551716648f;
-constexpr float kRoundMagic = 12582912.f;           // 1.5 * 2^23
-
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + kRoundMagic;
-  const float j = t - kRoundMagic;
-  const float f = x - j;
-  float p = fmaf(kExp2C3, f, kExp2C2);
-  p = fmaf(p, f, kExp2C1);
-  p = fmaf(p, f, kExp2C0);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
 
 // ---- packed fp32x2 arithmetic (sm_100): two fp32 lanes in one 64-bit register pair
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
@@ -371,23 +348,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// exp2_poly on a packed pair: the same steps with the FMA-pipe work done two lanes at a time.
-__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& r0, float& r1) {
-  float x0, x1;
-  f2_unpack(x2, x0, x1);
-  x2 = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const uint64_t t2 = f2_add(x2, f2_splat(kRoundMagic));
-  const uint64_t j2 = f2_add(t2, f2_splat(-kRoundMagic));
-  const uint64_t f = f2_fma(j2, f2_splat(-1.f), x2);
-  uint64_t p = f2_fma(f2_splat(kExp2C3), f, f2_splat(kExp2C2));
-  p = f2_fma(p, f, f2_splat(kExp2C1));
-  p = f2_fma(p, f, f2_splat(kExp2C0));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t2, t0, t1);
-  r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

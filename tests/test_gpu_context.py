@@ -94,6 +94,23 @@ def test_context_ratio_one_is_dense_attention():
         P.compare_out(P.to64(out[h]), O.dense_attention(q, k, v), "dense with context")
 
 
+def test_sink_logit_far_above_the_video_rows():
+    """A context (sink) key ~100 nats above every video logit of every query: the context
+    tiles come after the video tiles, so the reference taken from the first two tiles is far
+    below the row maxima and the attention repeats those query blocks with the true maxima."""
+    x = custom_inputs(75, H=2, N=2000, d=128, dtype="bf16", lo=40, hi=128)
+    H, N, d = x["Q"].shape
+    g = torch.Generator().manual_seed(76)
+    u = torch.randn(d, generator=g, dtype=torch.float64)
+    u /= u.norm()
+    x["Q"] = (x["Q"].cpu().double() + 6.0 * u).to(x["Q"].dtype).to(DEV)
+    x = with_context(x, 77, 40)
+    Kc = x["Kc"].cpu().clone()
+    Kc[:, 17] = (300.0 * u).to(Kc.dtype)
+    x["Kc"] = Kc.to(DEV)
+    check_forward_ctx(x, 0.2)
+
+
 def test_empty_context_is_the_plain_call():
     x = custom_inputs(65, H=2, N=3000, d=128, dtype="bf16", lo=50, hi=128)
     a, _, _ = spark_bsa_forward(x["Q"], x["K"], x["V"], x["q_perm"], x["k_perm"],

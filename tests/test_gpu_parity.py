@@ -127,6 +127,55 @@ def test_ratio_one_is_dense_attention():
         P.compare_out(P.to64(out[h]), ref, "dense")
 
 
+def plant_far_key(x, offset, scale, seed):
+    """Queries share a direction u (offset * u added to every row) and the first key of the
+    last key block is scale * u in every head, so its logit lies far above the logits of the
+    first key tiles of every query block."""
+    H, N, d = x["Q"].shape
+    g = torch.Generator().manual_seed(seed)
+    u = torch.randn(d, generator=g, dtype=torch.float64)
+    u /= u.norm()
+    Q = (x["Q"].cpu().double() + offset * u).to(x["Q"].dtype)
+    K = x["K"].cpu().clone()
+    last = int(x["k_offsets"][-2])
+    for h in range(H):
+        K[h, int(x["k_perm"][h, last])] = (scale * u).to(K.dtype)
+    x = dict(x)
+    x["Q"], x["K"] = Q.to(DEV), K.to(DEV)
+    return x, last
+
+
+def test_logit_far_above_the_first_tiles():
+    """The attention exponentiates against a reference taken from the first two key tiles of
+    each query block and repeats a query block whose row sums leave [2^-60, 2^60] with the
+    true row maxima.  Here a key in the last block sits ~100 nats above every logit of the
+    first two blocks, which forces the repeat; dense attention (ratio 1) in float64 is the
+    reference."""
+    x = custom_inputs(71, H=2, N=1800, d=128, dtype="fp32", lo=60, hi=128)
+    x, last = plant_far_key(x, 6.0, 300.0, 72)
+    H, N, d = x["Q"].shape
+    second = int(x["k_offsets"][2])
+    for h in range(H):
+        hi = P.head_inputs(x, h)
+        s = hi["Q"] @ hi["K"][hi["k_perm"]].T / math.sqrt(d)
+        gap = s[:, last] - s[:, :second].max(axis=1)
+        assert np.mean(gap > 60 * math.log(2)) > 0.9    # beyond the window for most rows
+    # (the summaries' bias is checked elsewhere: at ~150-nat logits its bf16 rounding of k~
+    # exceeds that check's absolute bound, while the output is insensitive to it)
+    out, _ = check_forward(x, 1.0, check_inter=False)
+    for h in range(H):
+        q, k, v = P.bf16_64(x["Q"][h]), P.bf16_64(x["K"][h]), P.bf16_64(x["V"][h])
+        P.compare_out(P.to64(out[h]), O.dense_attention(q, k, v), "dense, far key")
+
+
+def test_logit_far_above_at_a_sparse_ratio():
+    """The same planted key at ratio 0.1: it sits in the exact branch of the query blocks that
+    select the last block and in the compressed branch (through k~, c) of the others."""
+    x = custom_inputs(73, H=2, N=2600, d=128, dtype="bf16", lo=40, hi=128)
+    x, _ = plant_far_key(x, 6.0, 300.0, 74)
+    check_forward(x, 0.1, check_inter=False)
+
+
 @pytest.mark.parametrize("case", ["single_token", "one_block", "unit_blocks", "two_summary_tiles",
                                   "q_reuse_k", "k_equals_nkb_minus_1"])
 def test_edge_cases(case):
