@@ -24,7 +24,8 @@ __all__ = [
     "spark_bsa_attend_ctx", "ReblockLayout", "spark_reblock_workspace_layout",
     "spark_reblock_workspace_size", "spark_reblock_levels", "spark_reblock",
     "spark_reblock_whiten", "spark_reblock_level", "reblock_views",
-    "spark_bsa_host_staging_size", "spark_bsa_forward_host",
+    "spark_bsa_host_staging_size", "spark_bsa_forward_host", "spark_bsa_quantize_fp8",
+    "spark_bsa_attend_fp8", "spark_bsa_workspace_size_fp8", "spark_bsa_forward_fp8",
 ]
 
 SPARK_BF16, SPARK_F32 = 0, 1
@@ -37,7 +38,8 @@ EXPORTED = [
     "spark_bsa_workspace_size_ctx", "spark_bsa_forward_ctx", "spark_bsa_context_bf16",
     "spark_bsa_attend_ctx", "spark_reblock_workspace_layout", "spark_reblock_workspace_size",
     "spark_reblock_levels", "spark_reblock", "spark_reblock_whiten", "spark_reblock_level",
-    "spark_bsa_host_staging_size", "spark_bsa_forward_host",
+    "spark_bsa_host_staging_size", "spark_bsa_forward_host", "spark_bsa_quantize_fp8",
+    "spark_bsa_attend_fp8", "spark_bsa_workspace_size_fp8", "spark_bsa_forward_fp8",
 ]
 REBLOCK_MODES = {"q_reuse_k": 0, "separate": 1}
 
@@ -108,6 +110,12 @@ def lib():
         "spark_bsa_host_staging_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
         "spark_bsa_forward_host": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _I, _D,
                                         _P, _I, _P, _SZ, _P, _SZ, _P, _P, _P]),
+        "spark_bsa_quantize_fp8": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P]),
+        "spark_bsa_attend_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I,
+                                      _P, _P, _I, _P, _I, _I, _I, _I, _P, _I, _P, _P]),
+        "spark_bsa_workspace_size_fp8": (_SZ, [_I, _I, _I, _I, _I, _D, _I]),
+        "spark_bsa_forward_fp8": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _I,
+                                       _P, _I, _D, _P, _P, _SZ, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -446,6 +454,108 @@ def spark_bsa_attend_ctx(Qp, Kp, Vp, k_tilde, v_tilde, cbias, sel, Kc, Vc, q_per
                                     _stream(stream))
     _check("spark_bsa_attend_ctx", st)
     return out
+
+
+# ------------------------------------------------------------------------- FP8 logits
+
+def spark_bsa_quantize_fp8(src, group_offsets=None, dst=None, scales=None, err=None,
+                           stream=None):
+    """e4m3 codes (torch.uint8 [H, R, d]) and power-of-two group scales (fp32 [H, ngroups]) of
+    bf16 rows src [H, R, d]; groups are the blocks of group_offsets (int32 [ngroups+1]) or,
+    when it is None, 128-row tiles.  Returns (dst, scales)."""
+    _need(src, "src", torch.bfloat16)
+    dev = src.device
+    H, R, d = src.shape
+    if group_offsets is None:
+        ngroups = (R + 127) // 128
+    else:
+        _need(group_offsets, "group_offsets", torch.int32, dev)
+        ngroups = group_offsets.numel() - 1
+    if dst is None:
+        dst = torch.empty(H, R, d, dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(H, ngroups, dtype=torch.float32, device=dev)
+    _need(dst, "dst", torch.uint8, dev)
+    _need(scales, "scales", torch.float32, dev)
+    st = lib().spark_bsa_quantize_fp8(_ptr(src), H, R, d, _ptr(group_offsets), ngroups,
+                                      _ptr(dst), _ptr(scales), _ptr(err), _stream(stream))
+    _check("spark_bsa_quantize_fp8", st)
+    return dst, scales
+
+
+def spark_bsa_attend_fp8(Qp8, q_scale, Kp8, k_scale, Vp, kt8, kt_scale, v_tilde, cbias, sel,
+                         q_perm, q_offsets, k_offsets, Kc8=None, kc_scale=None, Vc=None,
+                         out_dtype=torch.bfloat16, out=None, err=None, stream=None):
+    """The attention step with FP8 logits (codes and scales from spark_bsa_quantize_fp8,
+    values in bf16; d = 128)."""
+    _need(Qp8, "Qp8", torch.uint8)
+    dev = Qp8.device
+    H, N, d = Qp8.shape
+    for n, t, dt in (("q_scale", q_scale, torch.float32), ("Kp8", Kp8, torch.uint8),
+                     ("k_scale", k_scale, torch.float32), ("Vp", Vp, torch.bfloat16),
+                     ("kt8", kt8, torch.uint8), ("kt_scale", kt_scale, torch.float32),
+                     ("v_tilde", v_tilde, torch.bfloat16), ("cbias", cbias, torch.float32),
+                     ("sel", sel, torch.int32), ("q_perm", q_perm, torch.int32),
+                     ("q_offsets", q_offsets, torch.int32), ("k_offsets", k_offsets, torch.int32)):
+        _need(t, n, dt, dev)
+    nc = 0
+    if Kc8 is not None:
+        _need(Kc8, "Kc8", torch.uint8, dev)
+        _need(kc_scale, "kc_scale", torch.float32, dev)
+        _need(Vc, "Vc", torch.bfloat16, dev)
+        nc = Kc8.shape[1]
+    nqb, nkb = q_offsets.numel() - 1, k_offsets.numel() - 1
+    k = sel.shape[-1]
+    if out is None:
+        out = torch.empty(H, N, d, dtype=out_dtype, device=dev)
+    _need(out, "out", out_dtype, dev)
+    st = lib().spark_bsa_attend_fp8(_ptr(Qp8), _ptr(q_scale), _ptr(Kp8), _ptr(k_scale), _ptr(Vp),
+                                    _ptr(kt8), _ptr(kt_scale), _ptr(v_tilde), _ptr(cbias),
+                                    _ptr(sel), k, _ptr(Kc8), _ptr(kc_scale), _ptr(Vc), nc,
+                                    _ptr(q_perm), _ptr(q_offsets), nqb, _ptr(k_offsets), nkb,
+                                    H, N, d, _ptr(out), _code(out_dtype), _ptr(err),
+                                    _stream(stream))
+    _check("spark_bsa_attend_fp8", st)
+    return out
+
+
+def spark_bsa_workspace_size_fp8(H, N, d, nqb, nkb, topk_ratio, nc=0) -> int:
+    return int(lib().spark_bsa_workspace_size_fp8(H, N, d, nqb, nkb, float(topk_ratio), int(nc)))
+
+
+def spark_bsa_forward_fp8(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, topk_ratio, Kc=None,
+                          Vc=None, out=None, workspace=None, stream=None):
+    """spark_bsa_forward_ctx with FP8 logits (d = 128); returns (out, workspace, layout)."""
+    _need(Q, "Q", (torch.bfloat16, torch.float32))
+    dev = Q.device
+    H, N, d = Q.shape
+    for n, t in (("K", K), ("V", V)):
+        _need(t, n, Q.dtype, dev)
+    if K.shape != Q.shape or V.shape != Q.shape:
+        raise ValueError("Q, K, V must share the shape [H, N, d]")
+    Kc, Vc, nc = _context_args(Kc, Vc, H, d, Q.dtype, dev)
+    for n, t in (("q_perm", q_perm), ("k_perm", k_perm)):
+        _need(t, n, torch.int32, dev)
+    for n, t in (("q_offsets", q_offsets), ("k_offsets", k_offsets)):
+        _need(t, n, torch.int32, dev)
+    nqb, nkb = q_offsets.numel() - 1, k_offsets.numel() - 1
+    layout = spark_bsa_workspace_layout(H, N, d, nqb, nkb, topk_ratio)
+    size = spark_bsa_workspace_size_fp8(H, N, d, nqb, nkb, topk_ratio, nc)
+    if size == 0:
+        raise SparkError("spark_bsa_workspace_size_fp8", 2)
+    if out is None:
+        out = torch.empty_like(Q)
+    _need(out, "out", Q.dtype, dev)
+    if workspace is None:
+        workspace = torch.empty(size, dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    st = lib().spark_bsa_forward_fp8(_ptr(Q), _ptr(K), _ptr(V), _ptr(Kc), _ptr(Vc), nc,
+                                     _code(Q.dtype), H, N, d, _ptr(q_perm), _ptr(k_perm),
+                                     _ptr(q_offsets), nqb, _ptr(k_offsets), nkb,
+                                     float(topk_ratio), _ptr(out), _ptr(workspace),
+                                     workspace.numel(), _stream(stream))
+    _check("spark_bsa_forward_fp8", st)
+    return out, workspace, layout
 
 
 # ------------------------------------------------------------ Spark-Reblock partitioner

@@ -20,7 +20,8 @@ INCLUDE = os.path.join(os.path.dirname(PKG_DIR), "include")
 BUILD_DIR = os.path.join(PKG_DIR, "_build")
 LIB_NAME = "libspark_bsa.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
-SOURCES = ["api.cu", "gather.cu", "route.cu", "attention.cu", "noalloc.cu", "reblock.cu"]
+SOURCES = ["api.cu", "gather.cu", "route.cu", "attention.cu", "noalloc.cu", "reblock.cu",
+           "quant.cu"]
 HEADERS = ["spark_ptx.cuh", "spark_kernels.cuh"]
 
 NVCC_FLAGS = [

@@ -42,6 +42,22 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int H, int rows, int d) {
   return r == CUDA_SUCCESS;
 }
 
+// 3-D e4m3 (byte) tensor [H][rows][d] with a 128-row x 128-byte box and 128-byte swizzle.
+bool encode_rows_map_u8(CUtensorMap* m, const void* base, int H, int rows, int d) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(H)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d),
+                           static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(d)};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace spark
 
 namespace {
@@ -128,6 +144,59 @@ spark_status attend_impl(const void* Qp, const void* Kp, const void* Vp, const v
                                  H, N, d, out, out_dtype, err, s));
 }
 
+// FP8 logits: e4m3 Qp8/Kp8/kt8/Kc8 with their group scales, bf16 values.
+spark_status attend_fp8_impl(const void* Qp8, const float* q_scale, const void* Kp8,
+                             const float* k_scale, const void* Vp, const void* kt8,
+                             const float* kt_scale, const void* v_tilde, const float* cbias,
+                             const int32_t* sel, int k, const void* Kc8, const float* kc_scale,
+                             const void* Vc, int nc, const int32_t* q_perm,
+                             const int32_t* q_offsets, int nqb, const int32_t* k_offsets,
+                             int nkb, int H, int N, int d, void* out, int out_dtype,
+                             uint32_t* err, cudaStream_t s) {
+  AttendMaps maps;
+  if (!encode_rows_map_u8(&maps.q, Qp8, H, N, d) || !encode_rows_map_u8(&maps.k, Kp8, H, N, d) ||
+      !encode_rows_map(&maps.v, Vp, H, N, d) || !encode_rows_map_u8(&maps.kt, kt8, H, nkb, d) ||
+      !encode_rows_map(&maps.vt, v_tilde, H, nkb, d))
+    return SPARK_ERR_CUDA;
+  if (nc > 0) {
+    if (!encode_rows_map_u8(&maps.kc, Kc8, H, nc, d) || !encode_rows_map(&maps.vc, Vc, H, nc, d))
+      return SPARK_ERR_CUDA;
+  } else {
+    maps.kc = maps.k;                            // never loaded: the kernel has no context tile
+    maps.vc = maps.v;
+  }
+  return from_cuda(launch_attend_fp8(maps, q_scale, k_scale, kt_scale, kc_scale, nc, cbias, sel,
+                                     k, q_perm, q_offsets, nqb, k_offsets, nkb, H, N, out,
+                                     out_dtype, err, s));
+}
+
+// Byte offsets of the FP8 operands and scales of spark_bsa_forward_fp8 (from the start of
+// their region, 256-byte aligned).
+struct Fp8Layout {
+  size_t Qp8, Kp8, kt8, Kc8, q_scale, k_scale, kt_scale, kc_scale, total;
+};
+
+Fp8Layout fp8_layout(int H, int N, int d, int nqb, int nkb, int nc) {
+  Fp8Layout F;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  const size_t h = static_cast<size_t>(H);
+  F.Qp8 = take(h * N * d);
+  F.Kp8 = take(h * N * d);
+  F.kt8 = take(h * nkb * d);
+  F.Kc8 = take(h * nc * d);
+  F.q_scale = take(h * nqb * 4);
+  F.k_scale = take(h * nkb * 4);
+  F.kt_scale = take(h * ((nkb + 127) / 128) * 4);
+  F.kc_scale = take(h * ((nc + 127) / 128) * 4);
+  F.total = off;
+  return F;
+}
+
 spark_status check_context(const void* Kc, const void* Vc, int nc) {
   if (nc < 0 || nc > SPARK_MAX_NC) return SPARK_ERR_INVALID_ARG;
   if (nc > 0 && (!Kc || !Vc || !aligned(Kc, 16) || !aligned(Vc, 16)))
@@ -141,7 +210,8 @@ spark_status forward_impl(const void* Q, const void* K, const void* V, const voi
                           const int32_t* q_perm, const int32_t* k_perm,
                           const int32_t* q_block_offsets, int nqb,
                           const int32_t* k_block_offsets, int nkb, double topk_ratio, void* out,
-                          void* workspace, size_t workspace_bytes, cudaStream_t s) {
+                          void* workspace, size_t workspace_bytes, cudaStream_t s,
+                          bool fp8 = false) {
   if (!Q || !K || !V || !q_perm || !k_perm || !q_block_offsets || !k_block_offsets || !out)
     return SPARK_ERR_INVALID_ARG;
   if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
@@ -152,8 +222,10 @@ spark_status forward_impl(const void* Q, const void* K, const void* V, const voi
   if (st != SPARK_OK) return st;
   if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16))
     return SPARK_ERR_INVALID_ARG;
+  if (fp8 && d != 128) return SPARK_ERR_UNSUPPORTED;
   const size_t cbytes = nc > 0 ? context_bytes(H, nc, d) : 0;
-  if (workspace == nullptr || workspace_bytes < L.total + 2 * cbytes ||
+  const size_t fp8_bytes = fp8 ? fp8_layout(H, N, d, nqb, nkb, nc).total : 0;
+  if (workspace == nullptr || workspace_bytes < L.total + 2 * cbytes + fp8_bytes ||
       !aligned(workspace, kAlign))
     return SPARK_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -192,8 +264,30 @@ spark_status forward_impl(const void* Q, const void* K, const void* V, const voi
     Kca = Kcb;
     Vca = Vcb;
   }
-  return attend_impl(Qp, Kp, Vp, kt, vt, cbias, sel, L.k, Kca, Vca, nc, q_perm, q_block_offsets,
-                     nqb, k_block_offsets, nkb, H, N, d, out, dtype, err, s);
+  if (!fp8)
+    return attend_impl(Qp, Kp, Vp, kt, vt, cbias, sel, L.k, Kca, Vca, nc, q_perm,
+                       q_block_offsets, nqb, k_block_offsets, nkb, H, N, d, out, dtype, err, s);
+  // FP8 logits: quantise the queries per query block, the keys per key block, the summary
+  // and context keys per 128-row tile, then attend
+  const Fp8Layout F = fp8_layout(H, N, d, nqb, nkb, nc);
+  uint8_t* f = ws + L.total + 2 * cbytes;
+  float* q_scale = reinterpret_cast<float*>(f + F.q_scale);
+  float* k_scale = reinterpret_cast<float*>(f + F.k_scale);
+  float* kt_scale = reinterpret_cast<float*>(f + F.kt_scale);
+  float* kc_scale = reinterpret_cast<float*>(f + F.kc_scale);
+  if (launch_quant_fp8(Qp, H, N, d, q_block_offsets, nqb, f + F.Qp8, q_scale, err, s) !=
+          cudaSuccess ||
+      launch_quant_fp8(Kp, H, N, d, k_block_offsets, nkb, f + F.Kp8, k_scale, err, s) !=
+          cudaSuccess ||
+      launch_quant_fp8(kt, H, nkb, d, nullptr, (nkb + 127) / 128, f + F.kt8, kt_scale, err, s) !=
+          cudaSuccess)
+    return SPARK_ERR_CUDA;
+  if (nc > 0 && launch_quant_fp8(Kca, H, nc, d, nullptr, (nc + 127) / 128, f + F.Kc8, kc_scale,
+                                 err, s) != cudaSuccess)
+    return SPARK_ERR_CUDA;
+  return attend_fp8_impl(f + F.Qp8, q_scale, f + F.Kp8, k_scale, Vp, f + F.kt8, kt_scale, vt,
+                         cbias, sel, L.k, f + F.Kc8, kc_scale, Vca, nc, q_perm, q_block_offsets,
+                         nqb, k_block_offsets, nkb, H, N, d, out, dtype, err, s);
 }
 
 }  // namespace
@@ -375,6 +469,68 @@ spark_status spark_bsa_forward(const void* Q, const void* K, const void* V, int 
   return forward_impl(Q, K, V, nullptr, nullptr, 0, dtype, H, N, d, q_perm, k_perm,
                       q_block_offsets, nqb, k_block_offsets, nkb, topk_ratio, out, workspace,
                       workspace_bytes, as_stream(stream));
+}
+
+// ------------------------------------------------------------------------ FP8 logits
+
+spark_status spark_bsa_quantize_fp8(const void* src, int H, int R, int d,
+                                    const int32_t* group_offsets, int ngroups, void* dst,
+                                    float* scales, uint32_t* err, void* stream) {
+  if (!src || !dst || !scales) return SPARK_ERR_INVALID_ARG;
+  if (H < 1 || H > 65535 || R < 1 || ngroups < 1) return SPARK_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SPARK_ERR_UNSUPPORTED;
+  if (group_offsets == nullptr && ngroups != (R + 127) / 128) return SPARK_ERR_INVALID_ARG;
+  if (!aligned(src, 16) || !aligned(dst, 16)) return SPARK_ERR_INVALID_ARG;
+  return from_cuda(launch_quant_fp8(src, H, R, d, group_offsets, ngroups, dst, scales, err,
+                                    as_stream(stream)));
+}
+
+spark_status spark_bsa_attend_fp8(const void* Qp8, const float* q_scale, const void* Kp8,
+                                  const float* k_scale, const void* Vp, const void* kt8,
+                                  const float* kt_scale, const void* v_tilde,
+                                  const float* cbias, const int32_t* sel, int k,
+                                  const void* Kc8, const float* kc_scale, const void* Vc, int nc,
+                                  const int32_t* q_perm, const int32_t* q_block_offsets,
+                                  int nqb, const int32_t* k_block_offsets, int nkb, int H,
+                                  int N, int d, void* out, int out_dtype, uint32_t* err,
+                                  void* stream) {
+  if (!Qp8 || !q_scale || !Kp8 || !k_scale || !Vp || !kt8 || !kt_scale || !v_tilde || !cbias ||
+      !sel || !q_perm || !q_block_offsets || !k_block_offsets || !out)
+    return SPARK_ERR_INVALID_ARG;
+  if (out_dtype != SPARK_BF16 && out_dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  spark_status st = check_sizes(H, N, d, nqb, nkb);
+  if (st != SPARK_OK) return st;
+  if (d != 128) return SPARK_ERR_UNSUPPORTED;
+  st = check_context(Kc8, Vc, nc);
+  if (st != SPARK_OK) return st;
+  if (nc > 0 && !kc_scale) return SPARK_ERR_INVALID_ARG;
+  if (k < 1 || k > nkb) return SPARK_ERR_INVALID_ARG;
+  if (!aligned(Qp8, 16) || !aligned(Kp8, 16) || !aligned(Vp, 16) || !aligned(kt8, 16) ||
+      !aligned(v_tilde, 16) || !aligned(out, 16))
+    return SPARK_ERR_INVALID_ARG;
+  return attend_fp8_impl(Qp8, q_scale, Kp8, k_scale, Vp, kt8, kt_scale, v_tilde, cbias, sel, k,
+                         Kc8, kc_scale, Vc, nc, q_perm, q_block_offsets, nqb, k_block_offsets,
+                         nkb, H, N, d, out, out_dtype, err, as_stream(stream));
+}
+
+size_t spark_bsa_workspace_size_fp8(int H, int N, int d, int nqb, int nkb, double topk_ratio,
+                                    int nc) {
+  if (d != 128) return 0;
+  const size_t base = spark_bsa_workspace_size_ctx(H, N, d, nqb, nkb, topk_ratio, nc);
+  if (base == 0) return 0;
+  return base + fp8_layout(H, N, d, nqb, nkb, nc).total;
+}
+
+spark_status spark_bsa_forward_fp8(const void* Q, const void* K, const void* V, const void* Kc,
+                                   const void* Vc, int nc, int dtype, int H, int N, int d,
+                                   const int32_t* q_perm, const int32_t* k_perm,
+                                   const int32_t* q_block_offsets, int nqb,
+                                   const int32_t* k_block_offsets, int nkb, double topk_ratio,
+                                   void* out, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  return forward_impl(Q, K, V, Kc, Vc, nc, dtype, H, N, d, q_perm, k_perm, q_block_offsets, nqb,
+                      k_block_offsets, nkb, topk_ratio, out, workspace, workspace_bytes,
+                      as_stream(stream), true);
 }
 
 // ------------------------------------------------- host buffers, pipelined by head chunks

@@ -75,13 +75,26 @@ struct TileInfo {
   int nvalid;     // exact tiles: valid rows (rows >= nvalid are masked)
   int src;        // TileSrc
   bool exact;     // video or context rows (no summary offset)
+  float ks;       // FP8 keys: the tile's scale (its key block's, or its 128-row tile's); else 1
+};
+
+// Scales of the FP8 operands (all null for bf16 operands): per query block [H,nqb], per key
+// block [H,nkb], per 128-row tile of the summary rows [H,ceil(nkb/128)] and of the context
+// rows [H,ceil(nc/128)].
+struct Fp8Scales {
+  const float* q;
+  const float* k;
+  const float* kt;
+  const float* kc;
 };
 
 // Tiles 0..k-1: selected video blocks; then nxt context tiles; then the summary tiles.
+template <bool kFp8>
 __device__ __forceinline__ TileInfo tile_info(int t, int k, int nxt, int nc,
                                               const int32_t* sel_row, const int32_t* k_offsets,
-                                              int nkb, int N) {
+                                              int nkb, int N, const Fp8Scales& sc, int h) {
   TileInfo ti;
+  ti.ks = 1.f;
   if (t < k) {
     const int B = min(max(sel_row[t], 0), nkb - 1);
     const int lo = min(max(k_offsets[B], 0), N - 1);
@@ -90,26 +103,30 @@ __device__ __forceinline__ TileInfo tile_info(int t, int k, int nxt, int nc,
     ti.nvalid = min(hi - lo, kMaxBlock);
     ti.src = kSrcVideo;
     ti.exact = true;
+    if (kFp8) ti.ks = sc.k[static_cast<size_t>(h) * nkb + B];
   } else if (t < k + nxt) {
     ti.y = (t - k) * 128;
     ti.nvalid = min(nc - ti.y, 128);
     ti.src = kSrcContext;
     ti.exact = true;
+    if (kFp8) ti.ks = sc.kc[static_cast<size_t>(h) * nxt + (t - k)];
   } else {
     ti.y = (t - k - nxt) * 128;
     ti.nvalid = 128;
     ti.src = kSrcSummary;
     ti.exact = false;
+    if (kFp8) ti.ks = sc.kt[static_cast<size_t>(h) * ((nkb + 127) / 128) + (t - k - nxt)];
   }
   return ti;
 }
 
 // Reads 64 columns of this thread's S row (TMEM) and turns them into logits: exact tiles give
 // raw scores (the scale is applied in the exponent) with columns past the block set to -inf;
-// summary tiles give s*scale_log2 + offset (offset -inf for selected blocks and padding).
+// summary tiles give s*sl + offset (offset -inf for selected blocks and padding), sl being the
+// logit scale in log2 units (times the FP8 scales).
 template <bool kBiasSmem>
 __device__ __forceinline__ void load_logits(uint32_t taddr, int col0, const TileInfo& ti,
-                                            float scale_log2, const float* biasrow,
+                                            float sl, const float* biasrow,
                                             const float* cb, const uint32_t* selmask, int nkb,
                                             float (&x)[64]) {
   uint32_t r[64];
@@ -127,10 +144,10 @@ __device__ __forceinline__ void load_logits(uint32_t taddr, int col0, const Tile
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const float4 b = br[j];
-      x[4 * j] = fmaf(x[4 * j], scale_log2, b.x);
-      x[4 * j + 1] = fmaf(x[4 * j + 1], scale_log2, b.y);
-      x[4 * j + 2] = fmaf(x[4 * j + 2], scale_log2, b.z);
-      x[4 * j + 3] = fmaf(x[4 * j + 3], scale_log2, b.w);
+      x[4 * j] = fmaf(x[4 * j], sl, b.x);
+      x[4 * j + 1] = fmaf(x[4 * j + 1], sl, b.y);
+      x[4 * j + 2] = fmaf(x[4 * j + 2], sl, b.z);
+      x[4 * j + 3] = fmaf(x[4 * j + 3], sl, b.w);
     }
   } else {
 #pragma unroll
@@ -140,7 +157,7 @@ __device__ __forceinline__ void load_logits(uint32_t taddr, int col0, const Tile
       const float c = cb[Bc];                         // unconditional: the loads batch up
       const uint32_t bits = selmask[Bc >> 5];
       const bool live = B < nkb && !((bits >> (Bc & 31)) & 1u);
-      x[j] = live ? fmaf(x[j], scale_log2, c * kLog2e) : -INFINITY;
+      x[j] = live ? fmaf(x[j], sl, c * kLog2e) : -INFINITY;
     }
   }
 }
@@ -179,7 +196,7 @@ __device__ __forceinline__ float exp32_at(const float (&x)[64], int j0, float c,
 
 }  // namespace
 
-template <int D, bool kBiasSmem>
+template <int D, bool kBiasSmem, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kt,
@@ -187,16 +204,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     const __grid_constant__ CUtensorMap map_vc, int nc, const float* __restrict__ cbias,
     const int32_t* __restrict__ sel, int k, const int32_t* __restrict__ q_perm,
     const int32_t* __restrict__ q_offsets, int nqb, const int32_t* __restrict__ k_offsets,
-    int nkb, int N, void* __restrict__ out, int out_dtype, uint32_t* err) {
-  constexpr int TILE_BYTES = 128 * D * 2;        // one Q, K or V tile (bf16)
-  constexpr int NATOM = D / 64;                  // 128-byte swizzle atoms across d
+    int nkb, int N, void* __restrict__ out, int out_dtype, uint32_t* err, const Fp8Scales sc) {
+  static_assert(!kFp8 || D == 128, "FP8 logits: d = 128 (one 128-byte row per key)");
+  constexpr int QK_BYTES = 128 * D * (kFp8 ? 1 : 2);   // one Q or K tile
+  constexpr int V_BYTES = 128 * D * 2;                 // one V tile (bf16)
+  constexpr int QK_ATOMS = kFp8 ? 1 : D / 64;          // 128-byte swizzle atoms across a row
+  constexpr int V_ATOMS = D / 64;
+  constexpr int QK_ATOM_X = kFp8 ? 128 : 64;           // elements per atom row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* qst = smem;
-  uint8_t* kst = qst + TILE_BYTES;
-  uint8_t* vst = kst + kKStages * TILE_BYTES;
-  Barriers* bars = reinterpret_cast<Barriers*>(vst + kVStages * TILE_BYTES);
+  uint8_t* kst = qst + QK_BYTES;
+  uint8_t* vst = kst + kKStages * QK_BYTES;
+  Barriers* bars = reinterpret_cast<Barriers*>(vst + kVStages * V_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* selmask = reinterpret_cast<uint32_t*>(tmem_slot + 4);
@@ -278,6 +299,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       if (lane == 0) {
         const bool is_k = (warp == kWarpK);
         const int stages = is_k ? kKStages : kVStages;
+        const int tile_bytes = is_k ? QK_BYTES : V_BYTES;
+        const int atoms = is_k ? QK_ATOMS : V_ATOMS;
+        const int atom_x = is_k ? QK_ATOM_X : 64;
         uint8_t* ring = is_k ? kst : vst;
         uint64_t* full = is_k ? bars->kfull : bars->vfull;
         uint64_t* empty = is_k ? bars->kempty : bars->vempty;
@@ -290,25 +314,26 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           if (nxt > 0) tma_prefetch_desc(mc);
           if (is_k) {
             tma_prefetch_desc(&map_q);
-            mbar_arrive_expect_tx(&bars->qfull, TILE_BYTES);
+            mbar_arrive_expect_tx(&bars->qfull, QK_BYTES);
             const int qrow = min(max(qlo, 0), N - 1);   // rows past the block are never stored
-            for (int a = 0; a < NATOM; ++a)
-              tma_load_3d(qst + a * 16384, &map_q, &bars->qfull, a * 64, qrow, h);
+            for (int a = 0; a < QK_ATOMS; ++a)
+              tma_load_3d(qst + a * 16384, &map_q, &bars->qfull, a * QK_ATOM_X, qrow, h);
           }
         }
-        TileInfo next = tile_info(0, k, nxt, nc, sel_row, k_offsets, nkb, N);
+        TileInfo next = tile_info<false>(0, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
         for (int t = 0; t < T; ++t) {
           const int tg = tg0 + t;
           const int s = tg % stages;
           const TileInfo ti = next;
           if (tg >= stages && !mbar_wait(&empty[s], ((tg / stages) - 1) & 1, abort_flag, err))
             break;
-          mbar_arrive_expect_tx(&full[s], TILE_BYTES);
+          mbar_arrive_expect_tx(&full[s], tile_bytes);
           const CUtensorMap* map = ti.src == kSrcVideo ? mx : (ti.src == kSrcContext ? mc : ms);
-          for (int a = 0; a < NATOM; ++a)
-            tma_load_3d(ring + s * TILE_BYTES + a * 16384, map, &full[s], a * 64, ti.y, h);
+          for (int a = 0; a < atoms; ++a)
+            tma_load_3d(ring + s * tile_bytes + a * 16384, map, &full[s], a * atom_x, ti.y, h);
           issued = tg + 1;
-          if (t + 1 < T) next = tile_info(t + 1, k, nxt, nc, sel_row, k_offsets, nkb, N);
+          if (t + 1 < T)
+            next = tile_info<false>(t + 1, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
         }
         if (*abort_flag) {
           // drain: wait for every load still in flight (the last round of each stage)
@@ -320,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     } else if (warp == kWarpMma) {
       // ---------------------------------------------------------------- MMA issuer
       if (lane == 0) {
-        constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
+        constexpr uint32_t idS = kFp8 ? idesc_e4m3(128, 128) : idesc_bf16(128, 128, false, false);
         constexpr uint32_t idO = idesc_bf16(128, D, false, true);
         // descriptors built once; per MMA only a compile-time offset (16-byte units) changes
         const uint64_t qd = sdesc_sw128(smem_u32(qst), 16, 1024);
@@ -333,11 +358,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           const int s = tg % kKStages;
           if (!mbar_wait(&bars->kfull[s], (tg / kKStages) & 1, abort_flag, err)) return false;
           const uint32_t dcol = tbase + (tg % 3) * 128;
-          const uint64_t kd = kdesc0 + static_cast<uint64_t>(s * (TILE_BYTES >> 4));
+          const uint64_t kd = kdesc0 + static_cast<uint64_t>(s * (QK_BYTES >> 4));
+          if constexpr (kFp8) {
+            // 32 e4m3 values of d = 32 bytes per MMA, all inside the one 128-byte atom row
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) / 16;
-            mma_ss(dcol, qd + off, kd + off, idS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 32; ++kk)
+              mma_ss_f8(dcol, qd + kk * 2, kd + kk * 2, idS, kk > 0 ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) / 16;
+              mma_ss(dcol, qd + off, kd + off, idS, kk > 0 ? 1u : 0u);
+            }
           }
           tc_commit(&bars->sfull[tg % 3]);
           tc_commit(&bars->kempty[s]);
@@ -350,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           tc_fence_after_sync();
           const int s = tg % kVStages;
           if (!mbar_wait(&bars->vfull[s], (tg / kVStages) & 1, abort_flag, err)) break;
-          const uint64_t vd = vdesc0 + static_cast<uint64_t>(s * (TILE_BYTES >> 4));
+          const uint64_t vd = vdesc0 + static_cast<uint64_t>(s * (V_BYTES >> 4));
           const uint32_t pcol = tbase + (tg % 3) * 128;               // P(t) over S(t)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
@@ -370,7 +402,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       const int q4 = warp & 3, grp = warp >> 2;          // row quarter, tile group
       const int row = q4 * 32 + lane;                    // 0..127 == TMEM lane
       const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-      const float scale_log2 = kLog2e * rsqrtf(static_cast<float>(D));
+      // logit scale in log2 units; FP8 queries carry their block's scale
+      const float scale_log2 = kLog2e * rsqrtf(static_cast<float>(D)) *
+                               (kFp8 ? sc.q[static_cast<size_t>(h) * nqb + A] : 1.f);
       float l_run = 0.f;
       bool ok = true;
       float x[64];
@@ -380,17 +414,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         float mt = -INFINITY;
         if (grp < T) {
           const int tg = tg0 + grp;
-          const TileInfo ti = tile_info(grp, k, nxt, nc, sel_row, k_offsets, nkb, N);
+          const TileInfo ti = tile_info<kFp8>(grp, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
+          const float tsl = scale_log2 * ti.ks;
           ok = __all_sync(0xffffffffu,
                           mbar_wait(&bars->sfull[tg % 3], (tg / 3) & 1, abort_flag, err));
           if (ok) {
             tc_fence_after_sync();
             const uint32_t sbuf = tbase + lane_off + (tg % 3) * 128;
-            load_logits<kBiasSmem>(sbuf, 0, ti, scale_log2, biasrow, cb, selmask, nkb, x);
+            load_logits<kBiasSmem>(sbuf, 0, ti, tsl, biasrow, cb, selmask, nkb, x);
             mt = max64(x);
-            load_logits<kBiasSmem>(sbuf + 64, 64, ti, scale_log2, biasrow, cb, selmask, nkb, x);
+            load_logits<kBiasSmem>(sbuf + 64, 64, ti, tsl, biasrow, cb, selmask, nkb, x);
             mt = fmaxf(mt, max64(x));
-            if (ti.exact) mt *= scale_log2;
+            if (ti.exact) mt *= tsl;
           }
         }
         ex_m[grp][row] = mt;
@@ -400,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         m_ref = m_true;                                  // both groups' maximum (epilogue)
       }
       if (!(m_ref > -INFINITY)) m_ref = 0.f;
-      TileInfo next = tile_info(grp, k, nxt, nc, sel_row, k_offsets, nkb, N);
+      TileInfo next = tile_info<kFp8>(grp, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
       for (int t = grp; ok && t < T; t += 2) {
         const TileInfo ti = next;
         const int tg = tg0 + t;
@@ -410,9 +445,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           if (!ok) break;
           tc_fence_after_sync();
         }
-        if (t + 2 < T) next = tile_info(t + 2, k, nxt, nc, sel_row, k_offsets, nkb, N);
+        if (t + 2 < T)
+          next = tile_info<kFp8>(t + 2, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
         const uint32_t sbuf = tbase + lane_off + b * 128;
-        const float c = ti.exact ? scale_log2 : 1.f;
+        const float tsl = scale_log2 * ti.ks;
+        const float c = ti.exact ? tsl : 1.f;
         // The row maximum is only needed for a repeat, and only to within a few units: a
         // chunk whose sum stays in [2^-40, 2^40] has its maximum within 40 of the reference
         // and cannot drive the row sum out of [2^-60, 2^60] (fewer than 2^16 chunks per row),
@@ -420,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         float rowsum = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          load_logits<kBiasSmem>(sbuf + half * 64, half * 64, ti, scale_log2, biasrow, cb,
+          load_logits<kBiasSmem>(sbuf + half * 64, half * 64, ti, tsl, biasrow, cb,
                                  selmask, nkb, x);
           uint32_t p16[16];
           float cs = exp32_at(x, 0, c, m_ref, p16);
@@ -429,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           tmem_st16(sbuf + half * 32 + 16, p16);
           if (!(cs >= 0x1p-40f && cs <= 0x1p40f)) {
             const float mt = max64(x);
-            m_true = fmaxf(m_true, ti.exact ? mt * scale_log2 : mt);
+            m_true = fmaxf(m_true, ti.exact ? mt * tsl : mt);
           }
           rowsum += cs;
         }
@@ -509,29 +546,31 @@ static bool bias_in_smem(int nkb, int k) {
   return nct > 0 && nct * 128 <= kMaxSmemBias;
 }
 
-static size_t attend_smem_bytes(int d, int nkb, int k) {
-  const size_t tile = static_cast<size_t>(128) * d * 2;
+static size_t attend_smem_bytes(int d, int nkb, int k, bool fp8) {
+  const size_t qk = static_cast<size_t>(128) * d * (fp8 ? 1 : 2);
+  const size_t v = static_cast<size_t>(128) * d * 2;
   const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
   const size_t words = (nkb + 31) / 32 + 4;          // + 16 bytes of alignment slack
   const size_t bias = bias_in_smem(nkb, k) ? static_cast<size_t>(nct) * 128 * 4 : 0;
-  return 1024 + (1 + kKStages + kVStages) * tile + sizeof(Barriers) + 16 + words * 4 + bias;
+  return 1024 + (1 + kKStages) * qk + kVStages * v + sizeof(Barriers) + 16 + words * 4 + bias;
 }
 
-template <int D, bool kBiasSmem>
+template <int D, bool kBiasSmem, bool kFp8>
 static cudaError_t launch_attend_t(const AttendMaps& m, int nc, const float* cbias,
                                    const int32_t* sel, int k, const int32_t* q_perm,
                                    const int32_t* q_offsets,
                                    int nqb, const int32_t* k_offsets, int nkb, int H, int N,
-                                   void* out, int out_dtype, uint32_t* err, cudaStream_t s) {
-  const size_t smem = attend_smem_bytes(D, nkb, k);
-  cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, kBiasSmem>,
+                                   void* out, int out_dtype, uint32_t* err, const Fp8Scales& sc,
+                                   cudaStream_t s) {
+  const size_t smem = attend_smem_bytes(D, nkb, k, kFp8);
+  cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, kBiasSmem, kFp8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(nqb, H);
-  attend_kernel<D, kBiasSmem><<<grid, kThreads, smem, s>>>(
+  attend_kernel<D, kBiasSmem, kFp8><<<grid, kThreads, smem, s>>>(
       m.q, m.k, m.v, m.kt, m.vt, m.kc, m.vc, nc, cbias, sel, k, q_perm, q_offsets, nqb,
-      k_offsets, nkb, N, out, out_dtype, err);
+      k_offsets, nkb, N, out, out_dtype, err, sc);
   return cudaGetLastError();
 }
 
@@ -541,15 +580,36 @@ cudaError_t launch_attend(const AttendMaps& maps, int nc, const float* cbias,
                           int H, int N, int d, void* out, int out_dtype, uint32_t* err,
                           cudaStream_t s) {
   const bool bs = bias_in_smem(nkb, k);
+  const Fp8Scales none{nullptr, nullptr, nullptr, nullptr};
   if (d == 128)
-    return bs ? launch_attend_t<128, true>(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb,
-                                           k_offsets, nkb, H, N, out, out_dtype, err, s)
-              : launch_attend_t<128, false>(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb,
-                                            k_offsets, nkb, H, N, out, out_dtype, err, s);
-  return bs ? launch_attend_t<64, true>(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb,
-                                        k_offsets, nkb, H, N, out, out_dtype, err, s)
-            : launch_attend_t<64, false>(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb,
-                                         k_offsets, nkb, H, N, out, out_dtype, err, s);
+    return bs ? launch_attend_t<128, true, false>(maps, nc, cbias, sel, k, q_perm, q_offsets,
+                                                  nqb, k_offsets, nkb, H, N, out, out_dtype,
+                                                  err, none, s)
+              : launch_attend_t<128, false, false>(maps, nc, cbias, sel, k, q_perm, q_offsets,
+                                                   nqb, k_offsets, nkb, H, N, out, out_dtype,
+                                                   err, none, s);
+  return bs ? launch_attend_t<64, true, false>(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb,
+                                               k_offsets, nkb, H, N, out, out_dtype, err, none,
+                                               s)
+            : launch_attend_t<64, false, false>(maps, nc, cbias, sel, k, q_perm, q_offsets,
+                                                nqb, k_offsets, nkb, H, N, out, out_dtype, err,
+                                                none, s);
+}
+
+cudaError_t launch_attend_fp8(const AttendMaps& maps, const float* q_scale,
+                              const float* k_scale, const float* kt_scale,
+                              const float* kc_scale, int nc, const float* cbias,
+                              const int32_t* sel, int k, const int32_t* q_perm,
+                              const int32_t* q_offsets, int nqb, const int32_t* k_offsets,
+                              int nkb, int H, int N, void* out, int out_dtype, uint32_t* err,
+                              cudaStream_t s) {
+  const Fp8Scales sc{q_scale, k_scale, kt_scale, kc_scale};
+  return bias_in_smem(nkb, k)
+             ? launch_attend_t<128, true, true>(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb,
+                                                k_offsets, nkb, H, N, out, out_dtype, err, sc, s)
+             : launch_attend_t<128, false, true>(maps, nc, cbias, sel, k, q_perm, q_offsets,
+                                                 nqb, k_offsets, nkb, H, N, out, out_dtype, err,
+                                                 sc, s);
 }
 
 }  // namespace spark

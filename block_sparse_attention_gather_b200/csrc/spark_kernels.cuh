@@ -43,6 +43,24 @@ cudaError_t launch_attend(const AttendMaps& maps, int nc, const float* cbias,
 
 // 3-D bf16 tensor map [H][rows][d], box 64 columns x 128 rows, 128-byte swizzle (api.cu).
 bool encode_rows_map(CUtensorMap* m, const void* base, int H, int rows, int d);
+// 3-D e4m3 (byte) tensor map [H][rows][d], box 128 bytes x 128 rows, 128-byte swizzle.
+bool encode_rows_map_u8(CUtensorMap* m, const void* base, int H, int rows, int d);
+
+// FP8 logits: the attention with e4m3 Q, K, k~, Kc operands (maps from encode_rows_map_u8)
+// and their group scales, bf16 V, v~, Vc (d = 128).
+cudaError_t launch_attend_fp8(const AttendMaps& maps, const float* q_scale,
+                              const float* k_scale, const float* kt_scale,
+                              const float* kc_scale, int nc, const float* cbias,
+                              const int32_t* sel, int k, const int32_t* q_perm,
+                              const int32_t* q_offsets, int nqb, const int32_t* k_offsets,
+                              int nkb, int H, int N, void* out, int out_dtype, uint32_t* err,
+                              cudaStream_t s);
+
+// e4m3 codes of bf16 rows [H,R,d], one power-of-two scale per group: the blocks of `offsets`
+// ([ngroups+1], shared by all heads), or 128-row tiles when offsets is null (quant.cu).
+cudaError_t launch_quant_fp8(const void* src, int H, int R, int d, const int32_t* offsets,
+                             int ngroups, void* dst, float* scales, uint32_t* err,
+                             cudaStream_t s);
 
 // ---- Spark-Reblock partitioner (reblock.cu)
 // Byte offsets of its workspace regions (256-byte aligned).

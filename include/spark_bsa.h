@@ -225,6 +225,66 @@ SPARK_API spark_status spark_bsa_attend_ctx(const void* Qp, const void* Kp, cons
                                             int N, int d, void* out, int out_dtype,
                                             uint32_t* err, void* stream);
 
+/* ---- FP8 logits ----
+ * Spark-H3 blog, section "Benchmark Results": Spark-H3's attention is also timed in FP8; the
+ * scheme is not given.  Readings taken here:
+ *   - only the logit product is FP8: the queries Qp, the exact keys Kp, the summary keys k~
+ *     and the context keys enter it as e4m3 (OCP E4M3FN: largest finite 448, round to
+ *     nearest even, saturating); routing, anchor, summaries, values and probabilities are
+ *     those of the bf16 path;
+ *   - one power-of-two scale 2^e per group of rows: each query block, each key block, each
+ *     128-row tile of the summary rows and of the context rows, e the smallest integer with
+ *     max|x| <= 448 * 2^e (at least -126; 0 for an all-zero group); the code of x is
+ *     e4m3(x * 2^-e), which is exact before the rounding;
+ *   - the logit of query i (block A) and key j (group G) is sigma * sA * sG * (qcode . kcode),
+ *     plus c_B for a summary row.
+ * d must be 128 (one 128-byte row of codes per token). */
+
+/* Codes of bf16 rows src [H,R,d] (device, 16-byte aligned) into dst [H,R,d] (one byte per
+ * value) and scales [H,ngroups] (fp32, 2^e).  Groups are the blocks of `group_offsets`
+ * ([ngroups+1] device int32, shared by all heads, non-decreasing within 0..R), or, when it is
+ * NULL, the 128-row tiles (ngroups must then be ceil(R/128)).  Bad offsets set
+ * SPARK_DEVERR_OFFSETS and leave that group unwritten (scale 1). */
+SPARK_API spark_status spark_bsa_quantize_fp8(const void* src, int H, int R, int d,
+                                              const int32_t* group_offsets, int ngroups,
+                                              void* dst, float* scales, uint32_t* err,
+                                              void* stream);
+
+/* Step 5 with FP8 logits: as spark_bsa_attend_ctx, with Qp8 [H,N,d] / q_scale [H,nqb] (per
+ * query block), Kp8 [H,N,d] / k_scale [H,nkb] (per key block), kt8 [H,nkb,d] / kt_scale
+ * [H,ceil(nkb/128)] and Kc8 [H,nc,d] / kc_scale [H,ceil(nc/128)] (per 128-row tile; Kc8,
+ * kc_scale and Vc may be NULL when nc == 0), as written by spark_bsa_quantize_fp8; Vp,
+ * v_tilde and Vc stay bf16.  d must be 128 (SPARK_ERR_UNSUPPORTED otherwise). */
+SPARK_API spark_status spark_bsa_attend_fp8(const void* Qp8, const float* q_scale,
+                                            const void* Kp8, const float* k_scale,
+                                            const void* Vp, const void* kt8,
+                                            const float* kt_scale, const void* v_tilde,
+                                            const float* cbias, const int32_t* sel, int k,
+                                            const void* Kc8, const float* kc_scale,
+                                            const void* Vc, int nc, const int32_t* q_perm,
+                                            const int32_t* q_block_offsets, int nqb,
+                                            const int32_t* k_block_offsets, int nkb, int H,
+                                            int N, int d, void* out, int out_dtype,
+                                            uint32_t* err, void* stream);
+
+/* Workspace bytes of spark_bsa_forward_fp8: spark_bsa_workspace_size_ctx plus the codes and
+ * scales; 0 when d != 128 or the sizes are invalid. */
+SPARK_API size_t spark_bsa_workspace_size_fp8(int H, int N, int d, int nqb, int nkb,
+                                              double topk_ratio, int nc);
+
+/* The forward pass of spark_bsa_forward_ctx (nc may be 0, Kc/Vc then NULL) with FP8 logits:
+ * after the routing, Qp, Kp, k~ and the context keys are quantised in the workspace and the
+ * attention runs on the codes.  The bf16 layout (spark_bsa_workspace_layout) stays at the
+ * start of the workspace. */
+SPARK_API spark_status spark_bsa_forward_fp8(const void* Q, const void* K, const void* V,
+                                             const void* Kc, const void* Vc, int nc, int dtype,
+                                             int H, int N, int d, const int32_t* q_perm,
+                                             const int32_t* k_perm,
+                                             const int32_t* q_block_offsets, int nqb,
+                                             const int32_t* k_block_offsets, int nkb,
+                                             double topk_ratio, void* out, void* workspace,
+                                             size_t workspace_bytes, void* stream);
+
 /* ---- Host buffers, pipelined by head chunks ----
  * No counterpart in the pages: the forward pass for inputs and output in host memory.  The
  * heads are processed in chunks of `heads_per_chunk`; the copies of chunk c+1 in and of

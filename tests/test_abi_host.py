@@ -124,6 +124,28 @@ def test_step_entry_points_reject_bad_arguments(L):
     assert L.spark_bsa_read_error(None, None, ctypes.byref(flags)) == INVALID
 
 
+def test_fp8_entry_points_reject_bad_arguments(L):
+    p = ctypes.c_void_p(0x100000)
+    # quantise: null operands, d not 64/128, tiles with the wrong group count
+    assert L.spark_bsa_quantize_fp8(None, 1, 10, 128, None, 1, p, p, None, None) == INVALID
+    assert L.spark_bsa_quantize_fp8(p, 1, 10, 96, None, 1, p, p, None, None) == UNSUPPORTED
+    assert L.spark_bsa_quantize_fp8(p, 1, 300, 128, None, 2, p, p, None, None) == INVALID
+    # FP8 attention: d must be 128; k in [1, nkb]; out dtype
+    args = [p] * 10 + [1, p, p, p, 0, p, p, 1, p, 1, 1, 10, 128, p, 0, None, None]
+    bad_d = list(args)
+    bad_d[22] = 64
+    assert L.spark_bsa_attend_fp8(*bad_d) == UNSUPPORTED
+    bad_k = list(args)
+    bad_k[10] = 2
+    assert L.spark_bsa_attend_fp8(*bad_k) == INVALID
+    bad_out = list(args)
+    bad_out[24] = 3
+    assert L.spark_bsa_attend_fp8(*bad_out) == INVALID
+    assert L.spark_bsa_workspace_size_fp8(1, 1024, 64, 16, 16, 0.125, 0) == 0
+    assert L.spark_bsa_workspace_size_fp8(1, 1024, 128, 16, 16, 0.125, 0) > \
+        L.spark_bsa_workspace_size_ctx(1, 1024, 128, 16, 16, 0.125, 0)
+
+
 def test_context_entry_points_reject_bad_arguments(L):
     from block_sparse_attention_gather_b200 import (spark_bsa_workspace_layout,
                                                     spark_bsa_workspace_size_ctx)
