@@ -41,6 +41,7 @@ DEFAULT_WORKLOAD = "768p-24x241920-d128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attention_768p_dram.json")
 KERNELS = ["gather_q", "anchor", "gather_kv_summary", "route", "attend"]
+KERNELS_FP8 = ["gather_q", "anchor", "gather_kv_summary", "route", "quantize", "attend"]
 
 
 def parse_args():
@@ -52,6 +53,9 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--precision", choices=["bf16", "fp8"], default="bf16",
+                    help="fp8: e4m3 logit product (queries, keys, summary and context keys "
+                         "quantised per group after the routing), bf16 values")
     ap.add_argument("--op", choices=["attention", "reblock"], default="attention",
                     help="attention: the two-branch forward (default); reblock: the "
                          "Spark-Reblock partitioner on the same workload's Q and K")
@@ -125,7 +129,7 @@ class HotPath:
     """Preallocated buffers and the five step entry points of the C ABI, called with raw
     device pointers on one stream."""
 
-    def __init__(self, x, ratio, device):
+    def __init__(self, x, ratio, device, fp8=False):
         from block_sparse_attention_gather_b200 import (lib, spark_bsa_workspace_layout,
                                                         workspace_views)
         self.L = lib()
@@ -151,13 +155,28 @@ class HotPath:
         self.out = torch.empty_like(Q)
         self.dtype_code = 0 if Q.dtype == torch.bfloat16 else 1
         self.stream = torch.cuda.current_stream(device)
+        # FP8 logits: codes and group scales of Qp, Kp, k~ (and the context keys)
+        self.fp8 = fp8
+        if fp8:
+            H, N, d, nqb, nkb = self.H, self.N, self.d, self.nqb, self.nkb
+            u8, f32 = torch.uint8, torch.float32
+            self.Qp8 = torch.empty(H, N, d, dtype=u8, device=device)
+            self.Kp8 = torch.empty(H, N, d, dtype=u8, device=device)
+            self.kt8 = torch.empty(H, nkb, d, dtype=u8, device=device)
+            self.q_scale = torch.empty(H, nqb, dtype=f32, device=device)
+            self.k_scale = torch.empty(H, nkb, dtype=f32, device=device)
+            self.kt_scale = torch.empty(H, (nkb + 127) // 128, dtype=f32, device=device)
+            if self.nc:
+                self.Kc8 = torch.empty(H, self.nc, d, dtype=u8, device=device)
+                self.kc_scale = torch.empty(H, (self.nc + 127) // 128, dtype=f32, device=device)
+        self.kernels = KERNELS_FP8 if fp8 else KERNELS
 
     def _p(self, t):
         return ctypes.c_void_p(t.data_ptr())
 
     def step(self, events=None):
-        """One pass of the whole path; if `events` (6 CUDA events) is given, records one
-        before each kernel and one after the last."""
+        """One pass of the whole path; if `events` (one per kernel group of self.kernels, plus
+        one) is given, records one before each group and one after the last."""
         L, x, v, p = self.L, self.x, self.v, self._p
         s = ctypes.c_void_p(self.stream.cuda_stream)
         H, N, d, nqb, nkb, k = self.H, self.N, self.d, self.nqb, self.nkb, self.k
@@ -179,23 +198,46 @@ class HotPath:
         st |= L.spark_bsa_route(p(v["qbar_blocks"]), p(v["kbar"]), H, nqb, nkb, d, k,
                                 p(v["sel"]), err, s)
         rec(4)
-        if self.nc == 0:
+        Kc, Vc = x.get("Kc"), x.get("Vc")
+        if self.convert_ctx:
+            st |= L.spark_bsa_context_bf16(p(Kc), p(Vc), self.dtype_code, H, self.nc, d,
+                                           p(self.Kcb), p(self.Vcb), s)
+            Kc, Vc = self.Kcb, self.Vcb
+        if self.fp8:
+            st |= L.spark_bsa_quantize_fp8(p(v["Qp"]), H, N, d, p(x["q_offsets"]), nqb,
+                                           p(self.Qp8), p(self.q_scale), err, s)
+            st |= L.spark_bsa_quantize_fp8(p(v["Kp"]), H, N, d, p(x["k_offsets"]), nkb,
+                                           p(self.Kp8), p(self.k_scale), err, s)
+            st |= L.spark_bsa_quantize_fp8(p(v["k_tilde"]), H, nkb, d, None, (nkb + 127) // 128,
+                                           p(self.kt8), p(self.kt_scale), err, s)
+            if self.nc:
+                st |= L.spark_bsa_quantize_fp8(p(Kc), H, self.nc, d, None,
+                                               (self.nc + 127) // 128, p(self.Kc8),
+                                               p(self.kc_scale), err, s)
+            rec(5)
+            nc = self.nc
+            st |= L.spark_bsa_attend_fp8(p(self.Qp8), p(self.q_scale), p(self.Kp8),
+                                         p(self.k_scale), p(v["Vp"]), p(self.kt8),
+                                         p(self.kt_scale), p(v["v_tilde"]), p(v["cbias"]),
+                                         p(v["sel"]), k, p(self.Kc8) if nc else None,
+                                         p(self.kc_scale) if nc else None,
+                                         p(Vc) if nc else None, nc, p(x["q_perm"]),
+                                         p(x["q_offsets"]), nqb, p(x["k_offsets"]), nkb, H, N,
+                                         d, p(self.out), self.dtype_code, err, s)
+            rec(6)
+        elif self.nc == 0:
             st |= L.spark_bsa_attend(p(v["Qp"]), p(v["Kp"]), p(v["Vp"]), p(v["k_tilde"]),
                                      p(v["v_tilde"]), p(v["cbias"]), p(v["sel"]), k,
                                      p(x["q_perm"]), p(x["q_offsets"]), nqb, p(x["k_offsets"]),
                                      nkb, H, N, d, p(self.out), self.dtype_code, err, s)
+            rec(5)
         else:
-            Kc, Vc = x["Kc"], x["Vc"]
-            if self.convert_ctx:
-                st |= L.spark_bsa_context_bf16(p(Kc), p(Vc), self.dtype_code, H, self.nc, d,
-                                               p(self.Kcb), p(self.Vcb), s)
-                Kc, Vc = self.Kcb, self.Vcb
             st |= L.spark_bsa_attend_ctx(p(v["Qp"]), p(v["Kp"]), p(v["Vp"]), p(v["k_tilde"]),
                                          p(v["v_tilde"]), p(v["cbias"]), p(v["sel"]), k, p(Kc),
                                          p(Vc), self.nc, p(x["q_perm"]), p(x["q_offsets"]),
                                          nqb, p(x["k_offsets"]), nkb, H, N, d, p(self.out),
                                          self.dtype_code, err, s)
-        rec(5)
+            rec(5)
         if st != 0:
             raise RuntimeError(f"a step entry point failed (status bits {st})")
 
@@ -222,6 +264,8 @@ def kernel_bytes(hp):
         "anchor": H * nqb * d * 4 + H * d * 4,
         "gather_kv_summary": 2 * H * N * d * (e + 2) + H * N * 4 + H * nkb * d * (4 + 2 + 2) + H * nkb * 4,
         "route": H * (nqb + nkb) * d * 4 + H * nqb * k * 4,
+        # bf16 rows read once, one code byte written per value (Qp, Kp, k~, context keys)
+        "quantize": (2 * H * N * d + H * nkb * d + H * hp.nc * d) * 3,
     }
 
 
@@ -512,7 +556,9 @@ def main():
     torch.cuda.set_device(device)
     w = WORKLOADS[args.workload]
     x = make_inputs(w, device=device)
-    hp = HotPath(x, w.ratio, device)
+    hp = HotPath(x, w.ratio, device, fp8=args.precision == "fp8")
+    if hp.fp8 and hp.d != 128:
+        raise SystemExit("--precision fp8 needs d = 128")
     peaks, peak_kind = load_peaks()
 
     def barrier():
@@ -527,7 +573,9 @@ def main():
     if flags:
         raise RuntimeError(f"device error word {flags:#x} after warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    names = hp.kernels
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+           for _ in range(args.steps)]
     clocks = ClockSampler(device)
     barrier()
     torch.cuda.synchronize()
@@ -537,12 +585,12 @@ def main():
     barrier()
     clock_info = clocks.stop()
 
-    per_kernel = {n: [] for n in KERNELS}
+    per_kernel = {n: [] for n in names}
     totals = []
     for e in evs:
-        for j, n in enumerate(KERNELS):
+        for j, n in enumerate(names):
             per_kernel[n].append(e[j].elapsed_time(e[j + 1]))
-        totals.append(e[0].elapsed_time(e[5]))
+        totals.append(e[0].elapsed_time(e[len(names)]))
     total_ms = max_over_ranks(sum(totals), world, device)
     ms_per_step = total_ms / args.steps
     dflops = dense_flops(w)
@@ -555,10 +603,17 @@ def main():
     att_ms = statistics.mean(per_kernel["attend"])
     achieved = att_flops / (att_ms / 1e3) / 1e12
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_note = f"bf16 sustained, {peak_kind}"
+    if hp.fp8:
+        # half of the FLOPs (Q K^T) run at the fp8 rate, twice bf16's (nominal 4.5 / 2.25
+        # PFLOP/s), half (P V) at bf16's: the mix's peak is 4/3 of bf16's
+        peak = peak * 4.0 / 3.0
+        peak_note = (f"bf16 sustained ({peak_kind}) x 4/3: Q K^T at fp8 = 2x bf16 (nominal "
+                     "ratio), P V at bf16")
     kb = kernel_bytes(hp)
     hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     kernels = {}
-    for n in KERNELS:
+    for n in names:
         ms = statistics.mean(per_kernel[n])
         entry = {"ms": ms, "share": ms / ms_per_step}
         if n in kb:
@@ -572,21 +627,28 @@ def main():
     e2e = None
     if args.e2e_steps > 0:
         from block_sparse_attention_gather_b200 import (spark_bsa_forward, spark_bsa_forward_ctx,
+                                                        spark_bsa_forward_fp8,
                                                         spark_bsa_forward_host,
                                                         spark_bsa_host_staging_size,
-                                                        spark_bsa_workspace_size)
+                                                        spark_bsa_workspace_size,
+                                                        spark_bsa_workspace_size_fp8)
         names = ["Q", "K", "V", "q_perm", "k_perm", "q_offsets", "k_offsets"]
         if hp.nc:
             names += ["Kc", "Vc"]
         host = {n: x[n].to("cpu").pin_memory() for n in names}
-        dev_in = {n: torch.empty_like(x[n]) for n in host} if hp.nc else {}
+        piped = not hp.nc and not hp.fp8
+        dev_in = {n: torch.empty_like(x[n]) for n in host} if not piped else {}
+        if hp.fp8:
+            ws8 = torch.empty(spark_bsa_workspace_size_fp8(hp.H, hp.N, hp.d, hp.nqb, hp.nkb,
+                                                           w.ratio, hp.nc),
+                              dtype=torch.uint8, device=device)
         out_host = torch.empty(hp.out.shape, dtype=hp.out.dtype).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = out_host.numel() * out_host.element_size()
         s = torch.cuda.current_stream(device)
         # without context tokens: the host-buffer entry point, pipelined head by head
         hpc = 1
-        if not hp.nc:
+        if piped:
             staging = torch.empty(spark_bsa_host_staging_size(hp.H, hp.N, hp.d, hp.out.dtype,
                                                               hp.nqb, hp.nkb, hpc),
                                   dtype=torch.uint8, device=device)
@@ -596,7 +658,7 @@ def main():
             pipe = (s, torch.cuda.Stream(device), torch.cuda.Stream(device))
 
         def e2e_step():
-            if not hp.nc:
+            if piped:
                 spark_bsa_forward_host(host["Q"], host["K"], host["V"], host["q_perm"],
                                        host["k_perm"], host["q_offsets"], host["k_offsets"],
                                        w.ratio, out=out_host, heads_per_chunk=hpc,
@@ -604,7 +666,13 @@ def main():
                 return
             for n in host:
                 dev_in[n].copy_(host[n], non_blocking=True)
-            if hp.nc:
+            if hp.fp8:
+                o, _, _ = spark_bsa_forward_fp8(dev_in["Q"], dev_in["K"], dev_in["V"],
+                                                dev_in["q_perm"], dev_in["k_perm"],
+                                                dev_in["q_offsets"], dev_in["k_offsets"], w.ratio,
+                                                Kc=dev_in.get("Kc"), Vc=dev_in.get("Vc"),
+                                                out=hp.out, workspace=ws8)
+            elif hp.nc:
                 o, _, _ = spark_bsa_forward_ctx(dev_in["Q"], dev_in["K"], dev_in["V"],
                                                 dev_in["Kc"], dev_in["Vc"], dev_in["q_perm"],
                                                 dev_in["k_perm"], dev_in["q_offsets"],
@@ -632,16 +700,20 @@ def main():
         e2e = {"value": whole_job_rate(world, dflops, args.e2e_steps, e_ms), "unit": UNIT,
                "ms_per_call": e_ms / args.e2e_steps, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-               "call": ("spark_bsa_forward_ctx after host-to-device copies" if hp.nc else
+               "call": ("spark_bsa_forward_fp8 after host-to-device copies" if hp.fp8 else
+                        "spark_bsa_forward_ctx after host-to-device copies" if hp.nc else
                         f"spark_bsa_forward_host (host buffers, chunks of {hpc} heads, copies "
                         "overlapped with computation on three streams)")}
         del host, dev_in, out_host
+        if hp.fp8:
+            del ws8
 
     traffic = profiled_traffic(hp)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3 logits, bf16 values" if hp.fp8 else "bf16", "data": "synthetic",
         "config": {"workload": w.name, "H": w.H, "N": w.N, "d": w.d, "topk_ratio": w.ratio,
                    "k": hp.k, "nqb": hp.nqb, "nkb": hp.nkb, "context_tokens": hp.nc,
                    "block": w.block,
@@ -650,11 +722,12 @@ def main():
         "actual_tflops": att_flops / (ms_per_step / 1e3) / 1e12 * world,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "peak_kind": f"bf16 sustained, {peak_kind}",
+                     "peak_kind": peak_note,
                      "kernel": "attend (tcgen05 two-branch attention)",
                      "algorithmic_flops_per_launch": att_flops},
         "kernels": kernels,
-        "gpu_launches": (5 + (2 if hp.convert_ctx else 0)) * args.steps,
+        "gpu_launches": (5 + (2 if hp.convert_ctx else 0) +
+                         ((4 if hp.nc else 3) if hp.fp8 else 0)) * args.steps,
         "clocks": clock_info,
         "e2e": e2e,
     }
