@@ -19,7 +19,8 @@
 //              makes its CTA repeat all tiles with that row's true maximum as the reference
 //              (a second pass over the same pipeline; each chunk whose sum is out of range
 //              records its maximum, which is within a few units of the row's).
-//   warp 8     TMA producer: the Q tile once, then K tiles (3-stage ring).
+//   warp 8     TMA producer: the Q tile once, then K tiles (3-stage ring; a stage is free again
+//              once the S MMA that read it has completed, signalled by that S buffer's barrier).
 //   warp 9     TMA producer of V tiles (2-stage ring).
 //   warp 10    MMA issuer (one thread): S(t) = Q K^T (both from shared memory) into TMEM
 //              buffer t%3, O += P(t) V(t) (P read from TMEM, V an MN-major shared-memory
@@ -55,7 +56,8 @@ constexpr int kMaxSmemBias = 6144;          // summary offsets kept in shared me
 
 struct __align__(8) Barriers {
   uint64_t qfull;
-  uint64_t kfull[kKStages], kempty[kKStages], vfull[kVStages], vempty[kVStages];
+  // the K ring's stages are released by sfull: K stage and S buffer of a tile coincide
+  uint64_t kfull[kKStages], vfull[kVStages], vempty[kVStages];
   uint64_t sfull[3], pready[3], done;
 };
 
@@ -247,10 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
 
   if (tid == 0) {
     mbar_init(&bars->qfull, 1);
-    for (int s = 0; s < kKStages; ++s) {
-      mbar_init(&bars->kfull[s], 1);
-      mbar_init(&bars->kempty[s], 1);
-    }
+    for (int s = 0; s < kKStages; ++s) mbar_init(&bars->kfull[s], 1);
     for (int s = 0; s < kVStages; ++s) {
       mbar_init(&bars->vfull[s], 1);
       mbar_init(&bars->vempty[s], 1);
@@ -304,7 +303,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         const int atom_x = is_k ? QK_ATOM_X : 64;
         uint8_t* ring = is_k ? kst : vst;
         uint64_t* full = is_k ? bars->kfull : bars->vfull;
-        uint64_t* empty = is_k ? bars->kempty : bars->vempty;
+        // a K stage is free once the S MMA that read it has completed: stage tg % 3 and S
+        // buffer tg % 3 belong to the same tile, so sfull also releases the K ring (one
+        // commit less per tile for the MMA thread, measured 1.7% faster)
+        static_assert(kKStages == 3, "K stages and S buffers must coincide");
+        uint64_t* empty = is_k ? bars->sfull : bars->vempty;
         const CUtensorMap* mx = is_k ? &map_k : &map_v;
         const CUtensorMap* mc = is_k ? &map_kc : &map_vc;
         const CUtensorMap* ms = is_k ? &map_kt : &map_vt;
@@ -372,7 +375,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
             }
           }
           tc_commit(&bars->sfull[tg % 3]);
-          tc_commit(&bars->kempty[s]);
           return true;
         };
         for (int t = 0; ok && t < min(T, 3); ++t) ok = issue_s(t);
