@@ -463,9 +463,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
                                  selmask, nkb, x);
           uint32_t p16[16];
           float cs = exp32_at(x, 0, c, m_ref, p16);
-          tmem_st16(sbuf + half * 32, p16);
+          tmem_st16_issue(sbuf + half * 32, p16);
           cs += exp32_at(x, 32, c, m_ref, p16);
-          tmem_st16(sbuf + half * 32 + 16, p16);
+          tmem_st16_issue(sbuf + half * 32 + 16, p16);
           if (!(cs >= 0x1p-40f && cs <= 0x1p40f)) {
             const float mt = max64(x);
             m_true = fmaxf(m_true, ti.exact ? mt * tsl : mt);
@@ -473,6 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           rowsum += cs;
         }
         l_run += rowsum;
+        tmem_wait_st();                                 // P complete before it is signalled
         tc_fence_before_sync();
         mbar_arrive(&bars->pready[b]);
       }
