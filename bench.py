@@ -731,7 +731,8 @@ def main():
         "clocks": clock_info,
         "e2e": e2e,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    # the CPU leg times the bf16 oracle: it is reported for the bf16 line only
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not hp.fp8:
         per_call, threads, desc = oracle_sample(w, n_heads=2, n_units=320)
         line["cpu_baseline"] = {"value": dflops / per_call / 1e12, "unit": UNIT,
                                 "cores": threads, "kind": "oracle", "sample": desc,

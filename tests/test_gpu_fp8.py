@@ -13,7 +13,7 @@ import torch
 
 import _parity as P
 from block_sparse_attention_gather_b200 import (
-    spark_bsa_anchor, spark_bsa_attend_fp8, spark_bsa_forward_fp8,
+    SparkError, spark_bsa_anchor, spark_bsa_attend_fp8, spark_bsa_forward_fp8,
     spark_bsa_gather_kv_summarize, spark_bsa_gather_q, spark_bsa_quantize_fp8,
     spark_bsa_read_error, spark_bsa_topk_count, workspace_views)
 from block_sparse_attention_gather_b200.workloads import WORKLOADS, make_inputs, sample_units
@@ -106,7 +106,7 @@ def check_forward_fp8(x, ratio, heads=None, blocks_per_head=None, seed=0):
 def test_tiny_fp8_is_unsupported_for_d64():
     w = WORKLOADS["tiny-1x1024-d64-fp32"]
     x = {k: v.to(DEV) if torch.is_tensor(v) else v for k, v in make_inputs(w).items()}
-    with pytest.raises(Exception):
+    with pytest.raises(SparkError):
         spark_bsa_forward_fp8(x["Q"], x["K"], x["V"], x["q_perm"], x["k_perm"], x["q_offsets"],
                               x["k_offsets"], w.ratio)
 
