@@ -196,7 +196,7 @@ def workspace_views(workspace: torch.Tensor, layout: Layout, H, N, d, nqb, nkb) 
         "Vp": view(layout.Vp, H * N * d, torch.bfloat16).view(H, N, d),
         "qbar_blocks": view(layout.qbar_blocks, H * nqb * d, torch.float32).view(H, nqb, d),
         "qbar": view(layout.qbar, H * d, torch.float32).view(H, d),
-        "kbar": view(layout.kbar, H * nkb * d, torch.float32).view(H, nkb, d),
+        "kbar": view(layout.kbar, H * nkb * d, torch.float32).view(H, d, nkb),   # d-major
         "k_tilde": view(layout.k_tilde, H * nkb * d, torch.bfloat16).view(H, nkb, d),
         "v_tilde": view(layout.v_tilde, H * nkb * d, torch.bfloat16).view(H, nkb, d),
         "cbias": view(layout.cbias, H * nkb, torch.float32).view(H, nkb),
@@ -289,7 +289,7 @@ def spark_bsa_gather_kv_summarize(K, V, k_perm, k_offsets, qbar, err=None, strea
     _need(qbar, "qbar", torch.float32, dev)
     Kp = torch.empty(H, N, d, dtype=torch.bfloat16, device=dev)
     Vp = torch.empty_like(Kp)
-    kbar = torch.empty(H, nkb, d, dtype=torch.float32, device=dev)
+    kbar = torch.empty(H, d, nkb, dtype=torch.float32, device=dev)          # d-major
     k_tilde = torch.empty(H, nkb, d, dtype=torch.bfloat16, device=dev)
     v_tilde = torch.empty_like(k_tilde)
     cbias = torch.empty(H, nkb, dtype=torch.float32, device=dev)
@@ -305,7 +305,7 @@ def spark_bsa_route(qbar_blocks, kbar, k, err=None, stream=None):
     _need(qbar_blocks, "qbar_blocks", torch.float32)
     _need(kbar, "kbar", torch.float32, qbar_blocks.device)
     H, nqb, d = qbar_blocks.shape
-    nkb = kbar.shape[1]
+    nkb = kbar.shape[2]                                                     # kbar is [H, d, nkb]
     sel = torch.empty(H, nqb, k, dtype=torch.int32, device=qbar_blocks.device)
     st = lib().spark_bsa_route(_ptr(qbar_blocks), _ptr(kbar), H, nqb, nkb, d, int(k), _ptr(sel),
                                _ptr(err), _stream(stream))

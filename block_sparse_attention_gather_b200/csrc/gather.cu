@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(128) gather_kv_summary_kernel(
       cbias[bidx] = -INFINITY;
     }
     if (threadIdx.x < D) {
-      kbar[bidx * D + threadIdx.x] = 0.f;
+      kbar[(static_cast<size_t>(h) * D + threadIdx.x) * nkb + B] = 0.f;   // d-major
       k_tilde[bidx * D + threadIdx.x] = __float2bfloat16_rn(0.f);
       v_tilde[bidx * D + threadIdx.x] = __float2bfloat16_rn(0.f);
     }
@@ -291,7 +291,8 @@ __global__ void __launch_bounds__(128) gather_kv_summary_kernel(
     const __nv_bfloat16 kt = __float2bfloat16_rn(kk * inv);
     k_tilde[bidx * D + col] = kt;
     v_tilde[bidx * D + col] = __float2bfloat16_rn(vv * inv);
-    kbar[bidx * D + col] = ksum / static_cast<float>(m);
+    // d-major [H][D][nkb]: the routing kernel reads one coalesced row per dimension
+    kbar[(static_cast<size_t>(h) * D + col) * nkb + B] = ksum / static_cast<float>(m);
     // sigma * qbar . bf16(k~), reduced over the D columns (D/32 warps)
     float dq = sigma * qbar[static_cast<size_t>(h) * D + col] * __bfloat162float(kt);
 #pragma unroll

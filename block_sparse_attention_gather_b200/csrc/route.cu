@@ -3,11 +3,12 @@
 //
 // One CTA per (R consecutive query blocks, head), 512 threads:
 //   phase 1  S[r, B] = qbar_A(r) . kbar_B in fp32 (sequential FMA over d) for every key
-//            block.  A thread owns two key blocks at a time: their kbar rows stream through
-//            its registers in 8-element chunks straight from global memory (L2-resident:
-//            every CTA of the head reads them), the next chunk in flight while the current
-//            one is used, and the R query rows come from shared memory stored d-major, so
-//            each load is a warp-wide broadcast of four rows.  The scores of the R
+//            block.  A thread owns two key blocks at a time: their means stream through its
+//            registers in 8-dimension chunks straight from global memory (L2-resident: every
+//            CTA of the head reads them; kbar is stored d-major, so a warp's load is one
+//            coalesced row of 32 key blocks), the next chunk in flight while the current one
+//            is used, and the R query rows come from shared memory stored d-major, so each
+//            load is a warp-wide broadcast of four rows.  The scores of the R
 //            rows stay in shared memory as order-preserving uint32 keys.  The positive factor
 //            1/sqrt(d) is left out: it does not change the order.
 //   phase 2  one warp per row: an exact radix select (four 8-bit passes over the keys) finds
@@ -65,48 +66,48 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(const float* __restr
   __syncthreads();
 
   // ---- phase 1: scores (no collectives inside: the ragged last pass needs no uniformity)
-  const float4* kb4 = reinterpret_cast<const float4*>(kbar + static_cast<size_t>(h) * nkb * D);
+  // kbar is d-major ([D][nkb] per head): the threads of a warp read consecutive key blocks of
+  // one dimension, one coalesced 128-byte row per load.
+  const float* kbT = kbar + static_cast<size_t>(h) * D * nkb;
   for (int B0 = tid; B0 < nkb; B0 += kCols * kThreads) {
     float acc[kCols][R];
-    const float4* src[kCols];
+    int Bc[kCols];
     bool live[kCols];
 #pragma unroll
     for (int c = 0; c < kCols; ++c) {
       live[c] = B0 + c * kThreads < nkb;
-      src[c] = kb4 + static_cast<size_t>(live[c] ? B0 + c * kThreads : B0) * (D / 4);
+      Bc[c] = live[c] ? B0 + c * kThreads : B0;
 #pragma unroll
       for (int r = 0; r < R; ++r) acc[c][r] = 0.f;
     }
-    float4 b[kCols][kChunk / 4];
+    float b[kCols][kChunk];
 #pragma unroll
     for (int c = 0; c < kCols; ++c)
 #pragma unroll
-      for (int j = 0; j < kChunk / 4; ++j) b[c][j] = ld_nc_f4(src[c] + j);
+      for (int j = 0; j < kChunk; ++j) b[c][j] = __ldg(kbT + static_cast<size_t>(j) * nkb + Bc[c]);
 #pragma unroll 1
     for (int e0 = 0; e0 < D; e0 += kChunk) {
-      float4 nb[kCols][kChunk / 4];
+      float nb[kCols][kChunk];
       if (kPrefetch && e0 + kChunk < D) {
 #pragma unroll
         for (int c = 0; c < kCols; ++c)
 #pragma unroll
-          for (int j = 0; j < kChunk / 4; ++j) nb[c][j] = ld_nc_f4(src[c] + (e0 + kChunk) / 4 + j);
+          for (int j = 0; j < kChunk; ++j)
+            nb[c][j] = __ldg(kbT + static_cast<size_t>(e0 + kChunk + j) * nkb + Bc[c]);
       }
 #pragma unroll
-      for (int j = 0; j < kChunk / 4; ++j) {
+      for (int j = 0; j < kChunk; ++j) {
+        const float4* a = reinterpret_cast<const float4*>(qT + (e0 + j) * R);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4* a = reinterpret_cast<const float4*>(qT + (e0 + 4 * j + q) * R);
+        for (int r4 = 0; r4 < R / 4; ++r4) {
+          const float4 av = a[r4];
 #pragma unroll
-          for (int r4 = 0; r4 < R / 4; ++r4) {
-            const float4 av = a[r4];
-#pragma unroll
-            for (int c = 0; c < kCols; ++c) {
-              const float bv = q == 0 ? b[c][j].x : q == 1 ? b[c][j].y : q == 2 ? b[c][j].z : b[c][j].w;
-              acc[c][4 * r4 + 0] = fmaf(av.x, bv, acc[c][4 * r4 + 0]);
-              acc[c][4 * r4 + 1] = fmaf(av.y, bv, acc[c][4 * r4 + 1]);
-              acc[c][4 * r4 + 2] = fmaf(av.z, bv, acc[c][4 * r4 + 2]);
-              acc[c][4 * r4 + 3] = fmaf(av.w, bv, acc[c][4 * r4 + 3]);
-            }
+          for (int c = 0; c < kCols; ++c) {
+            const float bv = b[c][j];
+            acc[c][4 * r4 + 0] = fmaf(av.x, bv, acc[c][4 * r4 + 0]);
+            acc[c][4 * r4 + 1] = fmaf(av.y, bv, acc[c][4 * r4 + 1]);
+            acc[c][4 * r4 + 2] = fmaf(av.z, bv, acc[c][4 * r4 + 2]);
+            acc[c][4 * r4 + 3] = fmaf(av.w, bv, acc[c][4 * r4 + 3]);
           }
         }
       }
@@ -114,8 +115,9 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(const float* __restr
 #pragma unroll
         for (int c = 0; c < kCols; ++c)
 #pragma unroll
-          for (int j = 0; j < kChunk / 4; ++j)
-            b[c][j] = kPrefetch ? nb[c][j] : ld_nc_f4(src[c] + (e0 + kChunk) / 4 + j);
+          for (int j = 0; j < kChunk; ++j)
+            b[c][j] = kPrefetch ? nb[c][j]
+                                : __ldg(kbT + static_cast<size_t>(e0 + kChunk + j) * nkb + Bc[c]);
       }
     }
 #pragma unroll

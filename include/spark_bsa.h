@@ -97,7 +97,7 @@ typedef struct {
   size_t Qp, Kp, Vp;          /* bf16 [H,N,d] reblocked Q, K, V                          */
   size_t qbar_blocks;         /* fp32 [H,nqb,d] query-block means                        */
   size_t qbar;                /* fp32 [H,d] per-head anchor                              */
-  size_t kbar;                /* fp32 [H,nkb,d] key-block means                          */
+  size_t kbar;                /* fp32 [H,d,nkb] key-block means, d-major                 */
   size_t k_tilde, v_tilde;    /* bf16 [H,nkb,d] weighted summaries                       */
   size_t cbias;               /* fp32 [H,nkb] summary offsets c_B = b_B + log|B|        */
   size_t sel;                 /* int32 [H,nqb,k] selected key blocks, ascending          */
@@ -147,7 +147,8 @@ SPARK_API spark_status spark_bsa_anchor(const float* qbar_blocks, const int32_t*
                               int N, int d, int nqb, float* qbar, void* stream);
 
 /* Steps 1+3 fused (keys/values; blog "Spark-Reweight" weighted summaries and log-mass bias):
- * Kp, Vp (bf16 [H,N,d]) gathered by k_perm; kbar (fp32 [H,nkb,d]) block means;
+ * Kp, Vp (bf16 [H,N,d]) gathered by k_perm; kbar (fp32 [H,d,nkb], d-major: kbar[h][e][B] is
+ * dimension e of block B's mean) block means;
  * k_tilde, v_tilde (bf16 [H,nkb,d]) and cbias (fp32 [H,nkb]) as defined above, with
  * c_B computed against the bf16-rounded k~_B that the attention step consumes. */
 SPARK_API spark_status spark_bsa_gather_kv_summarize(const void* K, const void* V, int dtype, int H,
@@ -158,7 +159,8 @@ SPARK_API spark_status spark_bsa_gather_kv_summarize(const void* K, const void* 
                                            uint32_t* err, void* stream);
 
 /* Step 4 (blog "Discussion": block-mean scoring; "Spark-Reblock": fixed Top-K budget):
- * fp32 scores sigma*qbar_A.kbar_B, the k largest per (h,A) with ties to the smaller B,
+ * fp32 scores sigma*qbar_A.kbar_B (qbar_blocks [H,nqb,d], kbar d-major [H,d,nkb] as written by
+ * spark_bsa_gather_kv_summarize), the k largest per (h,A) with ties to the smaller B,
  * written ascending to sel [H,nqb,k].  1 <= k <= nkb <= SPARK_MAX_NKB. */
 SPARK_API spark_status spark_bsa_route(const float* qbar_blocks, const float* kbar, int H, int nqb,
                              int nkb, int d, int k, int32_t* sel, uint32_t* err, void* stream);

@@ -70,6 +70,8 @@ def check_forward(x, ratio, heads=None, blocks_per_head=None, seed=0, check_inte
             assert np.array_equal(P.to64(views["Vp"][h]), hi["V"][hi["k_perm"]])
             for name, refv in (("qbar_blocks", ref.qbar_blocks), ("kbar", ref.kbar)):
                 got = P.to64(views[name][h])
+                if name == "kbar":
+                    got = got.T                          # stored d-major [d, nkb]
                 err = np.abs(got - refv).max(axis=1) / np.maximum(np.linalg.norm(refv, axis=1), 1e-6)
                 assert err.max() < 1e-5, name
             gq = P.to64(views["qbar"][h])
