@@ -26,6 +26,7 @@ __all__ = [
     "spark_reblock_whiten", "spark_reblock_level", "reblock_views",
     "spark_bsa_host_staging_size", "spark_bsa_forward_host", "spark_bsa_quantize_fp8",
     "spark_bsa_attend_fp8", "spark_bsa_workspace_size_fp8", "spark_bsa_forward_fp8",
+    "spark_bsa_gather_kv_meanpool",
 ]
 
 SPARK_BF16, SPARK_F32 = 0, 1
@@ -40,6 +41,7 @@ EXPORTED = [
     "spark_reblock_levels", "spark_reblock", "spark_reblock_whiten", "spark_reblock_level",
     "spark_bsa_host_staging_size", "spark_bsa_forward_host", "spark_bsa_quantize_fp8",
     "spark_bsa_attend_fp8", "spark_bsa_workspace_size_fp8", "spark_bsa_forward_fp8",
+    "spark_bsa_gather_kv_meanpool",
 ]
 REBLOCK_MODES = {"q_reuse_k": 0, "separate": 1}
 
@@ -111,6 +113,8 @@ def lib():
         "spark_bsa_forward_host": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _I, _D,
                                         _P, _I, _P, _SZ, _P, _SZ, _P, _P, _P]),
         "spark_bsa_quantize_fp8": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P]),
+        "spark_bsa_gather_kv_meanpool": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P,
+                                              _P, _P, _P, _P, _P]),
         "spark_bsa_attend_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I,
                                       _P, _P, _I, _P, _I, _I, _I, _I, _P, _I, _P, _P]),
         "spark_bsa_workspace_size_fp8": (_SZ, [_I, _I, _I, _I, _I, _D, _I]),
@@ -298,6 +302,31 @@ def spark_bsa_gather_kv_summarize(K, V, k_perm, k_offsets, qbar, err=None, strea
         _ptr(qbar), _ptr(Kp), _ptr(Vp), _ptr(kbar), _ptr(k_tilde), _ptr(v_tilde), _ptr(cbias),
         _ptr(err), _stream(stream))
     _check("spark_bsa_gather_kv_summarize", st)
+    return Kp, Vp, kbar, k_tilde, v_tilde, cbias
+
+
+def spark_bsa_gather_kv_meanpool(K, V, k_perm, k_offsets, err=None, stream=None):
+    """The baseline BSA compressed branch (mean key, mean value, offset log|B|) with the same
+    gathered Kp, Vp and key-block means as spark_bsa_gather_kv_summarize; returns
+    (Kp, Vp, kbar, k_tilde, v_tilde, cbias)."""
+    _need(K, "K", (torch.bfloat16, torch.float32))
+    dev = K.device
+    H, N, d = K.shape
+    _need(V, "V", K.dtype, dev)
+    _need(k_perm, "k_perm", torch.int32, dev)
+    _need(k_offsets, "k_offsets", torch.int32, dev)
+    nkb = k_offsets.numel() - 1
+    Kp = torch.empty(H, N, d, dtype=torch.bfloat16, device=dev)
+    Vp = torch.empty_like(Kp)
+    kbar = torch.empty(H, d, nkb, dtype=torch.float32, device=dev)          # d-major
+    k_tilde = torch.empty(H, nkb, d, dtype=torch.bfloat16, device=dev)
+    v_tilde = torch.empty_like(k_tilde)
+    cbias = torch.empty(H, nkb, dtype=torch.float32, device=dev)
+    st = lib().spark_bsa_gather_kv_meanpool(
+        _ptr(K), _ptr(V), _code(K.dtype), H, N, d, _ptr(k_perm), _ptr(k_offsets), nkb, _ptr(Kp),
+        _ptr(Vp), _ptr(kbar), _ptr(k_tilde), _ptr(v_tilde), _ptr(cbias), _ptr(err),
+        _stream(stream))
+    _check("spark_bsa_gather_kv_meanpool", st)
     return Kp, Vp, kbar, k_tilde, v_tilde, cbias
 
 

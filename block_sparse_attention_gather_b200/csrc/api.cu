@@ -370,6 +370,24 @@ spark_status spark_bsa_gather_kv_summarize(const void* K, const void* V, int dty
                                             as_stream(stream)));
 }
 
+spark_status spark_bsa_gather_kv_meanpool(const void* K, const void* V, int dtype, int H, int N,
+                                          int d, const int32_t* k_perm,
+                                          const int32_t* k_block_offsets, int nkb, void* Kp,
+                                          void* Vp, float* kbar, void* k_tilde, void* v_tilde,
+                                          float* cbias, uint32_t* err, void* stream) {
+  if (!K || !V || !k_perm || !k_block_offsets || !Kp || !Vp || !kbar || !k_tilde || !v_tilde ||
+      !cbias)
+    return SPARK_ERR_INVALID_ARG;
+  if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  spark_status st = check_sizes(H, N, d, 1, nkb);
+  if (st != SPARK_OK) return st;
+  if (!aligned(K, 16) || !aligned(V, 16) || !aligned(Kp, 16) || !aligned(Vp, 16))
+    return SPARK_ERR_INVALID_ARG;
+  return from_cuda(launch_gather_kv_meanpool(K, V, dtype, H, N, d, k_perm, k_block_offsets, nkb,
+                                             Kp, Vp, kbar, k_tilde, v_tilde, cbias, err,
+                                             as_stream(stream)));
+}
+
 spark_status spark_bsa_route(const float* qbar_blocks, const float* kbar, int H, int nqb,
                              int nkb, int d, int k, int32_t* sel, uint32_t* err, void* stream) {
   if (!qbar_blocks || !kbar || !sel) return SPARK_ERR_INVALID_ARG;

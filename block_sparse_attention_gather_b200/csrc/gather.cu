@@ -170,7 +170,10 @@ __global__ void __launch_bounds__(1024) anchor_kernel(const float* __restrict__ 
 
 // ------------------------------------------------------------------ gather_kv + summaries
 
-template <int D, typename T>
+// kMeanPool: the baseline BSA compressed branch instead of Spark-Reweight's (blog
+// "Spark-Reblock", BSA equations: each unselected block repeats its uniform mean key and value
+// |B| times; as one row that is k~ = mean key, v~ = mean value, offset c = log|B|).
+template <int D, typename T, bool kMeanPool = false>
 __global__ void __launch_bounds__(128) gather_kv_summary_kernel(
     const T* __restrict__ K, const T* __restrict__ V, const int32_t* __restrict__ k_perm,
     const int32_t* __restrict__ k_offsets, int N, int nkb, const float* __restrict__ qbar,
@@ -203,7 +206,8 @@ __global__ void __launch_bounds__(128) gather_kv_summary_kernel(
   const float sigma = rsqrtf(static_cast<float>(D));
   float qs[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) qs[e] = sigma * qbar[static_cast<size_t>(h) * D + c * 8 + e];
+  for (int e = 0; e < 8; ++e)
+    qs[e] = kMeanPool ? 0.f : sigma * qbar[static_cast<size_t>(h) * D + c * 8 + e];   // no anchor
 
   float run_m = -INFINITY, run_l = 0.f;
   float ak[8], av[8], ks[8];
@@ -239,6 +243,18 @@ __global__ void __launch_bounds__(128) gather_kv_summary_kernel(
       float fk[8], fv[8];
       unpack_bf16x8(kv[u].packed, fk);
       unpack_bf16x8(vv[u].packed, fv);
+      if constexpr (kMeanPool) {
+        if (live) {
+          st_v4(Kp + (head + lo + r) * D + c * 8, kv[u].packed);
+          st_v4(Vp + (head + lo + r) * D + c * 8, vv[u].packed);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            ks[e] += fk[e];
+            av[e] += fv[e];                       // the value sum
+          }
+        }
+        continue;
+      }
       float dot = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) dot = fmaf(qs[e], fk[e], dot);
@@ -273,6 +289,23 @@ __global__ void __launch_bounds__(128) gather_kv_summary_kernel(
     s_ks[g][c * 8 + e] = ks[e];
   }
   __syncthreads();
+  if constexpr (kMeanPool) {
+    if (threadIdx.x < D) {
+      const int col = threadIdx.x;
+      float ksum = 0.f, vsum = 0.f;
+#pragma unroll
+      for (int gg = 0; gg < RG; ++gg) {
+        ksum += s_ks[gg][col];
+        vsum += s_v[gg][col];
+      }
+      const float inv_m = 1.f / static_cast<float>(m);
+      k_tilde[bidx * D + col] = __float2bfloat16_rn(ksum * inv_m);
+      v_tilde[bidx * D + col] = __float2bfloat16_rn(vsum * inv_m);
+      kbar[(static_cast<size_t>(h) * D + col) * nkb + B] = ksum / static_cast<float>(m);
+      if (col == 0) cbias[bidx] = logf(static_cast<float>(m));
+    }
+    return;
+  }
   if (threadIdx.x < D) {
     const int col = threadIdx.x;
     float M = -INFINITY;
@@ -343,14 +376,14 @@ cudaError_t launch_anchor(const float* qbar_blocks, const int32_t* q_offsets, in
   return cudaGetLastError();
 }
 
-template <int D, typename T>
+template <int D, typename T, bool kMeanPool = false>
 static cudaError_t launch_kv_t(const void* K, const void* V, int H, int N,
                                const int32_t* k_perm, const int32_t* k_offsets, int nkb,
                                const float* qbar, void* Kp, void* Vp, float* kbar,
                                void* k_tilde, void* v_tilde, float* cbias, uint32_t* err,
                                cudaStream_t s) {
   dim3 grid(nkb, H);
-  gather_kv_summary_kernel<D, T><<<grid, 128, 0, s>>>(
+  gather_kv_summary_kernel<D, T, kMeanPool><<<grid, 128, 0, s>>>(
       static_cast<const T*>(K), static_cast<const T*>(V), k_perm, k_offsets, N, nkb, qbar,
       static_cast<__nv_bfloat16*>(Kp), static_cast<__nv_bfloat16*>(Vp), kbar,
       static_cast<__nv_bfloat16*>(k_tilde), static_cast<__nv_bfloat16*>(v_tilde), cbias, err);
@@ -373,6 +406,26 @@ cudaError_t launch_gather_kv_summary(const void* K, const void* V, int dtype, in
                                               kbar, k_tilde, v_tilde, cbias, err, s)
              : launch_kv_t<64, float>(K, V, H, N, k_perm, k_offsets, nkb, qbar, Kp, Vp, kbar,
                                       k_tilde, v_tilde, cbias, err, s);
+}
+
+cudaError_t launch_gather_kv_meanpool(const void* K, const void* V, int dtype, int H, int N,
+                                      int d, const int32_t* k_perm, const int32_t* k_offsets,
+                                      int nkb, void* Kp, void* Vp, float* kbar, void* k_tilde,
+                                      void* v_tilde, float* cbias, uint32_t* err,
+                                      cudaStream_t s) {
+  if (d == 128)
+    return dtype == 0
+               ? launch_kv_t<128, __nv_bfloat16, true>(K, V, H, N, k_perm, k_offsets, nkb,
+                                                       nullptr, Kp, Vp, kbar, k_tilde, v_tilde,
+                                                       cbias, err, s)
+               : launch_kv_t<128, float, true>(K, V, H, N, k_perm, k_offsets, nkb, nullptr, Kp,
+                                               Vp, kbar, k_tilde, v_tilde, cbias, err, s);
+  return dtype == 0
+             ? launch_kv_t<64, __nv_bfloat16, true>(K, V, H, N, k_perm, k_offsets, nkb, nullptr,
+                                                    Kp, Vp, kbar, k_tilde, v_tilde, cbias, err,
+                                                    s)
+             : launch_kv_t<64, float, true>(K, V, H, N, k_perm, k_offsets, nkb, nullptr, Kp, Vp,
+                                            kbar, k_tilde, v_tilde, cbias, err, s);
 }
 
 // Context rows to bf16 (round to nearest even), four elements per thread and iteration.

@@ -21,6 +21,14 @@ cudaError_t launch_gather_kv_summary(const void* K, const void* V, int dtype, in
                                      float* kbar, void* k_tilde, void* v_tilde, float* cbias,
                                      uint32_t* err, cudaStream_t s);
 
+// The baseline BSA compressed branch (mean key, mean value, offset log|B|) with the same
+// gather and key-block means as launch_gather_kv_summary.
+cudaError_t launch_gather_kv_meanpool(const void* K, const void* V, int dtype, int H, int N,
+                                      int d, const int32_t* k_perm, const int32_t* k_offsets,
+                                      int nkb, void* Kp, void* Vp, float* kbar, void* k_tilde,
+                                      void* v_tilde, float* cbias, uint32_t* err,
+                                      cudaStream_t s);
+
 cudaError_t launch_route(const float* qbar_blocks, const float* kbar, int H, int nqb, int nkb,
                          int d, int k, int32_t* sel, uint32_t* err, cudaStream_t s);
 

@@ -158,6 +158,19 @@ SPARK_API spark_status spark_bsa_gather_kv_summarize(const void* K, const void* 
                                            void* k_tilde, void* v_tilde, float* cbias,
                                            uint32_t* err, void* stream);
 
+/* Step 1+3 with the baseline BSA compressed branch instead of Spark-Reweight's, as the
+ * comparator of the blog's ablations (section "Spark-Reblock", BSA equations: an unselected
+ * block repeats its uniform mean key and value |B| times): the same Kp, Vp and kbar as
+ * spark_bsa_gather_kv_summarize, with k_tilde = bf16(mean key), v_tilde = bf16(mean value)
+ * and cbias = log|B| (the |B| copies as one row).  No anchor is used.  The attention step
+ * then takes these in place of the weighted summaries. */
+SPARK_API spark_status spark_bsa_gather_kv_meanpool(const void* K, const void* V, int dtype, int H,
+                                                    int N, int d, const int32_t* k_perm,
+                                                    const int32_t* k_block_offsets, int nkb,
+                                                    void* Kp, void* Vp, float* kbar,
+                                                    void* k_tilde, void* v_tilde, float* cbias,
+                                                    uint32_t* err, void* stream);
+
 /* Step 4 (blog "Discussion": block-mean scoring; "Spark-Reblock": fixed Top-K budget):
  * fp32 scores sigma*qbar_A.kbar_B (qbar_blocks [H,nqb,d], kbar d-major [H,d,nkb] as written by
  * spark_bsa_gather_kv_summarize), the k largest per (h,A) with ties to the smaller B,

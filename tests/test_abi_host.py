@@ -124,6 +124,16 @@ def test_step_entry_points_reject_bad_arguments(L):
     assert L.spark_bsa_read_error(None, None, ctypes.byref(flags)) == INVALID
 
 
+def test_meanpool_entry_point_rejects_bad_arguments(L):
+    p = ctypes.c_void_p(0x100000)
+    assert L.spark_bsa_gather_kv_meanpool(p, p, 0, 1, 10, 128, p, p, 1, p, p, p, p, p, None,
+                                          None, None) == INVALID                 # cbias NULL
+    assert L.spark_bsa_gather_kv_meanpool(p, p, 2, 1, 10, 128, p, p, 1, p, p, p, p, p, p,
+                                          None, None) == INVALID                 # dtype
+    assert L.spark_bsa_gather_kv_meanpool(p, p, 0, 1, 10, 96, p, p, 1, p, p, p, p, p, p,
+                                          None, None) == UNSUPPORTED             # d
+
+
 def test_fp8_entry_points_reject_bad_arguments(L):
     p = ctypes.c_void_p(0x100000)
     # quantise: null operands, d not 64/128, tiles with the wrong group count
