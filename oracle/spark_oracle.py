@@ -69,6 +69,7 @@ __all__ = [
     "route_scores",
     "route_block",
     "route",
+    "route_threshold_block",
     "attend_block",
     "HeadResult",
     "forward_head",
@@ -196,6 +197,21 @@ def route(qbar_blocks: np.ndarray, kbar: np.ndarray, scale: float, k: int):
     S = route_scores(qbar_blocks, kbar, scale)
     sel = np.stack([route_block(S[A], k) for A in range(S.shape[0])])
     return sel, S
+
+
+def route_threshold_block(scores_A: np.ndarray, tau: float, kcap: int) -> np.ndarray:
+    """Sol-Attn's content-adaptive routing, as the comparator the Spark-H3 blog's "Discussion"
+    describes: the block-level logits of a query block are taken as roughly Gaussian and the
+    blocks above mu + tau * sigma get exact attention.  Readings (T1): mu and sigma are the
+    mean and the population standard deviation of the query block's nKB scores; "above" is
+    strict; at most kcap blocks are kept, the largest (ties to the smaller index), so a caller
+    can bound the exact branch; the set is reported ascending and may be empty."""
+    S = np.asarray(scores_A, dtype=np.float64)
+    thr = S.mean() + tau * S.std()
+    above = np.flatnonzero(S > thr)
+    if len(above) > kcap:
+        return route_block(S, kcap)
+    return above.astype(np.int64)
 
 
 def attend_block(Qp_A: np.ndarray, Kp: np.ndarray, Vp: np.ndarray, k_offsets: np.ndarray,

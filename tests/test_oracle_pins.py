@@ -630,3 +630,59 @@ def test_pins_catch_planted_mistake(mutation, monkeypatch):
 
 def name_of(mutation):
     return mutation(lambda *a, **k: None)[0]
+
+
+# ---------------------------------------------------------------- threshold routing (T1)
+
+def test_threshold_routing_is_affine_invariant_and_monotone():
+    """mu + tau*sigma moves with any positive affine change of the scores, so the selection
+    does not (a variance in place of sigma, or a dropped mu, breaks this); a larger tau never
+    selects more."""
+    rng = np.random.default_rng(40)
+    for _ in range(50):
+        S = rng.standard_normal(300) * rng.uniform(0.1, 5) + rng.uniform(-3, 3)
+        tau = rng.uniform(-1, 2.5)
+        a = O.route_threshold_block(S, tau, 300)
+        for scale, shift in ((3.7, 0.0), (0.21, 5.0), (1.0, -11.0)):
+            b = O.route_threshold_block(S * scale + shift, tau, 300)
+            assert np.array_equal(a, b)
+        c = O.route_threshold_block(S, tau + 0.3, 300)
+        assert set(c.tolist()) <= set(a.tolist())
+
+
+def test_threshold_routing_gaussian_fraction_and_limits():
+    """For Gaussian scores the selected fraction is the normal tail 1 - Phi(tau); a very
+    negative tau keeps every block, a very large one none; ties at the threshold stay out."""
+    from scipy.stats import norm
+    rng = np.random.default_rng(41)
+    S = rng.standard_normal(200000)
+    for tau in (-0.5, 0.0, 1.0, 2.0):
+        frac = len(O.route_threshold_block(S, tau, len(S))) / len(S)
+        assert abs(frac - (1 - norm.cdf(tau))) < 5e-3
+    small = rng.standard_normal(40)
+    assert len(O.route_threshold_block(small, -50.0, 40)) == 40
+    assert len(O.route_threshold_block(small, 50.0, 40)) == 0
+    assert len(O.route_threshold_block(np.full(10, 2.0), 0.0, 10)) == 0     # sigma = 0
+
+
+def test_threshold_routing_cap_keeps_the_top_blocks():
+    """With more blocks above the threshold than the cap, the cap's top blocks by score (ties to
+    the smaller index) are kept, i.e. the Top-K router's choice."""
+    rng = np.random.default_rng(42)
+    S = np.round(rng.standard_normal(500), 1)          # many exact ties
+    sel = O.route_threshold_block(S, -1.0, 37)
+    assert len(sel) == 37
+    assert np.array_equal(sel, O.route_block(S, 37))
+    # brute force on a tiny case: the cap's set by enumeration of the order
+    S = np.array([0.3, 2.0, 2.0, -1.0, 1.5, 2.0, 0.0])
+    assert O.route_threshold_block(S, -0.2, 2).tolist() == [1, 2]
+
+
+def test_threshold_routing_hand_case():
+    """Closed form: S = (0, 0, 0, 0, 10) has mu = 2 and sigma = 4 (population), so tau = -0.4
+    puts the threshold at 0.4 (only block 4 is above) and tau = -0.6 at -0.4 (all are)."""
+    S = np.array([0.0, 0.0, 0.0, 0.0, 10.0])
+    assert O.route_threshold_block(S, -0.4, 5).tolist() == [4]
+    assert O.route_threshold_block(S, -0.6, 5).tolist() == [0, 1, 2, 3, 4]
+    assert O.route_threshold_block(S, 1.9, 5).tolist() == [4]       # 9.6 < 10
+    assert O.route_threshold_block(S, 2.0, 5).tolist() == []        # 10 is not above 10
