@@ -228,8 +228,9 @@ def attend_block(Qp_A: np.ndarray, Kp: np.ndarray, Vp: np.ndarray, k_offsets: np
     k_offsets = np.asarray(k_offsets, dtype=np.int64)
     nkb = len(k_offsets) - 1
     selected = set(int(b) for b in sel_A)
-    exact_rows = np.concatenate(
-        [np.arange(k_offsets[B], k_offsets[B + 1]) for B in sorted(selected)])
+    exact_rows = (np.concatenate([np.arange(k_offsets[B], k_offsets[B + 1])
+                                  for B in sorted(selected)])
+                  if selected else np.zeros(0, dtype=np.int64))   # threshold routing: may be empty
     comp = np.array([B for B in range(nkb) if B not in selected], dtype=np.int64)
 
     logits_exact = scale * (Qp_A @ Kp[exact_rows].T)

@@ -686,3 +686,19 @@ def test_threshold_routing_hand_case():
     assert O.route_threshold_block(S, -0.6, 5).tolist() == [0, 1, 2, 3, 4]
     assert O.route_threshold_block(S, 1.9, 5).tolist() == [4]       # 9.6 < 10
     assert O.route_threshold_block(S, 2.0, 5).tolist() == []        # 10 is not above 10
+
+
+def test_empty_selection_is_the_compressed_branch_alone():
+    """Threshold routing may select no block (T1): the attention is then the compressed branch
+    alone, which for blocks of identical keys is still dense attention (pin P2's identity)."""
+    rng = np.random.default_rng(43)
+    d, nb, bs = 16, 6, 5
+    N = nb * bs
+    ko = np.arange(0, N + 1, bs)
+    K = np.repeat(rng.standard_normal((nb, d)), bs, axis=0)
+    V = rng.standard_normal((N, d))
+    Q = rng.standard_normal((7, d))
+    qbar = rng.standard_normal(d)
+    kt, vt, c = O.summarize(K, V, ko, qbar, 1.0 / math.sqrt(d))
+    got = O.attend_block(Q, K, V, ko, np.zeros(0, dtype=np.int64), kt, vt, c, 1.0 / math.sqrt(d))
+    assert np.abs(got - O.dense_attention(Q, K, V)).max() < 1e-12
