@@ -26,7 +26,7 @@ __all__ = [
     "spark_reblock_whiten", "spark_reblock_level", "reblock_views",
     "spark_bsa_host_staging_size", "spark_bsa_forward_host", "spark_bsa_quantize_fp8",
     "spark_bsa_attend_fp8", "spark_bsa_workspace_size_fp8", "spark_bsa_forward_fp8",
-    "spark_bsa_gather_kv_meanpool",
+    "spark_bsa_gather_kv_meanpool", "spark_bsa_route_threshold", "spark_bsa_attend_var",
 ]
 
 SPARK_BF16, SPARK_F32 = 0, 1
@@ -41,7 +41,7 @@ EXPORTED = [
     "spark_reblock_levels", "spark_reblock", "spark_reblock_whiten", "spark_reblock_level",
     "spark_bsa_host_staging_size", "spark_bsa_forward_host", "spark_bsa_quantize_fp8",
     "spark_bsa_attend_fp8", "spark_bsa_workspace_size_fp8", "spark_bsa_forward_fp8",
-    "spark_bsa_gather_kv_meanpool",
+    "spark_bsa_gather_kv_meanpool", "spark_bsa_route_threshold", "spark_bsa_attend_var",
 ]
 REBLOCK_MODES = {"q_reuse_k": 0, "separate": 1}
 
@@ -113,6 +113,9 @@ def lib():
         "spark_bsa_forward_host": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _I, _D,
                                         _P, _I, _P, _SZ, _P, _SZ, _P, _P, _P]),
         "spark_bsa_quantize_fp8": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P]),
+        "spark_bsa_route_threshold": (_I, [_P, _P, _I, _I, _I, _I, _D, _I, _P, _P, _P, _P]),
+        "spark_bsa_attend_var": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _P, _I,
+                                      _I, _I, _I, _P, _I, _P, _P]),
         "spark_bsa_gather_kv_meanpool": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P,
                                               _P, _P, _P, _P, _P]),
         "spark_bsa_attend_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I,
@@ -303,6 +306,47 @@ def spark_bsa_gather_kv_summarize(K, V, k_perm, k_offsets, qbar, err=None, strea
         _ptr(err), _stream(stream))
     _check("spark_bsa_gather_kv_summarize", st)
     return Kp, Vp, kbar, k_tilde, v_tilde, cbias
+
+
+def spark_bsa_route_threshold(qbar_blocks, kbar, tau, kcap, err=None, stream=None):
+    """Threshold routing (mu + tau*sigma per query block, at most kcap blocks); returns
+    (sel [H, nqb, kcap] with the first count entries of each row valid, count [H, nqb])."""
+    _need(qbar_blocks, "qbar_blocks", torch.float32)
+    _need(kbar, "kbar", torch.float32, qbar_blocks.device)
+    H, nqb, d = qbar_blocks.shape
+    nkb = kbar.shape[2]                                                     # kbar is [H, d, nkb]
+    sel = torch.full((H, nqb, kcap), -1, dtype=torch.int32, device=qbar_blocks.device)
+    count = torch.empty(H, nqb, dtype=torch.int32, device=qbar_blocks.device)
+    st = lib().spark_bsa_route_threshold(_ptr(qbar_blocks), _ptr(kbar), H, nqb, nkb, d,
+                                         float(tau), int(kcap), _ptr(sel), _ptr(count),
+                                         _ptr(err), _stream(stream))
+    _check("spark_bsa_route_threshold", st)
+    return sel, count
+
+
+def spark_bsa_attend_var(Qp, Kp, Vp, k_tilde, v_tilde, cbias, sel, count, q_perm, q_offsets,
+                         k_offsets, out_dtype=torch.bfloat16, out=None, err=None, stream=None):
+    """spark_bsa_attend with a per-query-block count of selected blocks (sel [H, nqb, kcap])."""
+    _need(Qp, "Qp", torch.bfloat16)
+    dev = Qp.device
+    H, N, d = Qp.shape
+    for n, t, dt in (("Kp", Kp, torch.bfloat16), ("Vp", Vp, torch.bfloat16),
+                     ("k_tilde", k_tilde, torch.bfloat16), ("v_tilde", v_tilde, torch.bfloat16),
+                     ("cbias", cbias, torch.float32), ("sel", sel, torch.int32),
+                     ("count", count, torch.int32), ("q_perm", q_perm, torch.int32),
+                     ("q_offsets", q_offsets, torch.int32), ("k_offsets", k_offsets, torch.int32)):
+        _need(t, n, dt, dev)
+    nqb, nkb = q_offsets.numel() - 1, k_offsets.numel() - 1
+    kcap = sel.shape[-1]
+    if out is None:
+        out = torch.empty(H, N, d, dtype=out_dtype, device=dev)
+    _need(out, "out", out_dtype, dev)
+    st = lib().spark_bsa_attend_var(_ptr(Qp), _ptr(Kp), _ptr(Vp), _ptr(k_tilde), _ptr(v_tilde),
+                                    _ptr(cbias), _ptr(sel), kcap, _ptr(count), _ptr(q_perm),
+                                    _ptr(q_offsets), nqb, _ptr(k_offsets), nkb, H, N, d,
+                                    _ptr(out), _code(out_dtype), _ptr(err), _stream(stream))
+    _check("spark_bsa_attend_var", st)
+    return out
 
 
 def spark_bsa_gather_kv_meanpool(K, V, k_perm, k_offsets, err=None, stream=None):

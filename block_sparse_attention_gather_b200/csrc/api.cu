@@ -127,7 +127,7 @@ spark_status attend_impl(const void* Qp, const void* Kp, const void* Vp, const v
                          const void* Kc, const void* Vc, int nc, const int32_t* q_perm,
                          const int32_t* q_offsets, int nqb, const int32_t* k_offsets, int nkb,
                          int H, int N, int d, void* out, int out_dtype, uint32_t* err,
-                         cudaStream_t s) {
+                         cudaStream_t s, const int32_t* sel_count = nullptr) {
   AttendMaps maps;
   if (!encode_rows_map(&maps.q, Qp, H, N, d) || !encode_rows_map(&maps.k, Kp, H, N, d) ||
       !encode_rows_map(&maps.v, Vp, H, N, d) || !encode_rows_map(&maps.kt, k_tilde, H, nkb, d) ||
@@ -141,7 +141,7 @@ spark_status attend_impl(const void* Qp, const void* Kp, const void* Vp, const v
     maps.vc = maps.v;
   }
   return from_cuda(launch_attend(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb, k_offsets, nkb,
-                                 H, N, d, out, out_dtype, err, s));
+                                 H, N, d, out, out_dtype, err, s, sel_count));
 }
 
 // FP8 logits: e4m3 Qp8/Kp8/kt8/Kc8 with their group scales, bf16 values.
@@ -487,6 +487,44 @@ spark_status spark_bsa_forward(const void* Q, const void* K, const void* V, int 
   return forward_impl(Q, K, V, nullptr, nullptr, 0, dtype, H, N, d, q_perm, k_perm,
                       q_block_offsets, nqb, k_block_offsets, nkb, topk_ratio, out, workspace,
                       workspace_bytes, as_stream(stream));
+}
+
+// ----------------------------------------------------------- threshold routing (comparator)
+
+spark_status spark_bsa_route_threshold(const float* qbar_blocks, const float* kbar, int H,
+                                       int nqb, int nkb, int d, double tau, int kcap,
+                                       int32_t* sel, int32_t* count, uint32_t* err,
+                                       void* stream) {
+  if (!qbar_blocks || !kbar || !sel || !count) return SPARK_ERR_INVALID_ARG;
+  if (H < 1 || nqb < 1 || nkb < 1 || kcap < 1 || kcap > nkb || !(tau == tau))
+    return SPARK_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SPARK_ERR_UNSUPPORTED;
+  if (H > 65535 || nkb > kMaxNkb) return SPARK_ERR_UNSUPPORTED;
+  (void)err;
+  return from_cuda(launch_route_threshold(qbar_blocks, kbar, H, nqb, nkb, d,
+                                          static_cast<float>(tau), kcap, sel, count,
+                                          as_stream(stream)));
+}
+
+spark_status spark_bsa_attend_var(const void* Qp, const void* Kp, const void* Vp,
+                                  const void* k_tilde, const void* v_tilde, const float* cbias,
+                                  const int32_t* sel, int kcap, const int32_t* count,
+                                  const int32_t* q_perm, const int32_t* q_block_offsets, int nqb,
+                                  const int32_t* k_block_offsets, int nkb, int H, int N, int d,
+                                  void* out, int out_dtype, uint32_t* err, void* stream) {
+  if (!Qp || !Kp || !Vp || !k_tilde || !v_tilde || !cbias || !sel || !count || !q_perm ||
+      !q_block_offsets || !k_block_offsets || !out)
+    return SPARK_ERR_INVALID_ARG;
+  if (out_dtype != SPARK_BF16 && out_dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  spark_status st = check_sizes(H, N, d, nqb, nkb);
+  if (st != SPARK_OK) return st;
+  if (kcap < 1 || kcap > nkb) return SPARK_ERR_INVALID_ARG;
+  if (!aligned(Qp, 16) || !aligned(Kp, 16) || !aligned(Vp, 16) || !aligned(k_tilde, 16) ||
+      !aligned(v_tilde, 16) || !aligned(out, 16))
+    return SPARK_ERR_INVALID_ARG;
+  return attend_impl(Qp, Kp, Vp, k_tilde, v_tilde, cbias, sel, kcap, nullptr, nullptr, 0, q_perm,
+                     q_block_offsets, nqb, k_block_offsets, nkb, H, N, d, out, out_dtype, err,
+                     as_stream(stream), count);
 }
 
 // ------------------------------------------------------------------------ FP8 logits

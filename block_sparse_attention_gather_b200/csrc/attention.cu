@@ -204,7 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kt,
     const __grid_constant__ CUtensorMap map_vt, const __grid_constant__ CUtensorMap map_kc,
     const __grid_constant__ CUtensorMap map_vc, int nc, const float* __restrict__ cbias,
-    const int32_t* __restrict__ sel, int k, const int32_t* __restrict__ q_perm,
+    const int32_t* __restrict__ sel, int kcap, const int32_t* __restrict__ sel_count,
+    const int32_t* __restrict__ q_perm,
     const int32_t* __restrict__ q_offsets, int nqb, const int32_t* __restrict__ k_offsets,
     int nkb, int N, void* __restrict__ out, int out_dtype, uint32_t* err, const Fp8Scales sc) {
   static_assert(!kFp8 || D == 128, "FP8 logits: d = 128 (one 128-byte row per key)");
@@ -239,10 +240,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   }
   __syncthreads();
   if (s_skip) return;                                      // uniform: no work, nothing held
+  // selected blocks of this query block: kcap, or its own count (threshold routing) when
+  // sel_count is given; rows of sel are kcap apart either way
+  const int k = sel_count ? max(0, min(sel_count[static_cast<size_t>(h) * nqb + A], kcap)) : kcap;
   const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
   const int nxt = (nc + 127) / 128;                 // context tiles
   const int T = k + nxt + nct;
-  const int32_t* sel_row = sel + (static_cast<size_t>(h) * nqb + A) * k;
+  const int32_t* sel_row = sel + (static_cast<size_t>(h) * nqb + A) * kcap;
   const int nwords = (nkb + 31) / 32;
   const float* cb = cbias + static_cast<size_t>(h) * nkb;
   const int qlo = q_offsets[A];
@@ -560,20 +564,21 @@ static size_t attend_smem_bytes(int d, int nkb, int k, bool fp8) {
 
 template <int D, bool kBiasSmem, bool kFp8>
 static cudaError_t launch_attend_t(const AttendMaps& m, int nc, const float* cbias,
-                                   const int32_t* sel, int k, const int32_t* q_perm,
-                                   const int32_t* q_offsets,
+                                   const int32_t* sel, int k, const int32_t* sel_count,
+                                   const int32_t* q_perm, const int32_t* q_offsets,
                                    int nqb, const int32_t* k_offsets, int nkb, int H, int N,
                                    void* out, int out_dtype, uint32_t* err, const Fp8Scales& sc,
                                    cudaStream_t s) {
-  const size_t smem = attend_smem_bytes(D, nkb, k, kFp8);
+  // with per-row counts any row may have summary tiles: size for k < nkb
+  const size_t smem = attend_smem_bytes(D, nkb, sel_count ? 0 : k, kFp8);
   cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, kBiasSmem, kFp8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(nqb, H);
   attend_kernel<D, kBiasSmem, kFp8><<<grid, kThreads, smem, s>>>(
-      m.q, m.k, m.v, m.kt, m.vt, m.kc, m.vc, nc, cbias, sel, k, q_perm, q_offsets, nqb,
-      k_offsets, nkb, N, out, out_dtype, err, sc);
+      m.q, m.k, m.v, m.kt, m.vt, m.kc, m.vc, nc, cbias, sel, k, sel_count, q_perm, q_offsets,
+      nqb, k_offsets, nkb, N, out, out_dtype, err, sc);
   return cudaGetLastError();
 }
 
@@ -581,22 +586,22 @@ cudaError_t launch_attend(const AttendMaps& maps, int nc, const float* cbias,
                           const int32_t* sel, int k, const int32_t* q_perm,
                           const int32_t* q_offsets, int nqb, const int32_t* k_offsets, int nkb,
                           int H, int N, int d, void* out, int out_dtype, uint32_t* err,
-                          cudaStream_t s) {
-  const bool bs = bias_in_smem(nkb, k);
+                          cudaStream_t s, const int32_t* sel_count) {
+  const bool bs = bias_in_smem(nkb, sel_count ? 0 : k);
   const Fp8Scales none{nullptr, nullptr, nullptr, nullptr};
   if (d == 128)
-    return bs ? launch_attend_t<128, true, false>(maps, nc, cbias, sel, k, q_perm, q_offsets,
-                                                  nqb, k_offsets, nkb, H, N, out, out_dtype,
-                                                  err, none, s)
-              : launch_attend_t<128, false, false>(maps, nc, cbias, sel, k, q_perm, q_offsets,
-                                                   nqb, k_offsets, nkb, H, N, out, out_dtype,
-                                                   err, none, s);
-  return bs ? launch_attend_t<64, true, false>(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb,
-                                               k_offsets, nkb, H, N, out, out_dtype, err, none,
-                                               s)
-            : launch_attend_t<64, false, false>(maps, nc, cbias, sel, k, q_perm, q_offsets,
-                                                nqb, k_offsets, nkb, H, N, out, out_dtype, err,
-                                                none, s);
+    return bs ? launch_attend_t<128, true, false>(maps, nc, cbias, sel, k, sel_count, q_perm,
+                                                  q_offsets, nqb, k_offsets, nkb, H, N, out,
+                                                  out_dtype, err, none, s)
+              : launch_attend_t<128, false, false>(maps, nc, cbias, sel, k, sel_count, q_perm,
+                                                   q_offsets, nqb, k_offsets, nkb, H, N, out,
+                                                   out_dtype, err, none, s);
+  return bs ? launch_attend_t<64, true, false>(maps, nc, cbias, sel, k, sel_count, q_perm,
+                                               q_offsets, nqb, k_offsets, nkb, H, N, out,
+                                               out_dtype, err, none, s)
+            : launch_attend_t<64, false, false>(maps, nc, cbias, sel, k, sel_count, q_perm,
+                                                q_offsets, nqb, k_offsets, nkb, H, N, out,
+                                                out_dtype, err, none, s);
 }
 
 cudaError_t launch_attend_fp8(const AttendMaps& maps, const float* q_scale,
@@ -608,11 +613,12 @@ cudaError_t launch_attend_fp8(const AttendMaps& maps, const float* q_scale,
                               cudaStream_t s) {
   const Fp8Scales sc{q_scale, k_scale, kt_scale, kc_scale};
   return bias_in_smem(nkb, k)
-             ? launch_attend_t<128, true, true>(maps, nc, cbias, sel, k, q_perm, q_offsets, nqb,
-                                                k_offsets, nkb, H, N, out, out_dtype, err, sc, s)
-             : launch_attend_t<128, false, true>(maps, nc, cbias, sel, k, q_perm, q_offsets,
-                                                 nqb, k_offsets, nkb, H, N, out, out_dtype, err,
-                                                 sc, s);
+             ? launch_attend_t<128, true, true>(maps, nc, cbias, sel, k, nullptr, q_perm,
+                                                q_offsets, nqb, k_offsets, nkb, H, N, out,
+                                                out_dtype, err, sc, s)
+             : launch_attend_t<128, false, true>(maps, nc, cbias, sel, k, nullptr, q_perm,
+                                                 q_offsets, nqb, k_offsets, nkb, H, N, out,
+                                                 out_dtype, err, sc, s);
 }
 
 }  // namespace spark

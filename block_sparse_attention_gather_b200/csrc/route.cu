@@ -33,6 +33,10 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
 __device__ __forceinline__ float4 ld_nc_f4(const float4* p) {
   float4 v;
   asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -43,11 +47,19 @@ __device__ __forceinline__ float4 ld_nc_f4(const float4* p) {
 
 }  // namespace
 
-template <int D, int R>
+// kThreshold: Sol-Attn-style routing (the blog's "Discussion": block logits taken as roughly
+// Gaussian, the blocks above mu + tau*sigma exact) instead of the fixed Top-K budget.  Per row:
+// mu and the population sigma of the row's nkb scores (two passes, fp32; the positive factor
+// 1/sqrt(d) left out of the scores moves mu + tau*sigma with them), the count of scores strictly
+// above the threshold, capped at k (the largest kept, ties to the smaller block, as Top-K); the
+// selection is written to the first count entries of the row (rows are k apart) and the count
+// to count[h, A].
+template <int D, int R, bool kThreshold>
 __global__ void __launch_bounds__(kThreads, 1) route_kernel(const float* __restrict__ qbar_blocks,
                                                             const float* __restrict__ kbar,
-                                                            int nqb, int nkb, int k,
-                                                            int32_t* __restrict__ sel) {
+                                                            int nqb, int nkb, int k, float tau,
+                                                            int32_t* __restrict__ sel,
+                                                            int32_t* __restrict__ count) {
   static_assert(R % 4 == 0 && D % kChunk == 0, "tile shape");
   extern __shared__ __align__(16) float sm[];
   uint32_t* keys = reinterpret_cast<uint32_t*>(sm);     // [R][nkb]
@@ -136,9 +148,34 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(const float* __restr
   for (int r = warp; r < rows; r += kWarps) {
     const uint32_t* krow = keys + static_cast<size_t>(r) * nkb;
     int32_t* out = sel + (static_cast<size_t>(h) * nqb + A0 + r) * k;
+    int kr = k;                        // blocks this row takes
+    if constexpr (kThreshold) {
+      float sum = 0.f;
+      for (int B = lane; B < nkb; B += 32) sum += key_value(krow[B]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      const float mu = sum / static_cast<float>(nkb);
+      float ss = 0.f;
+      for (int B = lane; B < nkb; B += 32) {
+        const float dv = key_value(krow[B]) - mu;
+        ss = fmaf(dv, dv, ss);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      const float thr = fmaf(tau, sqrtf(ss / static_cast<float>(nkb)), mu);
+      const uint32_t tkey = order_key(thr);
+      int above = 0;
+      for (int B0 = 0; B0 < nkb; B0 += 32) {
+        const int B = B0 + lane;
+        above += __popc(__ballot_sync(0xffffffffu, B < nkb && krow[min(B, nkb - 1)] > tkey));
+      }
+      kr = min(above, k);
+      if (lane == 0) count[static_cast<size_t>(h) * nqb + A0 + r] = kr;
+      if (kr == 0) continue;           // uniform: nothing to write
+    }
     uint32_t prefix = 0, pmask = 0;
-    int need = k;                      // still to take among keys matching `prefix`
-    if (k < nkb) {
+    int need = kr;                     // still to take among keys matching `prefix`
+    if (kr < nkb) {
       for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = lane; i < 256; i += 32) wh[i] = 0;
         __syncwarp();
@@ -190,8 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(const float* __restr
       const int B = B0 + lane;
       const uint32_t u = (B < nkb) ? krow[B] : 0u;
       const bool valid = B < nkb;
-      const bool gt = valid && (k == nkb || u > T);
-      const bool eq = valid && k < nkb && u == T;
+      const bool gt = valid && (kr == nkb || u > T);
+      const bool eq = valid && kr < nkb && u == T;
       const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
       const int eq_rank = eq_seen + __popc(eqb & lt_mask);
       const bool take = gt || (eq && eq_rank < need);
@@ -210,33 +247,47 @@ constexpr size_t route_smem_bytes(int nkb) {
 
 constexpr size_t kRouteSmemLimit = 232448;   // 227 KB of opt-in shared memory per CTA
 
-template <int D, int R>
+template <int D, int R, bool kThreshold>
 static cudaError_t launch_route_t(const float* qbar_blocks, const float* kbar, int H, int nqb,
-                                  int nkb, int k, int32_t* sel, cudaStream_t s) {
+                                  int nkb, int k, float tau, int32_t* sel, int32_t* count,
+                                  cudaStream_t s) {
   const size_t smem = route_smem_bytes<D, R>(nkb);
-  cudaError_t e = cudaFuncSetAttribute(route_kernel<D, R>,
+  cudaError_t e = cudaFuncSetAttribute(route_kernel<D, R, kThreshold>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid((nqb + R - 1) / R, H);
-  route_kernel<D, R><<<grid, kThreads, smem, s>>>(qbar_blocks, kbar, nqb, nkb, k, sel);
+  route_kernel<D, R, kThreshold><<<grid, kThreads, smem, s>>>(qbar_blocks, kbar, nqb, nkb, k,
+                                                              tau, sel, count);
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool kThreshold>
 static cudaError_t launch_route_d(const float* qbar_blocks, const float* kbar, int H, int nqb,
-                                  int nkb, int k, int32_t* sel, cudaStream_t s) {
+                                  int nkb, int k, float tau, int32_t* sel, int32_t* count,
+                                  cudaStream_t s) {
   if (route_smem_bytes<D, 16>(nkb) <= kRouteSmemLimit)
-    return launch_route_t<D, 16>(qbar_blocks, kbar, H, nqb, nkb, k, sel, s);
+    return launch_route_t<D, 16, kThreshold>(qbar_blocks, kbar, H, nqb, nkb, k, tau, sel, count,
+                                             s);
   if (route_smem_bytes<D, 8>(nkb) <= kRouteSmemLimit)
-    return launch_route_t<D, 8>(qbar_blocks, kbar, H, nqb, nkb, k, sel, s);
-  return launch_route_t<D, 4>(qbar_blocks, kbar, H, nqb, nkb, k, sel, s);
+    return launch_route_t<D, 8, kThreshold>(qbar_blocks, kbar, H, nqb, nkb, k, tau, sel, count,
+                                            s);
+  return launch_route_t<D, 4, kThreshold>(qbar_blocks, kbar, H, nqb, nkb, k, tau, sel, count, s);
 }
 
 cudaError_t launch_route(const float* qbar_blocks, const float* kbar, int H, int nqb, int nkb,
                          int d, int k, int32_t* sel, uint32_t* /*err*/, cudaStream_t s) {
-  if (d == 128) return launch_route_d<128>(qbar_blocks, kbar, H, nqb, nkb, k, sel, s);
-  return launch_route_d<64>(qbar_blocks, kbar, H, nqb, nkb, k, sel, s);
+  if (d == 128)
+    return launch_route_d<128, false>(qbar_blocks, kbar, H, nqb, nkb, k, 0.f, sel, nullptr, s);
+  return launch_route_d<64, false>(qbar_blocks, kbar, H, nqb, nkb, k, 0.f, sel, nullptr, s);
+}
+
+cudaError_t launch_route_threshold(const float* qbar_blocks, const float* kbar, int H, int nqb,
+                                   int nkb, int d, float tau, int kcap, int32_t* sel,
+                                   int32_t* count, cudaStream_t s) {
+  if (d == 128)
+    return launch_route_d<128, true>(qbar_blocks, kbar, H, nqb, nkb, kcap, tau, sel, count, s);
+  return launch_route_d<64, true>(qbar_blocks, kbar, H, nqb, nkb, kcap, tau, sel, count, s);
 }
 
 }  // namespace spark

@@ -32,6 +32,12 @@ cudaError_t launch_gather_kv_meanpool(const void* K, const void* V, int dtype, i
 cudaError_t launch_route(const float* qbar_blocks, const float* kbar, int H, int nqb, int nkb,
                          int d, int k, int32_t* sel, uint32_t* err, cudaStream_t s);
 
+// Threshold routing: per (h, A) the blocks scoring above mu + tau*sigma of the row (at most
+// kcap, the largest), written ascending to the first count[h, A] entries of sel's row.
+cudaError_t launch_route_threshold(const float* qbar_blocks, const float* kbar, int H, int nqb,
+                                   int nkb, int d, float tau, int kcap, int32_t* sel,
+                                   int32_t* count, cudaStream_t s);
+
 // Context rows converted to bf16: dst[i] = bf16(src[i]) for n elements (a plain copy for
 // bf16 sources).
 cudaError_t launch_to_bf16(const void* src, int dtype, size_t n, void* dst, cudaStream_t s);
@@ -43,11 +49,13 @@ struct AttendMaps {
   CUtensorMap q, k, v, kt, vt, kc, vc;
 };
 
+// sel rows are k apart; sel_count (optional [H,nqb]) gives each query block its own number
+// of selected blocks (<= k), as threshold routing produces.
 cudaError_t launch_attend(const AttendMaps& maps, int nc, const float* cbias,
                           const int32_t* sel, int k, const int32_t* q_perm,
                           const int32_t* q_offsets, int nqb, const int32_t* k_offsets, int nkb,
                           int H, int N, int d, void* out, int out_dtype, uint32_t* err,
-                          cudaStream_t s);
+                          cudaStream_t s, const int32_t* sel_count = nullptr);
 
 // 3-D bf16 tensor map [H][rows][d], box 64 columns x 128 rows, 128-byte swizzle (api.cu).
 bool encode_rows_map(CUtensorMap* m, const void* base, int H, int rows, int d);

@@ -178,6 +178,30 @@ SPARK_API spark_status spark_bsa_gather_kv_meanpool(const void* K, const void* V
 SPARK_API spark_status spark_bsa_route(const float* qbar_blocks, const float* kbar, int H, int nqb,
                              int nkb, int d, int k, int32_t* sel, uint32_t* err, void* stream);
 
+/* Step 4 as Sol-Attn's content-adaptive routing, the comparator the blog's "Discussion"
+ * describes (block logits taken as roughly Gaussian; blocks above mu + tau*sigma are exact).
+ * Readings: mu and sigma are the mean and population standard deviation of the query block's
+ * nkb scores (fp32); "above" is strict; at most kcap blocks are kept (the largest, ties to the
+ * smaller B).  Writes the selection ascending to the first count[h,A] entries of row (h,A) of
+ * sel [H,nqb,kcap] (the rest of the row is untouched) and count [H,nqb] (0..kcap).
+ * kbar is d-major as written by spark_bsa_gather_kv_summarize. */
+SPARK_API spark_status spark_bsa_route_threshold(const float* qbar_blocks, const float* kbar,
+                                                 int H, int nqb, int nkb, int d, double tau,
+                                                 int kcap, int32_t* sel, int32_t* count,
+                                                 uint32_t* err, void* stream);
+
+/* Step 5 with a per-query-block selection count (as spark_bsa_route_threshold writes): sel
+ * rows are kcap apart and row (h,A) holds count[h,A] ascending block ids; the other blocks
+ * enter the compressed branch.  Otherwise as spark_bsa_attend. */
+SPARK_API spark_status spark_bsa_attend_var(const void* Qp, const void* Kp, const void* Vp,
+                                            const void* k_tilde, const void* v_tilde,
+                                            const float* cbias, const int32_t* sel, int kcap,
+                                            const int32_t* count, const int32_t* q_perm,
+                                            const int32_t* q_block_offsets, int nqb,
+                                            const int32_t* k_block_offsets, int nkb, int H,
+                                            int N, int d, void* out, int out_dtype,
+                                            uint32_t* err, void* stream);
+
 /* Step 5 (blog "Spark-Reblock" BSA equations with the Spark-Reweight summaries): the
  * two-branch attention of every (h, A), one online softmax over the exact rows of the
  * selected blocks and the summary rows (logit sigma q.k~_B + c_B) of the others, written to

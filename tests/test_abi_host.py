@@ -124,6 +124,22 @@ def test_step_entry_points_reject_bad_arguments(L):
     assert L.spark_bsa_read_error(None, None, ctypes.byref(flags)) == INVALID
 
 
+def test_threshold_entry_points_reject_bad_arguments(L):
+    p = ctypes.c_void_p(0x100000)
+    assert L.spark_bsa_route_threshold(p, p, 1, 4, 4, 128, 1.0, 5, p, p, None, None) == INVALID
+    assert L.spark_bsa_route_threshold(p, p, 1, 4, 4, 128, 1.0, 0, p, p, None, None) == INVALID
+    assert L.spark_bsa_route_threshold(p, p, 1, 4, 4, 128, float("nan"), 2, p, p, None,
+                                       None) == INVALID
+    assert L.spark_bsa_route_threshold(p, p, 1, 4, 4, 128, 1.0, 2, p, None, None,
+                                       None) == INVALID                          # count NULL
+    assert L.spark_bsa_route_threshold(p, p, 1, 4, 4, 96, 1.0, 2, p, p, None,
+                                       None) == UNSUPPORTED
+    assert L.spark_bsa_attend_var(p, p, p, p, p, p, p, 1, None, p, p, 1, p, 1, 1, 10, 128, p, 0,
+                                  None, None) == INVALID                         # count NULL
+    assert L.spark_bsa_attend_var(p, p, p, p, p, p, p, 2, p, p, p, 1, p, 1, 1, 10, 128, p, 0,
+                                  None, None) == INVALID                         # kcap > nkb
+
+
 def test_meanpool_entry_point_rejects_bad_arguments(L):
     p = ctypes.c_void_p(0x100000)
     assert L.spark_bsa_gather_kv_meanpool(p, p, 0, 1, 10, 128, p, p, 1, p, p, p, p, p, None,
