@@ -1,0 +1,57 @@
+"""The byte and FLOP models behind bench.py's numbers (no GPU): the algorithmic attention
+FLOPs count valid rows only, the dense-equivalent FLOPs are 4 H N (N + nc) d, the HBM byte
+models of the bandwidth-bound kernels match their closed forms, and the DRAM traffic of the
+committed ncu summary is reported only for the attention source it was taken on."""
+
+import json
+import types
+
+import torch
+
+import bench
+
+
+def fake_hotpath(q_sizes, k_sizes, sel, H=1, d=128, nc=0, dtype=torch.bfloat16):
+    qo = torch.tensor([0] + list(torch.tensor(q_sizes).cumsum(0).tolist()), dtype=torch.int32)
+    ko = torch.tensor([0] + list(torch.tensor(k_sizes).cumsum(0).tolist()), dtype=torch.int32)
+    N = int(qo[-1])
+    x = {"q_offsets": qo, "k_offsets": ko, "Q": torch.empty(H, N, d, dtype=dtype)}
+    hp = types.SimpleNamespace(x=x, v={"sel": torch.tensor(sel, dtype=torch.int32)}, H=H, N=N,
+                               d=d, nqb=len(q_sizes), nkb=len(k_sizes), k=len(sel[0][0]), nc=nc)
+    return hp
+
+
+def test_attention_flops_counts_valid_rows_only():
+    # 2 query blocks (3 and 5 rows), 3 key blocks (4, 2, 6 rows), k = 1, 7 context rows:
+    # A0 selects B2 -> 6 exact + 7 context + 2 summary rows; A1 selects B0 -> 4 + 7 + 2
+    hp = fake_hotpath([3, 5], [4, 2, 6], [[[2], [0]]], d=64, nc=7)
+    expect = 4 * 64 * (3 * (6 + 7 + 2) + 5 * (4 + 7 + 2))
+    assert bench.attention_flops(hp) == expect
+
+
+def test_dense_flops_closed_form():
+    w = types.SimpleNamespace(H=3, N=1000, nc=24, d=128)
+    assert bench.dense_flops(w) == 4.0 * 3 * 1000 * 1024 * 128
+
+
+def test_kernel_byte_models():
+    hp = fake_hotpath([64] * 4, [64] * 4, [[[0], [1], [2], [3]]], H=2, d=128, nc=10)
+    H, N, d, nqb, nkb, k = 2, 256, 128, 4, 4, 1
+    kb = bench.kernel_bytes(hp)
+    assert kb["gather_q"] == H * N * d * (2 + 2) + H * N * 4 + H * nqb * d * 4
+    assert kb["route"] == H * (nqb + nkb) * d * 4 + H * nqb * k * 4
+    assert kb["quantize"] == (2 * H * N * d + H * nkb * d + H * 10 * d) * 3
+
+
+def test_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
+    hp = fake_hotpath([64] * 4, [64] * 4, [[[0], [1], [2], [3]]], H=2)
+    src = bench.os.path.join(bench.ROOT, "block_sparse_attention_gather_b200", "csrc",
+                             "attention.cu")
+    prof = tmp_path / "dram.json"
+    prof.write_text(json.dumps({"attention_cu_sha256_16": bench.file_hash(src),
+                                "dram_bytes_per_query_block": 1000.0}))
+    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(prof))
+    assert bench.profiled_traffic(hp) == 1000.0 * 2 * 4
+    prof.write_text(json.dumps({"attention_cu_sha256_16": "0" * 16,
+                                "dram_bytes_per_query_block": 1000.0}))
+    assert bench.profiled_traffic(hp) is None
