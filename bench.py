@@ -56,6 +56,12 @@ def parse_args():
     ap.add_argument("--precision", choices=["bf16", "fp8"], default="bf16",
                     help="fp8: e4m3 logit product (queries, keys, summary and context keys "
                          "quantised per group after the routing), bf16 values")
+    ap.add_argument("--summaries", choices=["reweight", "meanpool"], default="reweight",
+                    help="meanpool: the baseline BSA compressed branch (comparator)")
+    ap.add_argument("--routing", choices=["topk", "threshold"], default="topk",
+                    help="threshold: mu + tau*sigma per query block, capped at the Top-K k "
+                         "(comparator)")
+    ap.add_argument("--tau", type=float, default=1.0)
     ap.add_argument("--op", choices=["attention", "reblock"], default="attention",
                     help="attention: the two-branch forward (default); reblock: the "
                          "Spark-Reblock partitioner on the same workload's Q and K")
@@ -129,7 +135,8 @@ class HotPath:
     """Preallocated buffers and the five step entry points of the C ABI, called with raw
     device pointers on one stream."""
 
-    def __init__(self, x, ratio, device, fp8=False):
+    def __init__(self, x, ratio, device, fp8=False, summaries="reweight", routing="topk",
+                 tau=1.0):
         from block_sparse_attention_gather_b200 import (lib, spark_bsa_workspace_layout,
                                                         workspace_views)
         self.L = lib()
@@ -170,6 +177,12 @@ class HotPath:
                 self.Kc8 = torch.empty(H, self.nc, d, dtype=u8, device=device)
                 self.kc_scale = torch.empty(H, (self.nc + 127) // 128, dtype=f32, device=device)
         self.kernels = KERNELS_FP8 if fp8 else KERNELS
+        # comparators: mean-pool summaries, threshold routing with per-row counts
+        self.summaries, self.routing, self.tau = summaries, routing, tau
+        if routing == "threshold":
+            if fp8 or self.nc:
+                raise SystemExit("threshold routing runs without fp8 and context here")
+            self.count = torch.empty(self.H, self.nqb, dtype=torch.int32, device=device)
 
     def _p(self, t):
         return ctypes.c_void_p(t.data_ptr())
@@ -189,12 +202,33 @@ class HotPath:
         st |= L.spark_bsa_anchor(p(v["qbar_blocks"]), p(x["q_offsets"]), H, N, d, nqb,
                                  p(v["qbar"]), s)
         rec(2)
-        st |= L.spark_bsa_gather_kv_summarize(p(x["K"]), p(x["V"]), self.dtype_code, H, N, d,
-                                              p(x["k_perm"]), p(x["k_offsets"]), nkb,
-                                              p(v["qbar"]), p(v["Kp"]), p(v["Vp"]), p(v["kbar"]),
-                                              p(v["k_tilde"]), p(v["v_tilde"]), p(v["cbias"]),
-                                              err, s)
+        if self.summaries == "meanpool":
+            st |= L.spark_bsa_gather_kv_meanpool(p(x["K"]), p(x["V"]), self.dtype_code, H, N, d,
+                                                 p(x["k_perm"]), p(x["k_offsets"]), nkb,
+                                                 p(v["Kp"]), p(v["Vp"]), p(v["kbar"]),
+                                                 p(v["k_tilde"]), p(v["v_tilde"]),
+                                                 p(v["cbias"]), err, s)
+        else:
+            st |= L.spark_bsa_gather_kv_summarize(p(x["K"]), p(x["V"]), self.dtype_code, H, N,
+                                                  d, p(x["k_perm"]), p(x["k_offsets"]), nkb,
+                                                  p(v["qbar"]), p(v["Kp"]), p(v["Vp"]),
+                                                  p(v["kbar"]), p(v["k_tilde"]), p(v["v_tilde"]),
+                                                  p(v["cbias"]), err, s)
         rec(3)
+        if self.routing == "threshold":
+            st |= L.spark_bsa_route_threshold(p(v["qbar_blocks"]), p(v["kbar"]), H, nqb, nkb, d,
+                                              float(self.tau), k, p(v["sel"]), p(self.count),
+                                              err, s)
+            rec(4)
+            st |= L.spark_bsa_attend_var(p(v["Qp"]), p(v["Kp"]), p(v["Vp"]), p(v["k_tilde"]),
+                                         p(v["v_tilde"]), p(v["cbias"]), p(v["sel"]), k,
+                                         p(self.count), p(x["q_perm"]), p(x["q_offsets"]), nqb,
+                                         p(x["k_offsets"]), nkb, H, N, d, p(self.out),
+                                         self.dtype_code, err, s)
+            rec(5)
+            if st != 0:
+                raise RuntimeError(f"a step entry point failed (status bits {st})")
+            return
         st |= L.spark_bsa_route(p(v["qbar_blocks"]), p(v["kbar"]), H, nqb, nkb, d, k,
                                 p(v["sel"]), err, s)
         rec(4)
@@ -250,8 +284,14 @@ def attention_flops(hp):
     qs = (qo[1:] - qo[:-1]).double()                    # [nqb]
     ks = (ko[1:] - ko[:-1]).double()                    # [nkb]
     sel = hp.v["sel"].long()                            # [H,nqb,k]
-    exact = ks[sel].sum(-1)                             # [H,nqb]
-    cols = exact + hp.nc + (hp.nkb - hp.k)
+    if getattr(hp, "routing", "topk") == "threshold":   # per-row counts
+        cnt = hp.count.long().to(sel.device)            # [H,nqb]
+        valid = torch.arange(sel.shape[-1], device=sel.device)[None, None, :] < cnt[..., None]
+        exact = (ks.to(sel.device)[sel.clamp(0, hp.nkb - 1)] * valid).sum(-1)
+        cols = (exact + hp.nc + (hp.nkb - cnt)).to(qs.device)
+    else:
+        exact = ks[sel].sum(-1)                         # [H,nqb]
+        cols = exact + hp.nc + (hp.nkb - hp.k)
     return float(4.0 * hp.d * (cols * qs[None, :]).sum().item())
 
 
@@ -556,7 +596,8 @@ def main():
     torch.cuda.set_device(device)
     w = WORKLOADS[args.workload]
     x = make_inputs(w, device=device)
-    hp = HotPath(x, w.ratio, device, fp8=args.precision == "fp8")
+    hp = HotPath(x, w.ratio, device, fp8=args.precision == "fp8", summaries=args.summaries,
+                 routing=args.routing, tau=args.tau)
     if hp.fp8 and hp.d != 128:
         raise SystemExit("--precision fp8 needs d = 128")
     peaks, peak_kind = load_peaks()
@@ -625,7 +666,8 @@ def main():
 
     # ---- end to end through the public call with host buffers (pinned), copies timed
     e2e = None
-    if args.e2e_steps > 0:
+    comparator = args.summaries != "reweight" or args.routing != "topk"
+    if args.e2e_steps > 0 and not comparator:      # the public calls run the method itself
         from block_sparse_attention_gather_b200 import (spark_bsa_forward, spark_bsa_forward_ctx,
                                                         spark_bsa_forward_fp8,
                                                         spark_bsa_forward_host,
@@ -716,7 +758,8 @@ def main():
         "dtype": "fp8-e4m3 logits, bf16 values" if hp.fp8 else "bf16", "data": "synthetic",
         "config": {"workload": w.name, "H": w.H, "N": w.N, "d": w.d, "topk_ratio": w.ratio,
                    "k": hp.k, "nqb": hp.nqb, "nkb": hp.nkb, "context_tokens": hp.nc,
-                   "block": w.block,
+                   "block": w.block, "summaries": args.summaries, "routing": args.routing,
+                   **({"tau": args.tau} if args.routing == "threshold" else {}),
                    "layout": w.layout, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (4.5 GB of Q/K/V per call), no flush"},
         "actual_tflops": att_flops / (ms_per_step / 1e3) / 1e12 * world,
@@ -732,7 +775,7 @@ def main():
         "e2e": e2e,
     }
     # the CPU leg times the bf16 oracle: it is reported for the bf16 line only
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not hp.fp8:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not hp.fp8 and not comparator:
         per_call, threads, desc = oracle_sample(w, n_heads=2, n_units=320)
         line["cpu_baseline"] = {"value": dflops / per_call / 1e12, "unit": UNIT,
                                 "cores": threads, "kind": "oracle", "sample": desc,

@@ -55,3 +55,12 @@ def test_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     prof.write_text(json.dumps({"attention_cu_sha256_16": "0" * 16,
                                 "dram_bytes_per_query_block": 1000.0}))
     assert bench.profiled_traffic(hp) is None
+
+
+def test_attention_flops_with_threshold_counts():
+    # kcap = 2; A0 keeps one block (B2: 6 rows), A1 none: the other blocks are summary rows
+    hp = fake_hotpath([3, 5], [4, 2, 6], [[[2, -1], [-1, -1]]], d=32)
+    hp.routing = "threshold"
+    hp.count = torch.tensor([[1, 0]], dtype=torch.int32)
+    expect = 4 * 32 * (3 * (6 + 2) + 5 * (0 + 3))
+    assert bench.attention_flops(hp) == expect
