@@ -203,7 +203,7 @@ SPARK_API spark_status spark_bsa_attend_var(const void* Qp, const void* Kp, cons
                                             uint32_t* err, void* stream);
 
 /* Step 5 (blog "Spark-Reblock" BSA equations with the Spark-Reweight summaries): the
- * two-branch attention of every (h, A), one online softmax over the exact rows of the
+ * two-branch attention of every (h, A), one row-wise softmax over the exact rows of the
  * selected blocks and the summary rows (logit sigma q.k~_B + c_B) of the others, written to
  * out[h, q_perm[h,i], :] (out dtype `out_dtype`).  Qp/Kp/Vp/k_tilde/v_tilde are bf16 and
  * must be 16-byte aligned; sel [H,nqb,k] ascending, distinct. */
