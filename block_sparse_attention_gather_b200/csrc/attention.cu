@@ -16,9 +16,10 @@
 //              cancels in the division, so no accuracy is lost as long as every p stays in
 //              floating-point range.  A row whose sum leaves [2^-60, 2^60] (a maximum far above
 //              the reference, e.g. a sink or context key 50 nats above the first blocks)
-//              makes its CTA repeat all tiles with that row's true maximum as the reference
-//              (a second pass over the same pipeline; each chunk whose sum is out of range
-//              records its maximum, which is within a few units of the row's).
+//              makes its CTA repeat all tiles (a second pass over the same pipeline): such
+//              rows take their recorded maximum as the reference - each chunk whose sum is out
+//              of range records its maximum, which is within a few units of the row's - and the
+//              other rows keep theirs.
 //   warp 8     TMA producer: the Q tile once, then K tiles (3-stage ring; a stage is free again
 //              once the S MMA that read it has completed, signalled by that S buffer's barrier).
 //   warp 9     TMA producer of V tiles (2-stage ring).
@@ -290,10 +291,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   const uint32_t tbase = *tmem_slot;
 
   // Pass 0 exponentiates every tile against a fixed reference per row (the larger of the two
-  // groups' first-tile maxima) and tracks the true row maximum.  A CTA with a row whose sum
-  // leaves [2^-60, 2^60] (a maximum far above the reference) runs pass 1 over the same tiles
-  // with the true maximum as the reference.  Barrier phases count tiles over both passes.
+  // groups' first-tile maxima) and records the maximum of every chunk whose sum is out of
+  // range.  A CTA with a row whose sum leaves [2^-60, 2^60] runs pass 1 over the same tiles;
+  // there the rows out of the window take their recorded maximum as the reference and the
+  // others keep pass 0's.  Barrier phases count tiles over both passes.
   float m_true = -INFINITY;                        // softmax threads: row maximum (log2 units)
+  float m_ref0 = 0.f;                              //   pass 0's reference of the row
+  bool rerun_row = false;                          //   the row left the window in pass 0
   int issued = 0;                                  // producers: loads issued over both passes
   for (int pass = 0; pass < 2; ++pass) {
     const int tg0 = pass * T;                      // tile counter of this pass's first tile
@@ -438,9 +442,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         named_bar_sync(1 + q4, 64);                      // the two groups of this quarter
         m_ref = fmaxf(ex_m[0][row], ex_m[1][row]);
       } else {
-        m_ref = m_true;                                  // both groups' maximum (epilogue)
+        // rows that left the window take the recorded maximum (both groups' maxima, merged in
+        // the epilogue); the others keep the reference that served them
+        m_ref = rerun_row ? m_true : m_ref0;
       }
       if (!(m_ref > -INFINITY)) m_ref = 0.f;
+      if (pass == 0) m_ref0 = m_ref;
       TileInfo next = tile_info<kFp8>(grp, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
       for (int t = grp; ok && t < T; t += 2) {
         const TileInfo ti = next;
@@ -493,8 +500,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         tc_fence_after_sync();
         const int qsize = max(0, min(q_offsets[A + 1] - qlo, kMaxBlock));
         // a sum outside the window means the reference was far from the row maximum
-        if (pass == 0 && row < qsize && !(l_tot >= 0x1p-60f && l_tot <= 0x1p60f))
+        if (pass == 0 && row < qsize && !(l_tot >= 0x1p-60f && l_tot <= 0x1p60f)) {
           s_rerun = 1;
+          rerun_row = true;
+        }
         const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
         int tok = -1;
         if (row < qsize) {

@@ -170,6 +170,36 @@ def test_logit_far_above_the_first_tiles():
         P.compare_out(P.to64(out[h]), O.dense_attention(q, k, v), "dense, far key")
 
 
+def test_rerun_keeps_the_reference_of_rows_in_window():
+    """One query block holds a row that leaves the window (a key ~100 nats above its first
+    tiles) and a row whose logits all sit near +100 nats, in window against its own first
+    tiles.  The repeat must give the first row its recorded maximum and leave the second row
+    its own reference (a reference of 0 there would overflow)."""
+    x = custom_inputs(76, H=1, N=1000, d=128, dtype="fp32", lo=100, hi=100)
+    g = torch.Generator().manual_seed(77)
+    u = torch.randn(128, generator=g, dtype=torch.float64)
+    u /= u.norm()
+    v = torch.randn(128, generator=g, dtype=torch.float64)
+    v -= (v @ u) * u
+    v /= v.norm()
+    Q = x["Q"].cpu().double()
+    K = x["K"].cpu().double()
+    K += 40.0 * u                                 # every key shares a large u component
+    r0, r1 = int(x["q_perm"][0, 0]), int(x["q_perm"][0, 1])   # rows of query block 0
+    Q[0, r0] = 6.0 * v + 0.1 * Q[0, r0]
+    Q[0, r1] = 30.0 * u + 0.1 * Q[0, r1]          # ~106 nats against every key
+    far = int(x["k_perm"][0, int(x["k_offsets"][-2])])
+    K[0, far] += 300.0 * v                        # ~160 nats for row r0 only
+    x = dict(x)
+    x["Q"], x["K"] = Q.float().to(DEV), K.float().to(DEV)
+    out, _ = check_forward(x, 1.0, check_inter=False)
+    q, k, vv = P.bf16_64(x["Q"][0]), P.bf16_64(x["K"][0]), P.bf16_64(x["V"][0])
+    ref = O.dense_attention(q, k, vv)
+    got = P.to64(out[0])
+    assert np.isfinite(got).all()
+    P.compare_out(got, ref, "rerun with rows in window")
+
+
 def test_logit_far_above_at_a_sparse_ratio():
     """The same planted key at ratio 0.1: it sits in the exact branch of the query blocks that
     select the last block and in the compressed branch (through k~, c) of the others."""
