@@ -62,6 +62,9 @@ def parse_args():
                     help="threshold: mu + tau*sigma per query block, capped at the Top-K k "
                          "(comparator)")
     ap.add_argument("--tau", type=float, default=1.0)
+    ap.add_argument("--reblock-steps", type=int, default=5,
+                    help="timed calls of the Spark-Reblock partitioner on the same Q and K, "
+                         "reported under the 'reblock' key after the timed steps (0: skip)")
     ap.add_argument("--op", choices=["attention", "reblock"], default="attention",
                     help="attention: the two-branch forward (default); reblock: the "
                          "Spark-Reblock partitioner on the same workload's Q and K")
@@ -295,6 +298,21 @@ def attention_flops(hp):
     return float(4.0 * hp.d * (cols * qs[None, :]).sum().item())
 
 
+def attention_issued_flops(hp):
+    """Tensor-core FLOPs the attention kernel issues, padding included: every key tile is a
+    128 x 128 box (M = 128 query rows, N = 128 keys) multiplied over d for S = Q K^T and again
+    for O += P V, so a (head, query block) with T tiles issues 4 * 128 * 128 * d * T whatever
+    the sizes of its blocks.  T = selected blocks + context tiles + summary tiles."""
+    nct = -(-hp.nkb // 128)
+    nxt = -(-hp.nc // 128)
+    if getattr(hp, "routing", "topk") == "threshold":
+        cnt = hp.count.long().cpu()
+        tiles = (cnt + nxt + torch.where(cnt < hp.nkb, nct, 0)).sum().item()
+    else:
+        tiles = hp.H * hp.nqb * (hp.k + nxt + (nct if hp.k < hp.nkb else 0))
+    return 4.0 * 128 * 128 * hp.d * float(tiles)
+
+
 def kernel_bytes(hp):
     """Algorithmic HBM bytes per launch of the four bandwidth-bound kernels."""
     H, N, d, nqb, nkb, k = hp.H, hp.N, hp.d, hp.nqb, hp.nkb, hp.k
@@ -421,16 +439,22 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     w = WORKLOADS[args.workload]
-    times = []
+    times, walls = [], []
     for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         per_call, threads, desc = oracle_sample(w, n_heads=1, n_units=4, seed=i)
         if i >= args.warmup:
             times.append(per_call)
+            walls.append(time.perf_counter() - t0)
     t = statistics.mean(times)
+    # each step does a bounded sample of one call's work (the share wall/t of it, by the linear
+    # extrapolation), so the rate is one call's dense-equivalent work over the extrapolated
+    # call time; ms_per_step is the wall time a step actually took
     value = dense_flops(w) / t / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(walls) * 1e3,
+        "ms_per_call_extrapolated": t * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": w.name, "H": w.H, "N": w.N, "d": w.d, "topk_ratio": w.ratio,
@@ -480,17 +504,12 @@ def reblock_bytes_flops(H, N, d, block, e_in, power_iters=4, moment_min_node=256
     return flops, prep_bytes, level_bytes
 
 
-def run_reblock(args, world, rank, local):
+def measure_reblock(Q, K, block, steps, warmup, world, device, sample_clocks=True):
+    """Times the Spark-Reblock partitioner (q_reuse_k) on Q, K: `warmup` untimed calls, then
+    `steps` calls bracketed by CUDA events on the launching stream (max over ranks), then the
+    whitening steps alone the same way; returns a dict of the figures."""
     from block_sparse_attention_gather_b200 import (lib, spark_reblock_workspace_layout)
-    from block_sparse_attention_gather_b200.workloads import WORKLOADS, make_inputs
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    w = WORKLOADS[args.workload]
-    x = make_inputs(w, device=device)
-    Q, K = x["Q"], x["K"]
-    del x
     H, N, d = Q.shape
-    block = w.block
     L = lib()
     lay = spark_reblock_workspace_layout(H, N, d, block)
     ws = torch.empty(lay.total, dtype=torch.uint8, device=device)
@@ -513,34 +532,54 @@ def run_reblock(args, world, rank, local):
         if st != 0:
             raise RuntimeError(f"spark_reblock_whiten failed with status {st}")
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         call()
     torch.cuda.synchronize()
-    peaks, peak_kind = load_peaks()
-    clocks = ClockSampler(device)
+    clocks = ClockSampler(device) if sample_clocks else None
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     ev[0].record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         call()
     ev[1].record(stream)
     torch.cuda.synchronize()
-    clock_info = clocks.stop()
+    clock_info = clocks.stop() if clocks else None
     total_ms = max_over_ranks(ev[0].elapsed_time(ev[1]), world, device)
-    ms = total_ms / args.steps
-    # the whitening steps alone (same kernels as inside the call)
+    ms = total_ms / steps
     pe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     pe[0].record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         prep()
     pe[1].record(stream)
     torch.cuda.synchronize()
-    prep_ms = pe[0].elapsed_time(pe[1]) / args.steps
+    prep_ms = max_over_ranks(pe[0].elapsed_time(pe[1]), world, device) / steps
     part_ms = ms - prep_ms
     flops, prep_bytes, level_bytes = reblock_bytes_flops(H, N, d, block, Q.element_size())
+    del ws, qp, kp, offs
+    return {"ms": ms, "prep_ms": prep_ms, "levels_ms": part_ms, "flops": flops,
+            "prep_bytes": prep_bytes, "level_bytes": level_bytes, "levels": lay.levels,
+            "clocks": clock_info,
+            "launches_per_call": 6 + sum(11 + (2 if (d == 128 and m >= 256) else 8)
+                                         for m in reblock_level_min_nodes(N, block))}
+
+
+def run_reblock(args, world, rank, local):
+    from block_sparse_attention_gather_b200.workloads import WORKLOADS, make_inputs
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w, device=device)
+    Q, K = x["Q"], x["K"]
+    del x
+    H, N, d = Q.shape
+    block = w.block
+    peaks, peak_kind = load_peaks()
+    r = measure_reblock(Q, K, block, args.steps, args.warmup, world, device)
+    ms, prep_ms, part_ms = r["ms"], r["prep_ms"], r["levels_ms"]
+    flops, prep_bytes, level_bytes = r["flops"], r["prep_bytes"], r["level_bytes"]
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     gbs = level_bytes / (part_ms / 1e3) / 1e9
     line = {
@@ -549,7 +588,7 @@ def run_reblock(args, world, rank, local):
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if Q.dtype == torch.bfloat16 else "f32", "data": "synthetic",
         "config": {"workload": w.name, "H": H, "N": N, "d": d, "block": block,
-                   "levels": lay.levels, "mode": "q_reuse_k", "power_iters": 4,
+                   "levels": r["levels"], "mode": "q_reuse_k", "power_iters": 4,
                    "l2": "inputs larger than L2, no flush"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
                      "frac": gbs / hbm, "traffic": None,
@@ -564,9 +603,8 @@ def run_reblock(args, world, rank, local):
                     "levels": {"ms": part_ms, "GB/s": gbs, "bytes": level_bytes}},
         # per call: 4 whitening kernels, the identity order, offsets, and per level 11
         # selection/scatter kernels plus 8 power-pass kernels or 2 node-moment kernels
-        "gpu_launches": (6 + sum(11 + (2 if (d == 128 and m >= 256) else 8)
-                                 for m in reblock_level_min_nodes(N, block))) * args.steps,
-        "clocks": clock_info,
+        "gpu_launches": r["launches_per_call"] * args.steps,
+        "clocks": r["clocks"],
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -641,6 +679,7 @@ def main():
         raise RuntimeError(f"device error word {flags:#x} after the timed region")
 
     att_flops = attention_flops(hp)
+    issued_flops = attention_issued_flops(hp)
     att_ms = statistics.mean(per_kernel["attend"])
     achieved = att_flops / (att_ms / 1e3) / 1e12
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
@@ -661,7 +700,11 @@ def main():
             gbs = kb[n] / (ms / 1e3) / 1e9
             entry.update({"bytes": kb[n], "GB/s": gbs, "hbm_frac": gbs / hbm_peak})
         else:
-            entry.update({"flops": att_flops, "TFLOP/s": achieved, "tensor_frac": achieved / peak})
+            issued = issued_flops / (ms / 1e3) / 1e12
+            entry.update({"flops": att_flops, "TFLOP/s": achieved, "tensor_frac": achieved / peak,
+                          "issued_flops": issued_flops, "issued_TFLOP/s": issued,
+                          "issued_tensor_frac": issued / peak,
+                          "valid_share_of_issued": att_flops / issued_flops})
         kernels[n] = entry
 
     # ---- end to end through the public call with host buffers (pinned), copies timed
@@ -750,6 +793,18 @@ def main():
         if hp.fp8:
             del ws8
 
+    # ---- the partitioner upstream of the path, on the same Q and K (its own timed calls)
+    reblock = None
+    if args.reblock_steps > 0 and not comparator and not hp.fp8 and not hp.nc:
+        r = measure_reblock(x["Q"], x["K"], w.block, args.reblock_steps, 2, world, device,
+                            sample_clocks=False)
+        gbs = r["level_bytes"] / (r["levels_ms"] / 1e3) / 1e9
+        reblock = {"ms_per_call": r["ms"], "whiten_ms": r["prep_ms"],
+                   "levels_ms": r["levels_ms"], "levels_GB/s": gbs,
+                   "levels_hbm_frac": gbs / hbm_peak, "levels_bytes": r["level_bytes"],
+                   "steps": args.reblock_steps, "mode": "q_reuse_k", "block": w.block,
+                   "note": "separate timed calls after the timed steps; not part of value"}
+
     traffic = profiled_traffic(hp)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -767,12 +822,16 @@ def main():
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_kind": peak_note,
                      "kernel": "attend (tcgen05 two-branch attention)",
-                     "algorithmic_flops_per_launch": att_flops},
+                     "algorithmic_flops_per_launch": att_flops,
+                     "frac_of_burst": achieved / peaks.get("bf16_tflops",
+                                                           FALLBACK_PEAKS["bf16_tflops"]) *
+                                      (0.75 if hp.fp8 else 1.0)},
         "kernels": kernels,
         "gpu_launches": (5 + (2 if hp.convert_ctx else 0) +
                          ((4 if hp.nc else 3) if hp.fp8 else 0)) * args.steps,
         "clocks": clock_info,
         "e2e": e2e,
+        "reblock": reblock,
     }
     # the CPU leg times the bf16 oracle: it is reported for the bf16 line only
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not hp.fp8 and not comparator:

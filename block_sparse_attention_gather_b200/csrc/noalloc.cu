@@ -7,12 +7,15 @@
 // work into a CUDA stream capture (where cudaMalloc is not allowed), or an inference plugin
 // invoked from a real-time path where an allocation could block or fail.  For them the
 // caller-sized workspace of spark_bsa_forward is not an option, so this entry point uses a
-// file-scope __device__ array instead.  The array is part of this file's module: every GPU on
-// which the library is used this way holds it until the process exits.
+// file-scope __device__ array instead.  The array is part of this file's module: it is reserved
+// on every GPU where the module loads (first use under lazy loading, context creation under
+// eager loading) and held until the process exits.
 //
 // The set-up (resolving the array's device address with cudaGetSymbolAddress) runs once per
 // device, on the first call made while that device is current; the host-side name of the
-// array is only a stand-in and must never be handed to a kernel.
+// array is only a stand-in and must never be handed to a kernel.  The cached address does not
+// survive a device reset (cudaDeviceReset tears the context down and the module reloads
+// elsewhere); the header states that calls after one are not supported.
 #include <mutex>
 
 #include "../../include/spark_bsa.h"

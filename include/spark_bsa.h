@@ -425,7 +425,13 @@ SPARK_API spark_status spark_reblock_level(int H, int N, int d, int block, int l
  *     with SPARK_ERR_WORKSPACE before anything is launched.
  *   - The first call on a device (with that device current) resolves the array's device
  *     address; make that first call before any stream capture.
- *   - Every GPU on which this entry point is used holds the array until the process exits.
+ *   - The array is reserved on a device when the library's module is loaded there: on the
+ *     first use of the library on that device under CUDA's lazy module loading (the default),
+ *     at context creation under eager loading (CUDA_MODULE_LOADING=EAGER).  It is held until
+ *     the process exits.
+ *   - The device address is resolved once per device and cached.  A device reset
+ *     (cudaDeviceReset) or any other teardown of the device's context makes the cached address
+ *     stale; calling this entry point after one is not supported.
  *   - All calls share the one array and it keeps the last call's contents; the call clears
  *     the error word itself.  Calls that overlap on the GPU (two streams, or two host threads)
  *     race on the array: serialise them.
