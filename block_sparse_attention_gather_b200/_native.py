@@ -27,6 +27,7 @@ __all__ = [
     "spark_bsa_host_staging_size", "spark_bsa_forward_host", "spark_bsa_quantize_fp8",
     "spark_bsa_attend_fp8", "spark_bsa_workspace_size_fp8", "spark_bsa_forward_fp8",
     "spark_bsa_gather_kv_meanpool", "spark_bsa_route_threshold", "spark_bsa_attend_var",
+    "spark_bsa_set_wait_limit_ns", "spark_bsa_get_wait_limit_ns",
 ]
 
 SPARK_BF16, SPARK_F32 = 0, 1
@@ -42,6 +43,7 @@ EXPORTED = [
     "spark_bsa_host_staging_size", "spark_bsa_forward_host", "spark_bsa_quantize_fp8",
     "spark_bsa_attend_fp8", "spark_bsa_workspace_size_fp8", "spark_bsa_forward_fp8",
     "spark_bsa_gather_kv_meanpool", "spark_bsa_route_threshold", "spark_bsa_attend_var",
+    "spark_bsa_set_wait_limit_ns", "spark_bsa_get_wait_limit_ns",
 ]
 REBLOCK_MODES = {"q_reuse_k": 0, "separate": 1}
 
@@ -83,6 +85,8 @@ def lib():
     sig = {
         "spark_status_string": (ctypes.c_char_p, [_I]),
         "spark_bsa_topk_count": (_I, [_I, _D]),
+        "spark_bsa_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+        "spark_bsa_get_wait_limit_ns": (ctypes.c_uint64, []),
         "spark_bsa_workspace_layout": (_I, [_I, _I, _I, _I, _I, _D, ctypes.POINTER(Layout)]),
         "spark_bsa_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _D]),
         "spark_bsa_forward": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _I, _D, _P,
@@ -178,6 +182,15 @@ def spark_status_string(status: int) -> str:
 
 def spark_bsa_topk_count(nkb: int, topk_ratio: float) -> int:
     return int(lib().spark_bsa_topk_count(int(nkb), float(topk_ratio)))
+
+
+def spark_bsa_set_wait_limit_ns(limit_ns: int) -> None:
+    """Process-wide limit of the kernels' bounded waits (nanoseconds; default 4e9)."""
+    lib().spark_bsa_set_wait_limit_ns(int(limit_ns))
+
+
+def spark_bsa_get_wait_limit_ns() -> int:
+    return int(lib().spark_bsa_get_wait_limit_ns())
 
 
 def spark_bsa_workspace_layout(H, N, d, nqb, nkb, topk_ratio) -> Layout:

@@ -2,6 +2,7 @@
 // descriptor encoding and the launch sequence of the forward pass.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
@@ -57,6 +58,11 @@ bool encode_rows_map_u8(CUtensorMap* m, const void* base, int H, int rows, int d
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+// Process-wide limit of the kernels' bounded waits (nanoseconds), read at each launch.
+static std::atomic<uint64_t> g_wait_limit_ns{kWaitLimitNs};
+
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 }  // namespace spark
 
@@ -307,6 +313,12 @@ const char* spark_status_string(int status) {
 }
 
 int spark_bsa_topk_count(int nkb, double topk_ratio) { return topk_count(nkb, topk_ratio); }
+
+void spark_bsa_set_wait_limit_ns(uint64_t limit_ns) {
+  g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+}
+
+uint64_t spark_bsa_get_wait_limit_ns(void) { return wait_limit_ns(); }
 
 spark_status spark_bsa_workspace_layout(int H, int N, int d, int nqb, int nkb,
                                         double topk_ratio, spark_bsa_layout* layout) {

@@ -39,8 +39,9 @@
 // TMEM columns (512 allocated, one CTA per SM): S/P buffers [0,128), [128,256), [256,384),
 // O [384,384+D).
 //
-// Every wait is bounded (spark_ptx.cuh); on expiry the kernel flags kErrTimeout, stops every
-// role, drains the copies and MMAs it issued, frees TMEM and returns.
+// Every wait is bounded by the launch parameter wait_ns (the library's process-wide setting,
+// 4 s by default); on expiry the kernel flags kErrTimeout, stops every role, drains the copies
+// and MMAs it issued (waits bounded by the default limit), frees TMEM and returns.
 #include "spark_kernels.cuh"
 
 namespace spark {
@@ -208,7 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     const int32_t* __restrict__ sel, int kcap, const int32_t* __restrict__ sel_count,
     const int32_t* __restrict__ q_perm,
     const int32_t* __restrict__ q_offsets, int nqb, const int32_t* __restrict__ k_offsets,
-    int nkb, int N, void* __restrict__ out, int out_dtype, uint32_t* err, const Fp8Scales sc) {
+    int nkb, int N, void* __restrict__ out, int out_dtype, uint32_t* err, const Fp8Scales sc,
+    uint64_t wait_ns) {
   static_assert(!kFp8 || D == 128, "FP8 logits: d = 128 (one 128-byte row per key)");
   constexpr int QK_BYTES = 128 * D * (kFp8 ? 1 : 2);   // one Q or K tile
   constexpr int V_BYTES = 128 * D * 2;                 // one V tile (bf16)
@@ -336,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           const int tg = tg0 + t;
           const int s = tg % stages;
           const TileInfo ti = next;
-          if (tg >= stages && !mbar_wait(&empty[s], ((tg / stages) - 1) & 1, abort_flag, err))
+          if (tg >= stages && !mbar_wait(&empty[s], ((tg / stages) - 1) & 1, abort_flag, err, wait_ns))
             break;
           mbar_arrive_expect_tx(&full[s], tile_bytes);
           const CUtensorMap* map = ti.src == kSrcVideo ? mx : (ti.src == kSrcContext ? mc : ms);
@@ -362,12 +364,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         const uint64_t qd = sdesc_sw128(smem_u32(qst), 16, 1024);
         const uint64_t kdesc0 = sdesc_sw128(smem_u32(kst), 16, 1024);
         const uint64_t vdesc0 = sdesc_sw128(smem_u32(vst), 16384, 1024);
-        bool ok = pass > 0 || mbar_wait(&bars->qfull, 0, abort_flag, err);
+        bool ok = pass > 0 || mbar_wait(&bars->qfull, 0, abort_flag, err, wait_ns);
         // S(t) of this pass into buffer (tg0 + t) % 3
         auto issue_s = [&](int t) -> bool {
           const int tg = tg0 + t;
           const int s = tg % kKStages;
-          if (!mbar_wait(&bars->kfull[s], (tg / kKStages) & 1, abort_flag, err)) return false;
+          if (!mbar_wait(&bars->kfull[s], (tg / kKStages) & 1, abort_flag, err, wait_ns)) return false;
           const uint32_t dcol = tbase + (tg % 3) * 128;
           const uint64_t kd = kdesc0 + static_cast<uint64_t>(s * (QK_BYTES >> 4));
           if constexpr (kFp8) {
@@ -388,10 +390,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         for (int t = 0; ok && t < min(T, 3); ++t) ok = issue_s(t);
         for (int t = 0; ok && t < T; ++t) {
           const int tg = tg0 + t;
-          if (!mbar_wait(&bars->pready[tg % 3], (tg / 3) & 1, abort_flag, err)) break;
+          if (!mbar_wait(&bars->pready[tg % 3], (tg / 3) & 1, abort_flag, err, wait_ns)) break;
           tc_fence_after_sync();
           const int s = tg % kVStages;
-          if (!mbar_wait(&bars->vfull[s], (tg / kVStages) & 1, abort_flag, err)) break;
+          if (!mbar_wait(&bars->vfull[s], (tg / kVStages) & 1, abort_flag, err, wait_ns)) break;
           const uint64_t vd = vdesc0 + static_cast<uint64_t>(s * (V_BYTES >> 4));
           const uint32_t pcol = tbase + (tg % 3) * 128;               // P(t) over S(t)
 #pragma unroll
@@ -427,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           const TileInfo ti = tile_info<kFp8>(grp, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
           const float tsl = scale_log2 * ti.ks;
           ok = __all_sync(0xffffffffu,
-                          mbar_wait(&bars->sfull[tg % 3], (tg / 3) & 1, abort_flag, err));
+                          mbar_wait(&bars->sfull[tg % 3], (tg / 3) & 1, abort_flag, err, wait_ns));
           if (ok) {
             tc_fence_after_sync();
             const uint32_t sbuf = tbase + lane_off + (tg % 3) * 128;
@@ -454,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         const int tg = tg0 + t;
         const int b = tg % 3;
         if (pass > 0 || t >= 2) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&bars->sfull[b], (tg / 3) & 1, abort_flag, err));
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars->sfull[b], (tg / 3) & 1, abort_flag, err, wait_ns));
           if (!ok) break;
           tc_fence_after_sync();
         }
@@ -490,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       }
       // ---- epilogue: O / (l_0 + l_1), scattered to the original token order
       bool fine = ok && T > 0;
-      if (fine) fine = __all_sync(0xffffffffu, mbar_wait(&bars->done, pass, abort_flag, err));
+      if (fine) fine = __all_sync(0xffffffffu, mbar_wait(&bars->done, pass, abort_flag, err, wait_ns));
       ex_l[grp][row] = l_run;
       ex_mt[grp][row] = m_true;
       named_bar_sync(1 + q4, 64);
@@ -587,7 +589,7 @@ static cudaError_t launch_attend_t(const AttendMaps& m, int nc, const float* cbi
   dim3 grid(nqb, H);
   attend_kernel<D, kBiasSmem, kFp8><<<grid, kThreads, smem, s>>>(
       m.q, m.k, m.v, m.kt, m.vt, m.kc, m.vc, nc, cbias, sel, k, sel_count, q_perm, q_offsets,
-      nqb, k_offsets, nkb, N, out, out_dtype, err, sc);
+      nqb, k_offsets, nkb, N, out, out_dtype, err, sc, wait_limit_ns());
   return cudaGetLastError();
 }
 

@@ -256,7 +256,8 @@ __device__ __forceinline__ bool rb_wait_quiet(uint64_t* bar, uint32_t parity) {
 // MN-major from the same shared-memory tile; the 128 x 128 fp32 sum stays in TMEM.
 __global__ void __launch_bounds__(128) rb_moment_tc_kernel(const __grid_constant__ CUtensorMap map_y,
                                                            int tiles, float* __restrict__ part,
-                                                           uint32_t* __restrict__ err) {
+                                                           uint32_t* __restrict__ err,
+                                                           uint64_t wait_ns) {
   extern __shared__ uint8_t rb_tc_raw[];
   uint8_t* st = align1024(rb_tc_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(st + kMomStages * kTcTile);
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(128) rb_moment_tc_kernel(const __grid_constant
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int s = t % kMomStages;
-      if (!mbar_wait(&full[s], (t / kMomStages) & 1, abort_flag, err)) { ok = false; break; }
+      if (!mbar_wait(&full[s], (t / kMomStages) & 1, abort_flag, err, wait_ns)) { ok = false; break; }
       tc_fence_after_sync();
       const uint64_t d0 = sdesc_sw128(smem_u32(st + s * kTcTile), 16384, 1024);
 #pragma unroll
@@ -309,7 +310,7 @@ __global__ void __launch_bounds__(128) rb_moment_tc_kernel(const __grid_constant
       }
       tc_commit(&empty[s]);
       if (t + kMomStages < T) {
-        if (!mbar_wait(&empty[s], (t / kMomStages) & 1, abort_flag, err)) { ok = false; break; }
+        if (!mbar_wait(&empty[s], (t / kMomStages) & 1, abort_flag, err, wait_ns)) { ok = false; break; }
         load(t + kMomStages);
       }
     }
@@ -352,7 +353,8 @@ __global__ void __launch_bounds__(160) rb_whiten_tc_kernel(const __grid_constant
                                                            const __grid_constant__ CUtensorMap map_w,
                                                            int N, int tiles,
                                                            __nv_bfloat16* __restrict__ X,
-                                                           uint32_t* __restrict__ err) {
+                                                           uint32_t* __restrict__ err,
+                                                           uint64_t wait_ns) {
   extern __shared__ uint8_t rb_tc_raw[];
   uint8_t* wst = align1024(rb_tc_raw);
   uint8_t* yst = wst + kTcTile;                          // 2 stages
@@ -404,12 +406,12 @@ __global__ void __launch_bounds__(160) rb_whiten_tc_kernel(const __grid_constant
         issued = t + 1;
       };
       for (int t = 0; t < min(T, 2); ++t) load(t);
-      bool ok = mbar_wait(wfull, 0, abort_flag, err);
+      bool ok = mbar_wait(wfull, 0, abort_flag, err, wait_ns);
       const uint64_t wd = sdesc_sw128(smem_u32(wst), 16, 1024);
       for (int t = 0; ok && t < T; ++t) {
         const int s = t & 1;
-        if (!mbar_wait(&yfull[s], (t >> 1) & 1, abort_flag, err)) { ok = false; break; }
-        if (t >= 2 && !mbar_wait(&accempty[s], ((t >> 1) - 1) & 1, abort_flag, err)) {
+        if (!mbar_wait(&yfull[s], (t >> 1) & 1, abort_flag, err, wait_ns)) { ok = false; break; }
+        if (t >= 2 && !mbar_wait(&accempty[s], ((t >> 1) - 1) & 1, abort_flag, err, wait_ns)) {
           ok = false;
           break;
         }
@@ -423,7 +425,7 @@ __global__ void __launch_bounds__(160) rb_whiten_tc_kernel(const __grid_constant
         tc_commit(&accfull[s]);
         tc_commit(&yempty[s]);
         if (t + 2 < T) {
-          if (!mbar_wait(&yempty[s], (t >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          if (!mbar_wait(&yempty[s], (t >> 1) & 1, abort_flag, err, wait_ns)) { ok = false; break; }
           load(t + 2);
         }
       }
@@ -438,7 +440,7 @@ __global__ void __launch_bounds__(160) rb_whiten_tc_kernel(const __grid_constant
     const int row = tid;                                 // TMEM lane = token row of the tile
     for (int t = 0; t < T; ++t) {
       const int b = t & 1;
-      const bool got = __all_sync(0xffffffffu, mbar_wait(&accfull[b], (t >> 1) & 1, abort_flag, err));
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&accfull[b], (t >> 1) & 1, abort_flag, err, wait_ns));
       if (!got) break;
       tc_fence_after_sync();
       float v[128];
@@ -959,7 +961,8 @@ __global__ void __launch_bounds__(128) rb_cov_tc_kernel(const __nv_bfloat16* __r
                                                         const int32_t* __restrict__ perm, int N,
                                                         const int4* __restrict__ cchunks,
                                                         int ncch, float* __restrict__ cpart,
-                                                        uint32_t* __restrict__ err) {
+                                                        uint32_t* __restrict__ err,
+                                                        uint64_t wait_ns) {
   extern __shared__ uint8_t rb_tc_raw[];
   uint8_t* st = align1024(rb_tc_raw);                    // 2 stages x 32 KB
   uint64_t* mdone = reinterpret_cast<uint64_t*>(st + 2 * kTcTile);   // [2]
@@ -1043,7 +1046,7 @@ __global__ void __launch_bounds__(128) rb_cov_tc_kernel(const __nv_bfloat16* __r
     if (t + 1 < T) {
       // stage s^1 held tile t-1: its MMAs must be done before it is overwritten
       if (t >= 1)
-        ok = __syncthreads_and(mbar_wait(&mdone[s ^ 1], ((t - 1) >> 1) & 1, abort_flag, err));
+        ok = __syncthreads_and(mbar_wait(&mdone[s ^ 1], ((t - 1) >> 1) & 1, abort_flag, err, wait_ns));
       if (!ok) break;
       issue_tile(t + 1);
     }
@@ -1272,7 +1275,7 @@ static cudaError_t whiten_t(const void* Xin, const void* Yin, int H, int N, uint
     e = cudaFuncSetAttribute(rb_moment_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    rb_moment_tc_kernel<<<dim3(kMomentTcParts, H), 128, smem, s>>>(map_y, tiles, part, err);
+    rb_moment_tc_kernel<<<dim3(kMomentTcParts, H), 128, smem, s>>>(map_y, tiles, part, err, wait_limit_ns());
     rb_moment_reduce_kernel<D><<<H, kRbThreads, 0, s>>>(part, kMomentTcParts, N, M);
   } else {
     rb_moment_partial_kernel<D, T><<<dim3(kMomentParts, H), kRbThreads, 0, s>>>(
@@ -1290,7 +1293,7 @@ static cudaError_t whiten_t(const void* Xin, const void* Yin, int H, int N, uint
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const int ctas = (tiles + kWhitenTcTiles - 1) / kWhitenTcTiles;
-    rb_whiten_tc_kernel<<<dim3(ctas, H), 160, smem, s>>>(map_x, map_w, N, tiles, X, err);
+    rb_whiten_tc_kernel<<<dim3(ctas, H), 160, smem, s>>>(map_x, map_w, N, tiles, X, err, wait_limit_ns());
   } else {
     const size_t wh_smem = (D * D + kRbWarps * 8 * D) * sizeof(float);
     e = cudaFuncSetAttribute(rb_whiten_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1359,7 +1362,7 @@ static cudaError_t level_t(int H, int N, int block, int level, const int32_t* pe
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     rb_cov_tc_kernel<<<dim3(lm.ncch, H), 128, smem, s>>>(X, perm_in, N, cchunks, lm.ncch, cpart,
-                                                         err);
+                                                         err, wait_limit_ns());
     const size_t nsmem = 128 * 128 * 4;
     e = cudaFuncSetAttribute(rb_cov_node_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(nsmem));

@@ -8,6 +8,10 @@ namespace spark {
 constexpr int kMaxBlock = 128;     // tokens per block (one MMA tile of keys / queries)
 constexpr int kMaxNkb = 12800;     // key blocks per head accepted by the routing kernel
 
+// Limit of every bounded wait in the kernels launched from now on (nanoseconds): the
+// process-wide setting of spark_bsa_set_wait_limit_ns, kWaitLimitNs by default (api.cu).
+uint64_t wait_limit_ns();
+
 cudaError_t launch_gather_q(const void* Q, int dtype, int H, int N, int d,
                             const int32_t* q_perm, const int32_t* q_offsets, int nqb, void* Qp,
                             float* qbar_blocks, uint32_t* err, cudaStream_t s);

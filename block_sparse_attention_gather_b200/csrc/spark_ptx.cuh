@@ -19,7 +19,9 @@ constexpr uint32_t kErrOffsets = 0x2u;
 constexpr uint32_t kErrSel = 0x4u;
 constexpr uint32_t kErrTimeout = 0x8u;
 
-// Upper bound of any single wait inside a kernel (nanoseconds of %globaltimer).
+// Default upper bound of a single wait inside a kernel (nanoseconds of %globaltimer).  The
+// kernels with waits take the bound as a launch parameter (the library's process-wide setting,
+// this value unless the caller changed it); the drains after an abort always use this value.
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
 __device__ __forceinline__ void flag_error(uint32_t* err, uint32_t bits) {
@@ -89,26 +91,27 @@ __device__ __forceinline__ bool launch_timed_out(const uint32_t* err) {
 }
 
 // Waits for the phase of `bar` with parity `parity` to complete.  Gives up when the CTA's
-// abort flag is raised, when another CTA of the launch timed out, or after kWaitLimitNs, in
+// abort flag is raised, when another CTA of the launch timed out, or after `limit_ns`, in
 // which case it records kErrTimeout, raises the abort flag and returns false.  Never spins
-// forever, and one expired wait stops every CTA of the launch within microseconds.
+// forever, and one expired wait stops every CTA of the launch within microseconds.  A limit
+// of 0 makes every wait that is not complete at its first test expire.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* err) {
+                                          uint32_t* err, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_test_sleep(bar, parity, 200000u)) return true;   // sleeps at most ~0.2 ms
-    {
-      if (*abort_flag) return false;
-      if (launch_timed_out(err)) {
-        *abort_flag = 1;
-        return false;
-      }
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        flag_error(err, kErrTimeout);
-        *abort_flag = 1;
-        return false;
-      }
+  // sleep at most ~0.2 ms per test, less when the limit is shorter
+  const uint32_t hint = limit_ns < 200000ull ? static_cast<uint32_t>(limit_ns) + 32u : 200000u;
+  for (;;) {
+    if (mbar_test_sleep(bar, parity, hint)) return true;
+    if (*abort_flag) return false;
+    if (launch_timed_out(err)) {
+      *abort_flag = 1;
+      return false;
+    }
+    if (globaltimer_ns() - t0 >= limit_ns) {
+      flag_error(err, kErrTimeout);
+      *abort_flag = 1;
+      return false;
     }
   }
 }

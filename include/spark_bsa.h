@@ -86,6 +86,18 @@ typedef enum { SPARK_BF16 = 0, SPARK_F32 = 1 } spark_dtype;
 /* Human-readable name of a status code; never NULL. */
 SPARK_API const char* spark_status_string(int status);
 
+/* Limit of every bounded wait inside the library's kernels, in nanoseconds of the GPU's
+ * global timer (no counterpart in the pages: a safety bound of this implementation).  The
+ * kernels that wait on barriers (the attention, the partitioner's tensor-core kernels) take
+ * the value current at their launch as a parameter; default 4e9 (4 s).  When a wait runs out
+ * the kernel sets SPARK_DEVERR_TIMEOUT in the device error word, stops every CTA of the
+ * launch, waits (with the default limit) for its own copies and MMAs in flight, frees its
+ * tensor memory and returns, so the context stays usable and the error is read with
+ * spark_bsa_read_error.  0 makes every wait that is not complete at its first test expire
+ * (used by a test of that path).  Process-wide (all devices and threads); atomic. */
+SPARK_API void spark_bsa_set_wait_limit_ns(uint64_t limit_ns);
+SPARK_API uint64_t spark_bsa_get_wait_limit_ns(void);
+
 /* k = clamp(ceil(topk_ratio * nkb - 1e-9), 1, nkb) - the blog's "top ratio" budget with
  * a guard against binary rounding of the ratio.  Returns -1 if nkb < 1 or the ratio is
  * outside (0, 1]. */
