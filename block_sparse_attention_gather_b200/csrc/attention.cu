@@ -23,7 +23,7 @@
 //   warp 8     TMA producer: the Q tile once, then K tiles (3-stage ring; a stage is free again
 //              once the S MMA that read it has completed, signalled by that S buffer's barrier).
 //   warp 9     TMA producer of V tiles (2-stage ring).
-//   warp 10    MMA issuer (one thread): S(t) = Q K^T (both from shared memory) into TMEM
+//   warp 10    MMA issuer (the warp runs the loop, one elected lane issues): S(t) = Q K^T (both from shared memory) into TMEM
 //              buffer t%3, O += P(t) V(t) (P read from TMEM, V an MN-major shared-memory
 //              operand).  Issue order S(0), S(1), S(2), PV(0), S(3), PV(1), S(4), ...: MMAs
 //              of one thread execute in order, so S(t+3) overwrites its buffer only after
@@ -357,21 +357,27 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       }
     } else if (warp == kWarpMma) {
       // ---------------------------------------------------------------- MMA issuer
-      if (lane == 0) {
-        constexpr uint32_t idS = kFp8 ? idesc_e4m3(128, 128) : idesc_bf16(128, 128, false, false);
-        constexpr uint32_t idO = idesc_bf16(128, D, false, true);
-        // descriptors built once; per MMA only a compile-time offset (16-byte units) changes
-        const uint64_t qd = sdesc_sw128(smem_u32(qst), 16, 1024);
-        const uint64_t kdesc0 = sdesc_sw128(smem_u32(kst), 16, 1024);
-        const uint64_t vdesc0 = sdesc_sw128(smem_u32(vst), 16384, 1024);
-        bool ok = pass > 0 || mbar_wait(&bars->qfull, 0, abort_flag, err, wait_ns);
-        // S(t) of this pass into buffer (tg0 + t) % 3
-        auto issue_s = [&](int t) -> bool {
-          const int tg = tg0 + t;
-          const int s = tg % kKStages;
-          if (!mbar_wait(&bars->kfull[s], (tg / kKStages) & 1, abort_flag, err, wait_ns)) return false;
-          const uint32_t dcol = tbase + (tg % 3) * 128;
-          const uint64_t kd = kdesc0 + static_cast<uint64_t>(s * (QK_BYTES >> 4));
+      // The whole warp runs the issue loop, so stage indices and descriptors are warp-uniform
+      // values; one elected lane issues the MMAs and their commits (the same lane each time:
+      // the warp is converged at every election, and a commit tracks its own thread's MMAs).
+      constexpr uint32_t idS = kFp8 ? idesc_e4m3(128, 128) : idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idO = idesc_bf16(128, D, false, true);
+      constexpr uint32_t kAll = 0xffffffffu;
+      // descriptors built once; per MMA only a compile-time offset (16-byte units) changes
+      const uint64_t qd = sdesc_sw128(smem_u32(qst), 16, 1024);
+      const uint64_t kdesc0 = sdesc_sw128(smem_u32(kst), 16, 1024);
+      const uint64_t vdesc0 = sdesc_sw128(smem_u32(vst), 16384, 1024);
+      bool ok = pass > 0 || __all_sync(kAll, mbar_wait(&bars->qfull, 0, abort_flag, err, wait_ns));
+      // S(t) of this pass into buffer (tg0 + t) % 3
+      auto issue_s = [&](int t) -> bool {
+        const int tg = tg0 + t;
+        const int s = tg % kKStages;
+        if (!__all_sync(kAll, mbar_wait(&bars->kfull[s], (tg / kKStages) & 1, abort_flag, err,
+                                        wait_ns)))
+          return false;
+        const uint32_t dcol = tbase + (tg % 3) * 128;
+        const uint64_t kd = kdesc0 + static_cast<uint64_t>(s * (QK_BYTES >> 4));
+        if (elect_one()) {
           if constexpr (kFp8) {
             // 32 e4m3 values of d = 32 bytes per MMA, all inside the one 128-byte atom row
 #pragma unroll
@@ -385,30 +391,39 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
             }
           }
           tc_commit(&bars->sfull[tg % 3]);
-          return true;
-        };
-        for (int t = 0; ok && t < min(T, 3); ++t) ok = issue_s(t);
-        for (int t = 0; ok && t < T; ++t) {
-          const int tg = tg0 + t;
-          if (!mbar_wait(&bars->pready[tg % 3], (tg / 3) & 1, abort_flag, err, wait_ns)) break;
-          tc_fence_after_sync();
-          const int s = tg % kVStages;
-          if (!mbar_wait(&bars->vfull[s], (tg / kVStages) & 1, abort_flag, err, wait_ns)) break;
-          const uint64_t vd = vdesc0 + static_cast<uint64_t>(s * (V_BYTES >> 4));
-          const uint32_t pcol = tbase + (tg % 3) * 128;               // P(t) over S(t)
+        }
+        __syncwarp();
+        return true;
+      };
+      for (int t = 0; ok && t < min(T, 3); ++t) ok = issue_s(t);
+      for (int t = 0; ok && t < T; ++t) {
+        const int tg = tg0 + t;
+        if (!__all_sync(kAll, mbar_wait(&bars->pready[tg % 3], (tg / 3) & 1, abort_flag, err,
+                                        wait_ns)))
+          break;
+        tc_fence_after_sync();
+        const int s = tg % kVStages;
+        if (!__all_sync(kAll, mbar_wait(&bars->vfull[s], (tg / kVStages) & 1, abort_flag, err,
+                                        wait_ns)))
+          break;
+        const uint64_t vd = vdesc0 + static_cast<uint64_t>(s * (V_BYTES >> 4));
+        const uint32_t pcol = tbase + (tg % 3) * 128;               // P(t) over S(t)
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tbase + kColO, pcol + kk * 8, vd + (kk * 2048) / 16, idO,
                    (kk > 0 || t > 0) ? 1u : 0u);
           tc_commit(&bars->vempty[s]);
-          // S(t+3) reuses the columns of P(t): issued after PV(t), and MMAs of one thread
-          // execute in order
-          if (t + 3 < T && !(ok = issue_s(t + 3))) break;
         }
-        // every MMA complete: the softmax epilogue reads O, and TMEM is reused or freed after
-        tc_commit(&bars->done);
-        wait_bounded_ignore_abort(&bars->done, pass);
+        __syncwarp();
+        // S(t+3) reuses the columns of P(t): issued after PV(t), and MMAs of one thread
+        // execute in order
+        if (t + 3 < T && !(ok = issue_s(t + 3))) break;
       }
+      // every MMA complete: the softmax epilogue reads O, and TMEM is reused or freed after
+      if (elect_one()) tc_commit(&bars->done);
+      __syncwarp();
+      wait_bounded_ignore_abort(&bars->done, pass);
     } else {
       // ---------------------------------------------------------------- softmax rows
       const int q4 = warp & 3, grp = warp >> 2;          // row quarter, tile group
