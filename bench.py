@@ -711,64 +711,36 @@ def main():
     e2e = None
     comparator = args.summaries != "reweight" or args.routing != "topk"
     if args.e2e_steps > 0 and not comparator:      # the public calls run the method itself
-        from block_sparse_attention_gather_b200 import (spark_bsa_forward, spark_bsa_forward_ctx,
-                                                        spark_bsa_forward_fp8,
-                                                        spark_bsa_forward_host,
-                                                        spark_bsa_host_staging_size,
-                                                        spark_bsa_workspace_size,
+        from block_sparse_attention_gather_b200 import (spark_bsa_forward_host,
+                                                        spark_bsa_host_staging_size_ex,
+                                                        spark_bsa_workspace_size_ctx,
                                                         spark_bsa_workspace_size_fp8)
         names = ["Q", "K", "V", "q_perm", "k_perm", "q_offsets", "k_offsets"]
         if hp.nc:
             names += ["Kc", "Vc"]
         host = {n: x[n].to("cpu").pin_memory() for n in names}
-        piped = not hp.nc and not hp.fp8
-        dev_in = {n: torch.empty_like(x[n]) for n in host} if not piped else {}
-        if hp.fp8:
-            ws8 = torch.empty(spark_bsa_workspace_size_fp8(hp.H, hp.N, hp.d, hp.nqb, hp.nkb,
-                                                           w.ratio, hp.nc),
-                              dtype=torch.uint8, device=device)
         out_host = torch.empty(hp.out.shape, dtype=hp.out.dtype).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = out_host.numel() * out_host.element_size()
         s = torch.cuda.current_stream(device)
-        # without context tokens: the host-buffer entry point, pipelined head by head
+        # the host-buffer entry point, pipelined head by head (every variant: context rows and
+        # FP8 logits included)
         hpc = 1
-        if piped:
-            staging = torch.empty(spark_bsa_host_staging_size(hp.H, hp.N, hp.d, hp.out.dtype,
-                                                              hp.nqb, hp.nkb, hpc),
-                                  dtype=torch.uint8, device=device)
-            chunk_ws = torch.empty(spark_bsa_workspace_size(min(hpc, hp.H), hp.N, hp.d, hp.nqb,
-                                                            hp.nkb, w.ratio),
-                                   dtype=torch.uint8, device=device)
-            pipe = (s, torch.cuda.Stream(device), torch.cuda.Stream(device))
+        staging = torch.empty(spark_bsa_host_staging_size_ex(hp.H, hp.N, hp.d, hp.out.dtype,
+                                                             hp.nqb, hp.nkb, hpc, hp.nc),
+                              dtype=torch.uint8, device=device)
+        ws_size = (spark_bsa_workspace_size_fp8(1, hp.N, hp.d, hp.nqb, hp.nkb, w.ratio, hp.nc)
+                   if hp.fp8 else
+                   spark_bsa_workspace_size_ctx(1, hp.N, hp.d, hp.nqb, hp.nkb, w.ratio, hp.nc))
+        chunk_ws = torch.empty(ws_size, dtype=torch.uint8, device=device)
+        pipe = (s, torch.cuda.Stream(device), torch.cuda.Stream(device))
 
         def e2e_step():
-            if piped:
-                spark_bsa_forward_host(host["Q"], host["K"], host["V"], host["q_perm"],
-                                       host["k_perm"], host["q_offsets"], host["k_offsets"],
-                                       w.ratio, out=out_host, heads_per_chunk=hpc,
-                                       staging=staging, workspace=chunk_ws, streams=pipe)
-                return
-            for n in host:
-                dev_in[n].copy_(host[n], non_blocking=True)
-            if hp.fp8:
-                o, _, _ = spark_bsa_forward_fp8(dev_in["Q"], dev_in["K"], dev_in["V"],
-                                                dev_in["q_perm"], dev_in["k_perm"],
-                                                dev_in["q_offsets"], dev_in["k_offsets"], w.ratio,
-                                                Kc=dev_in.get("Kc"), Vc=dev_in.get("Vc"),
-                                                out=hp.out, workspace=ws8)
-            elif hp.nc:
-                o, _, _ = spark_bsa_forward_ctx(dev_in["Q"], dev_in["K"], dev_in["V"],
-                                                dev_in["Kc"], dev_in["Vc"], dev_in["q_perm"],
-                                                dev_in["k_perm"], dev_in["q_offsets"],
-                                                dev_in["k_offsets"], w.ratio, out=hp.out,
-                                                workspace=hp.ws)
-            else:
-                o, _, _ = spark_bsa_forward(dev_in["Q"], dev_in["K"], dev_in["V"],
-                                            dev_in["q_perm"], dev_in["k_perm"],
-                                            dev_in["q_offsets"], dev_in["k_offsets"], w.ratio,
-                                            out=hp.out, workspace=hp.ws)
-            out_host.copy_(o, non_blocking=True)
+            spark_bsa_forward_host(host["Q"], host["K"], host["V"], host["q_perm"],
+                                   host["k_perm"], host["q_offsets"], host["k_offsets"],
+                                   w.ratio, out=out_host, heads_per_chunk=hpc,
+                                   staging=staging, workspace=chunk_ws, streams=pipe,
+                                   Kc=host.get("Kc"), Vc=host.get("Vc"), fp8=hp.fp8)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -785,13 +757,10 @@ def main():
         e2e = {"value": whole_job_rate(world, dflops, args.e2e_steps, e_ms), "unit": UNIT,
                "ms_per_call": e_ms / args.e2e_steps, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-               "call": ("spark_bsa_forward_fp8 after host-to-device copies" if hp.fp8 else
-                        "spark_bsa_forward_ctx after host-to-device copies" if hp.nc else
-                        f"spark_bsa_forward_host (host buffers, chunks of {hpc} heads, copies "
-                        "overlapped with computation on three streams)")}
-        del host, dev_in, out_host
-        if hp.fp8:
-            del ws8
+               "call": (f"spark_bsa_forward_host{' (FP8 logits)' if hp.fp8 else ''}"
+                        f"{' with context rows' if hp.nc else ''} (host buffers, chunks of "
+                        f"{hpc} heads, copies overlapped with computation on three streams)")}
+        del host, out_host, staging, chunk_ws
 
     # ---- the partitioner upstream of the path, on the same Q and K (its own timed calls)
     reblock = None

@@ -28,6 +28,7 @@ __all__ = [
     "spark_bsa_attend_fp8", "spark_bsa_workspace_size_fp8", "spark_bsa_forward_fp8",
     "spark_bsa_gather_kv_meanpool", "spark_bsa_route_threshold", "spark_bsa_attend_var",
     "spark_bsa_set_wait_limit_ns", "spark_bsa_get_wait_limit_ns",
+    "spark_bsa_host_staging_size_ex",
 ]
 
 SPARK_BF16, SPARK_F32 = 0, 1
@@ -44,6 +45,7 @@ EXPORTED = [
     "spark_bsa_attend_fp8", "spark_bsa_workspace_size_fp8", "spark_bsa_forward_fp8",
     "spark_bsa_gather_kv_meanpool", "spark_bsa_route_threshold", "spark_bsa_attend_var",
     "spark_bsa_set_wait_limit_ns", "spark_bsa_get_wait_limit_ns",
+    "spark_bsa_host_staging_size_ex", "spark_bsa_forward_host_ex",
 ]
 REBLOCK_MODES = {"q_reuse_k": 0, "separate": 1}
 
@@ -114,6 +116,10 @@ def lib():
         "spark_reblock_whiten": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P]),
         "spark_reblock_level": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
         "spark_bsa_host_staging_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+        "spark_bsa_host_staging_size_ex": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
+        "spark_bsa_forward_host_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P,
+                                           _P, _I, _P, _I, _D, _P, _I, _P, _SZ, _P, _SZ, _P,
+                                           _P, _P]),
         "spark_bsa_forward_host": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _I, _D,
                                         _P, _I, _P, _SZ, _P, _SZ, _P, _P, _P]),
         "spark_bsa_quantize_fp8": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P]),
@@ -737,12 +743,18 @@ def _need_host(t, name, dtype=None):
         raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
 
 
+def spark_bsa_host_staging_size_ex(H, N, d, dtype, nqb, nkb, heads_per_chunk, nc) -> int:
+    return int(lib().spark_bsa_host_staging_size_ex(H, N, d, _code(dtype), nqb, nkb,
+                                                    heads_per_chunk, nc))
+
+
 def spark_bsa_forward_host(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, topk_ratio, out=None,
                            heads_per_chunk=1, device=None, staging=None, workspace=None,
-                           streams=None):
+                           streams=None, Kc=None, Vc=None, fp8=False):
     """The forward pass on HOST tensors (page-locked for overlap), pipelined by head chunks
     over three CUDA streams; returns `out` (host) once the work is enqueued on the compute
-    stream (synchronise that stream, or the device, before reading it)."""
+    stream (synchronise that stream, or the device, before reading it).  Kc, Vc (host
+    [H, nc, d]) add context rows; fp8=True takes the logits in e4m3 (d = 128)."""
     _need_host(Q, "Q", (torch.bfloat16, torch.float32))
     for n, t in (("K", K), ("V", V)):
         _need_host(t, n, Q.dtype)
@@ -750,6 +762,13 @@ def spark_bsa_forward_host(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, topk_r
                  ("k_offsets", k_offsets)):
         _need_host(t, n, torch.int32)
     H, N, d = Q.shape
+    nc = 0
+    if Kc is not None or Vc is not None:
+        for n, t in (("Kc", Kc), ("Vc", Vc)):
+            _need_host(t, n, Q.dtype)
+        if Kc.shape != Vc.shape or Kc.shape[0] != H or Kc.shape[2] != d:
+            raise ValueError("Kc, Vc must have the shape [H, nc, d]")
+        nc = Kc.shape[1]
     nqb, nkb = q_offsets.numel() - 1, k_offsets.numel() - 1
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
     hpc = max(1, min(int(heads_per_chunk), H))
@@ -757,18 +776,21 @@ def spark_bsa_forward_host(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, topk_r
         out = torch.empty_like(Q).pin_memory()
     _need_host(out, "out", Q.dtype)
     if staging is None:
-        staging = torch.empty(spark_bsa_host_staging_size(H, N, d, Q.dtype, nqb, nkb, hpc),
+        staging = torch.empty(spark_bsa_host_staging_size_ex(H, N, d, Q.dtype, nqb, nkb, hpc, nc),
                               dtype=torch.uint8, device=dev)
     if workspace is None:
-        workspace = torch.empty(spark_bsa_workspace_size(hpc, N, d, nqb, nkb, topk_ratio),
-                                dtype=torch.uint8, device=dev)
+        size = (spark_bsa_workspace_size_fp8(hpc, N, d, nqb, nkb, topk_ratio, nc) if fp8 else
+                spark_bsa_workspace_size_ctx(hpc, N, d, nqb, nkb, topk_ratio, nc))
+        workspace = torch.empty(size, dtype=torch.uint8, device=dev)
     if streams is None:
         streams = (torch.cuda.current_stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev))
     sc, sh, sd = (ctypes.c_void_p(s.cuda_stream) for s in streams)
-    st = lib().spark_bsa_forward_host(_ptr(Q), _ptr(K), _ptr(V), _code(Q.dtype), H, N, d,
-                                      _ptr(q_perm), _ptr(k_perm), _ptr(q_offsets), nqb,
-                                      _ptr(k_offsets), nkb, float(topk_ratio), _ptr(out), hpc,
-                                      _ptr(staging), staging.numel(), _ptr(workspace),
-                                      workspace.numel(), sc, sh, sd)
+    st = lib().spark_bsa_forward_host_ex(_ptr(Q), _ptr(K), _ptr(V),
+                                         _ptr(Kc) if nc else None, _ptr(Vc) if nc else None, nc,
+                                         1 if fp8 else 0, _code(Q.dtype), H, N, d,
+                                         _ptr(q_perm), _ptr(k_perm), _ptr(q_offsets), nqb,
+                                         _ptr(k_offsets), nkb, float(topk_ratio), _ptr(out), hpc,
+                                         _ptr(staging), staging.numel(), _ptr(workspace),
+                                         workspace.numel(), sc, sh, sd)
     _check("spark_bsa_forward_host", st)
     return out

@@ -606,10 +606,10 @@ spark_status spark_bsa_forward_fp8(const void* Q, const void* K, const void* V, 
 namespace {
 
 struct HostStaging {
-  size_t Q, K, V, qp, kp, out, slot, qo, ko, total;
+  size_t Q, K, V, qp, kp, out, Kc, Vc, slot, qo, ko, total;
 };
 
-HostStaging staging_layout(int hpc, int N, int d, int esize, int nqb, int nkb) {
+HostStaging staging_layout(int hpc, int N, int d, int esize, int nqb, int nkb, int nc = 0) {
   HostStaging L{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -624,6 +624,8 @@ HostStaging staging_layout(int hpc, int N, int d, int esize, int nqb, int nkb) {
   L.qp = take(rows * 4);
   L.kp = take(rows * 4);
   L.out = take(rows * d * esize);
+  L.Kc = take(static_cast<size_t>(hpc) * nc * d * esize);   // context rows of the chunk's heads
+  L.Vc = take(static_cast<size_t>(hpc) * nc * d * esize);
   L.slot = off;                                  // one slot; the second follows at +slot
   off = 2 * L.slot;
   L.qo = take(static_cast<size_t>(nqb + 1) * 4);
@@ -642,29 +644,35 @@ size_t spark_bsa_host_staging_size(int H, int N, int d, int dtype, int nqb, int 
   return staging_layout(hpc, N, d, dtype == SPARK_BF16 ? 2 : 4, nqb, nkb).total;
 }
 
-spark_status spark_bsa_forward_host(const void* Q, const void* K, const void* V, int dtype,
-                                    int H, int N, int d, const int32_t* q_perm,
-                                    const int32_t* k_perm, const int32_t* q_block_offsets,
-                                    int nqb, const int32_t* k_block_offsets, int nkb,
-                                    double topk_ratio, void* out, int heads_per_chunk,
-                                    void* staging, size_t staging_bytes, void* workspace,
-                                    size_t workspace_bytes, void* compute_stream,
-                                    void* h2d_stream, void* d2h_stream) {
+namespace {
+
+// The host-buffer pipeline for every variant: nc context rows per head (Kc, Vc host [H,nc,d],
+// none when nc == 0) and FP8 logits when fp8 is set.
+spark_status forward_host_impl(const void* Q, const void* K, const void* V, const void* Kc,
+                               const void* Vc, int nc, bool fp8, int dtype, int H, int N, int d,
+                               const int32_t* q_perm, const int32_t* k_perm,
+                               const int32_t* q_block_offsets, int nqb,
+                               const int32_t* k_block_offsets, int nkb, double topk_ratio,
+                               void* out, int heads_per_chunk, void* staging,
+                               size_t staging_bytes, void* workspace, size_t workspace_bytes,
+                               void* compute_stream, void* h2d_stream, void* d2h_stream) {
   if (!Q || !K || !V || !q_perm || !k_perm || !q_block_offsets || !k_block_offsets || !out)
     return SPARK_ERR_INVALID_ARG;
   if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
   if (heads_per_chunk < 1) return SPARK_ERR_INVALID_ARG;
+  if (nc < 0 || nc > SPARK_MAX_NC || (nc > 0 && (!Kc || !Vc))) return SPARK_ERR_INVALID_ARG;
+  if (fp8 && d != 128) return SPARK_ERR_UNSUPPORTED;
   spark_bsa_layout whole;
   spark_status st = layout_of(H, N, d, nqb, nkb, topk_ratio, &whole);
   if (st != SPARK_OK) return st;
   const int hpc = heads_per_chunk < H ? heads_per_chunk : H;
-  spark_bsa_layout chunk_layout;
-  st = layout_of(hpc, N, d, nqb, nkb, topk_ratio, &chunk_layout);
-  if (st != SPARK_OK) return st;
+  const size_t chunk_ws = fp8 ? spark_bsa_workspace_size_fp8(hpc, N, d, nqb, nkb, topk_ratio, nc)
+                              : spark_bsa_workspace_size_ctx(hpc, N, d, nqb, nkb, topk_ratio, nc);
+  if (chunk_ws == 0) return SPARK_ERR_INVALID_ARG;
   const int esize = dtype == SPARK_BF16 ? 2 : 4;
-  const HostStaging S = staging_layout(hpc, N, d, esize, nqb, nkb);
+  const HostStaging S = staging_layout(hpc, N, d, esize, nqb, nkb, nc);
   if (!staging || staging_bytes < S.total || !aligned(staging, kAlign)) return SPARK_ERR_WORKSPACE;
-  if (!workspace || workspace_bytes < chunk_layout.total || !aligned(workspace, kAlign))
+  if (!workspace || workspace_bytes < chunk_ws || !aligned(workspace, kAlign))
     return SPARK_ERR_WORKSPACE;
   cudaStream_t sc = as_stream(compute_stream), sh = as_stream(h2d_stream),
                sd = as_stream(d2h_stream);
@@ -702,6 +710,9 @@ spark_status spark_bsa_forward_host(const void* Q, const void* K, const void* V,
   const auto* q8 = static_cast<const uint8_t*>(Q);
   const auto* k8 = static_cast<const uint8_t*>(K);
   const auto* v8 = static_cast<const uint8_t*>(V);
+  const auto* kc8 = static_cast<const uint8_t*>(Kc);
+  const auto* vc8 = static_cast<const uint8_t*>(Vc);
+  const size_t ctx_bytes = static_cast<size_t>(nc) * d * esize;   // one head's context rows
   auto* o8 = static_cast<uint8_t*>(out);
   for (int c = 0; c < nchunks; ++c) {
     const int slot = c & 1;
@@ -719,16 +730,23 @@ spark_status spark_bsa_forward_host(const void* Q, const void* K, const void* V,
         cudaMemcpyAsync(base + S.qp, q_perm + static_cast<size_t>(h0) * N, hc * perm_bytes,
                         cudaMemcpyHostToDevice, sh) != cudaSuccess ||
         cudaMemcpyAsync(base + S.kp, k_perm + static_cast<size_t>(h0) * N, hc * perm_bytes,
-                        cudaMemcpyHostToDevice, sh) != cudaSuccess ||
-        cudaEventRecord(h2d_done[slot], sh) != cudaSuccess)
+                        cudaMemcpyHostToDevice, sh) != cudaSuccess)
       return fail();
+    if (nc > 0 &&
+        (cudaMemcpyAsync(base + S.Kc, kc8 + h0 * ctx_bytes, hc * ctx_bytes,
+                         cudaMemcpyHostToDevice, sh) != cudaSuccess ||
+         cudaMemcpyAsync(base + S.Vc, vc8 + h0 * ctx_bytes, hc * ctx_bytes,
+                         cudaMemcpyHostToDevice, sh) != cudaSuccess))
+      return fail();
+    if (cudaEventRecord(h2d_done[slot], sh) != cudaSuccess) return fail();
     // the forward pass of the chunk, once its inputs are in and the slot's output is read out
     if (cudaStreamWaitEvent(sc, h2d_done[slot], 0) != cudaSuccess) return fail();
     if (c >= 2 && cudaStreamWaitEvent(sc, d2h_done[slot], 0) != cudaSuccess) return fail();
-    st = forward_impl(base + S.Q, base + S.K, base + S.V, nullptr, nullptr, 0, dtype, hc, N, d,
+    st = forward_impl(base + S.Q, base + S.K, base + S.V, nc > 0 ? base + S.Kc : nullptr,
+                      nc > 0 ? base + S.Vc : nullptr, nc, dtype, hc, N, d,
                       reinterpret_cast<const int32_t*>(base + S.qp),
                       reinterpret_cast<const int32_t*>(base + S.kp), qo, nqb, ko, nkb,
-                      topk_ratio, base + S.out, workspace, workspace_bytes, sc);
+                      topk_ratio, base + S.out, workspace, workspace_bytes, sc, fp8);
     if (st != SPARK_OK) {
       for (auto& e : ev) cudaEventDestroy(e);
       return st;
@@ -746,6 +764,46 @@ spark_status spark_bsa_forward_host(const void* Q, const void* K, const void* V,
     if (cudaStreamWaitEvent(sc, d2h_done[slot], 0) != cudaSuccess) return fail();
   for (auto& e : ev) cudaEventDestroy(e);   // released once the pending work completes
   return SPARK_OK;
+}
+
+}  // namespace
+
+spark_status spark_bsa_forward_host(const void* Q, const void* K, const void* V, int dtype,
+                                    int H, int N, int d, const int32_t* q_perm,
+                                    const int32_t* k_perm, const int32_t* q_block_offsets,
+                                    int nqb, const int32_t* k_block_offsets, int nkb,
+                                    double topk_ratio, void* out, int heads_per_chunk,
+                                    void* staging, size_t staging_bytes, void* workspace,
+                                    size_t workspace_bytes, void* compute_stream,
+                                    void* h2d_stream, void* d2h_stream) {
+  return forward_host_impl(Q, K, V, nullptr, nullptr, 0, false, dtype, H, N, d, q_perm, k_perm,
+                           q_block_offsets, nqb, k_block_offsets, nkb, topk_ratio, out,
+                           heads_per_chunk, staging, staging_bytes, workspace, workspace_bytes,
+                           compute_stream, h2d_stream, d2h_stream);
+}
+
+size_t spark_bsa_host_staging_size_ex(int H, int N, int d, int dtype, int nqb, int nkb,
+                                      int heads_per_chunk, int nc) {
+  if (check_sizes(H, N, d, nqb, nkb) != SPARK_OK || heads_per_chunk < 1) return 0;
+  if (dtype != SPARK_BF16 && dtype != SPARK_F32) return 0;
+  if (nc < 0 || nc > SPARK_MAX_NC) return 0;
+  const int hpc = heads_per_chunk < H ? heads_per_chunk : H;
+  return staging_layout(hpc, N, d, dtype == SPARK_BF16 ? 2 : 4, nqb, nkb, nc).total;
+}
+
+spark_status spark_bsa_forward_host_ex(const void* Q, const void* K, const void* V,
+                                       const void* Kc, const void* Vc, int nc, int fp8_logits,
+                                       int dtype, int H, int N, int d, const int32_t* q_perm,
+                                       const int32_t* k_perm, const int32_t* q_block_offsets,
+                                       int nqb, const int32_t* k_block_offsets, int nkb,
+                                       double topk_ratio, void* out, int heads_per_chunk,
+                                       void* staging, size_t staging_bytes, void* workspace,
+                                       size_t workspace_bytes, void* compute_stream,
+                                       void* h2d_stream, void* d2h_stream) {
+  return forward_host_impl(Q, K, V, Kc, Vc, nc, fp8_logits != 0, dtype, H, N, d, q_perm, k_perm,
+                           q_block_offsets, nqb, k_block_offsets, nkb, topk_ratio, out,
+                           heads_per_chunk, staging, staging_bytes, workspace, workspace_bytes,
+                           compute_stream, h2d_stream, d2h_stream);
 }
 
 // ---------------------------------------------------------------- Spark-Reblock

@@ -20,7 +20,8 @@
 //              rows take their recorded maximum as the reference - each chunk whose sum is out
 //              of range records its maximum, which is within a few units of the row's - and the
 //              other rows keep theirs.
-//   warp 8     TMA producer: the Q tile once, then K tiles (3-stage ring; a stage is free again
+//   warp 8     TMA producer (the warp runs the loop, one elected lane issues): the Q tile once,
+//              then K tiles (3-stage ring; a stage is free again
 //              once the S MMA that read it has completed, signalled by that S buffer's barrier).
 //   warp 9     TMA producer of V tiles (2-stage ring).
 //   warp 10    MMA issuer (the warp runs the loop, one elected lane issues): S(t) = Q K^T (both from shared memory) into TMEM
@@ -61,6 +62,10 @@ struct __align__(8) Barriers {
   // the K ring's stages are released by sfull: K stage and S buffer of a tile coincide
   uint64_t kfull[kKStages], vfull[kVStages], vempty[kVStages];
   uint64_t sfull[3], pready[3], done;
+  // keys the MMAs of a tile cover (its valid rows rounded up to 16; 128 for summary tiles):
+  // written by the K producer per stage before the stage's loads, read by the MMA thread
+  uint32_t kn[kKStages];
+  uint32_t bn[3];                              // the MMA thread's copy per S buffer
 };
 
 __device__ __forceinline__ bool wait_bounded_ignore_abort(uint64_t* bar, uint32_t parity) {
@@ -124,6 +129,12 @@ __device__ __forceinline__ TileInfo tile_info(int t, int k, int nxt, int nc,
   return ti;
 }
 
+// Keys (columns of S, rows of V) the MMAs of a tile cover: exact tiles stop at their valid
+// rows rounded up to 16 (the MMA's N step for M = 128), summary tiles cover all 128.
+__device__ __forceinline__ int tile_cols(const TileInfo& ti) {
+  return ti.exact ? min(128, max(16, (ti.nvalid + 15) & ~15)) : 128;
+}
+
 // Reads 64 columns of this thread's S row (TMEM) and turns them into logits: exact tiles give
 // raw scores (the scale is applied in the exponent) with columns past the block set to -inf;
 // summary tiles give s*sl + offset (offset -inf for selected blocks and padding), sl being the
@@ -166,6 +177,28 @@ __device__ __forceinline__ void load_logits(uint32_t taddr, int col0, const Tile
   }
 }
 
+// The 32 columns col0 .. col0+31 of an exact tile into x[0..31] (columns past the valid rows
+// masked to -inf); x[32..63] are left as they are.
+__device__ __forceinline__ void load_logits32_exact(uint32_t taddr, int col0, const TileInfo& ti,
+                                                    float (&x)[64]) {
+  uint32_t r[32];
+  tmem_ld32(taddr, r);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) x[j] = (col0 + j < ti.nvalid) ? __uint_as_float(r[j]) : -INFINITY;
+}
+
+__device__ __forceinline__ float max32(const float (&x)[64]) {
+  float mx[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+  for (int j = 4; j < 32; j += 8) {
+    mx[0] = fmax3(mx[0], x[j], x[j + 1]);
+    mx[1] = fmax3(mx[1], x[j + 2], x[j + 3]);
+    mx[2] = fmax3(mx[2], x[j + 4], x[j + 5]);
+    mx[3] = fmax3(mx[3], x[j + 6], x[j + 7]);
+  }
+  return fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
+}
+
 __device__ __forceinline__ float max64(const float (&x)[64]) {
   float mx[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
@@ -178,6 +211,10 @@ __device__ __forceinline__ float max64(const float (&x)[64]) {
   return fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
 }
 
+// Every kPolyEvery-th pair of exponentials is computed on the FMA pipe (exp2_poly_x2) instead
+// of MUFU, whose throughput per SM matches the tensor cores' for this tile shape (0: none).
+constexpr int kPolyEvery = 0;
+
 // p = 2^(x*c - m) for the 32 columns x[j0 .. j0+31], packed to bf16 pairs; returns their sum.
 __device__ __forceinline__ float exp32_at(const float (&x)[64], int j0, float c, float m,
                                           uint32_t (&pk)[16]) {
@@ -187,9 +224,15 @@ __device__ __forceinline__ float exp32_at(const float (&x)[64], int j0, float c,
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const uint64_t a2 = f2_fma(f2_pack(x[j0 + 2 * j], x[j0 + 2 * j + 1]), c2, nm2);
-    float a0, a1;
-    f2_unpack(a2, a0, a1);
-    const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+    float p0, p1;
+    if (kPolyEvery > 0 && j % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+      f2_unpack(exp2_poly_x2(a2), p0, p1);
+    } else {
+      float a0, a1;
+      f2_unpack(a2, a0, a1);
+      p0 = ex2_approx(a0);
+      p1 = ex2_approx(a1);
+    }
     sum2[j & 1] = f2_add(sum2[j & 1], f2_pack(p0, p1));
     pk[j] = pack_bf16(p0, p1);
   }
@@ -305,23 +348,26 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     const int tg0 = pass * T;                      // tile counter of this pass's first tile
     if (warp == kWarpK || warp == kWarpV) {
       // ----------------------------------------------------------- TMA producers
-      if (lane == 0) {
-        const bool is_k = (warp == kWarpK);
-        const int stages = is_k ? kKStages : kVStages;
-        const int tile_bytes = is_k ? QK_BYTES : V_BYTES;
-        const int atoms = is_k ? QK_ATOMS : V_ATOMS;
-        const int atom_x = is_k ? QK_ATOM_X : 64;
-        uint8_t* ring = is_k ? kst : vst;
-        uint64_t* full = is_k ? bars->kfull : bars->vfull;
-        // a K stage is free once the S MMA that read it has completed: stage tg % 3 and S
-        // buffer tg % 3 belong to the same tile, so sfull also releases the K ring (one
-        // commit less per tile for the MMA thread, measured 1.7% faster)
-        static_assert(kKStages == 3, "K stages and S buffers must coincide");
-        uint64_t* empty = is_k ? bars->sfull : bars->vempty;
-        const CUtensorMap* mx = is_k ? &map_k : &map_v;
-        const CUtensorMap* mc = is_k ? &map_kc : &map_vc;
-        const CUtensorMap* ms = is_k ? &map_kt : &map_vt;
-        if (pass == 0) {
+      // The whole warp runs the loop (warp-uniform stage indices and coordinates); one elected
+      // lane issues the copies.
+      constexpr uint32_t kAll = 0xffffffffu;
+      const bool is_k = (warp == kWarpK);
+      const int stages = is_k ? kKStages : kVStages;
+      const int tile_bytes = is_k ? QK_BYTES : V_BYTES;
+      const int atoms = is_k ? QK_ATOMS : V_ATOMS;
+      const int atom_x = is_k ? QK_ATOM_X : 64;
+      uint8_t* ring = is_k ? kst : vst;
+      uint64_t* full = is_k ? bars->kfull : bars->vfull;
+      // a K stage is free once the S MMA that read it has completed: stage tg % 3 and S
+      // buffer tg % 3 belong to the same tile, so sfull also releases the K ring (one
+      // commit less per tile for the MMA thread, measured 1.7% faster)
+      static_assert(kKStages == 3, "K stages and S buffers must coincide");
+      uint64_t* empty = is_k ? bars->sfull : bars->vempty;
+      const CUtensorMap* mx = is_k ? &map_k : &map_v;
+      const CUtensorMap* mc = is_k ? &map_kc : &map_vc;
+      const CUtensorMap* ms = is_k ? &map_kt : &map_vt;
+      if (pass == 0) {
+        if (elect_one()) {
           tma_prefetch_desc(mx);
           tma_prefetch_desc(ms);
           if (nxt > 0) tma_prefetch_desc(mc);
@@ -333,34 +379,42 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
               tma_load_3d(qst + a * 16384, &map_q, &bars->qfull, a * QK_ATOM_X, qrow, h);
           }
         }
-        TileInfo next = tile_info<false>(0, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
-        for (int t = 0; t < T; ++t) {
-          const int tg = tg0 + t;
-          const int s = tg % stages;
-          const TileInfo ti = next;
-          if (tg >= stages && !mbar_wait(&empty[s], ((tg / stages) - 1) & 1, abort_flag, err, wait_ns))
-            break;
+        __syncwarp();
+      }
+      TileInfo next = tile_info<false>(0, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
+      for (int t = 0; t < T; ++t) {
+        const int tg = tg0 + t;
+        const int s = tg % stages;
+        const TileInfo ti = next;
+        if (tg >= stages &&
+            !__all_sync(kAll, mbar_wait(&empty[s], ((tg / stages) - 1) & 1, abort_flag, err,
+                                        wait_ns)))
+          break;
+        if (elect_one()) {
+          if (is_k) bars->kn[s] = static_cast<uint32_t>(tile_cols(ti));   // before the arrive
           mbar_arrive_expect_tx(&full[s], tile_bytes);
           const CUtensorMap* map = ti.src == kSrcVideo ? mx : (ti.src == kSrcContext ? mc : ms);
           for (int a = 0; a < atoms; ++a)
             tma_load_3d(ring + s * tile_bytes + a * 16384, map, &full[s], a * atom_x, ti.y, h);
-          issued = tg + 1;
-          if (t + 1 < T)
-            next = tile_info<false>(t + 1, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
         }
-        if (*abort_flag) {
-          // drain: wait for every load still in flight (the last round of each stage)
-          for (int tg = max(0, issued - stages); tg < issued; ++tg)
-            wait_bounded_ignore_abort(&full[tg % stages], (tg / stages) & 1);
-          if (is_k) wait_bounded_ignore_abort(&bars->qfull, 0);
-        }
+        __syncwarp();
+        issued = tg + 1;
+        if (t + 1 < T)
+          next = tile_info<false>(t + 1, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
       }
+      // every load this pass issued has landed before the pass ends (after an abort some were
+      // never consumed; otherwise these phases are complete already and the waits return at once)
+      for (int tg = max(tg0, issued - stages); tg < issued; ++tg)
+        wait_bounded_ignore_abort(&full[tg % stages], (tg / stages) & 1);
+      if (is_k) wait_bounded_ignore_abort(&bars->qfull, 0);
     } else if (warp == kWarpMma) {
       // ---------------------------------------------------------------- MMA issuer
       // The whole warp runs the issue loop, so stage indices and descriptors are warp-uniform
       // values; one elected lane issues the MMAs and their commits (the same lane each time:
       // the warp is converged at every election, and a commit tracks its own thread's MMAs).
-      constexpr uint32_t idS = kFp8 ? idesc_e4m3(128, 128) : idesc_bf16(128, 128, false, false);
+      // the S descriptor without its N field (set per tile)
+      constexpr uint32_t idS_base = (kFp8 ? idesc_e4m3(128, 128) : idesc_bf16(128, 128, false, false)) &
+                                    ~(0x3Fu << 17);
       constexpr uint32_t idO = idesc_bf16(128, D, false, true);
       constexpr uint32_t kAll = 0xffffffffu;
       // descriptors built once; per MMA only a compile-time offset (16-byte units) changes
@@ -377,17 +431,21 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           return false;
         const uint32_t dcol = tbase + (tg % 3) * 128;
         const uint64_t kd = kdesc0 + static_cast<uint64_t>(s * (QK_BYTES >> 4));
+        // S covers the tile's keys only (N = its valid rows rounded up to 16)
+        const uint32_t ncols = bars->kn[s];
+        const uint32_t idSn = idS_base | ((ncols >> 3) << 17);
         if (elect_one()) {
+          bars->bn[tg % 3] = ncols;
           if constexpr (kFp8) {
             // 32 e4m3 values of d = 32 bytes per MMA, all inside the one 128-byte atom row
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk)
-              mma_ss_f8(dcol, qd + kk * 2, kd + kk * 2, idS, kk > 0 ? 1u : 0u);
+              mma_ss_f8(dcol, qd + kk * 2, kd + kk * 2, idSn, kk > 0 ? 1u : 0u);
           } else {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) / 16;
-              mma_ss(dcol, qd + off, kd + off, idS, kk > 0 ? 1u : 0u);
+              mma_ss(dcol, qd + off, kd + off, idSn, kk > 0 ? 1u : 0u);
             }
           }
           tc_commit(&bars->sfull[tg % 3]);
@@ -409,10 +467,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         const uint64_t vd = vdesc0 + static_cast<uint64_t>(s * (V_BYTES >> 4));
         const uint32_t pcol = tbase + (tg % 3) * 128;               // P(t) over S(t)
         if (elect_one()) {
+          // the tile's keys only, 16 per MMA (P past them is never read)
+          const int nk = static_cast<int>(bars->bn[tg % 3] >> 4);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tbase + kColO, pcol + kk * 8, vd + (kk * 2048) / 16, idO,
-                   (kk > 0 || t > 0) ? 1u : 0u);
+            if (kk < nk)
+              mma_ts(tbase + kColO, pcol + kk * 8, vd + (kk * 2048) / 16, idO,
+                     (kk > 0 || t > 0) ? 1u : 0u);
           tc_commit(&bars->vempty[s]);
         }
         __syncwarp();
@@ -484,19 +545,30 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         // chunk whose sum stays in [2^-40, 2^40] has its maximum within 40 of the reference
         // and cannot drive the row sum out of [2^-60, 2^60] (fewer than 2^16 chunks per row),
         // so only chunks outside that range (rare) take their maximum.
+        // only the columns the MMAs covered (exact tiles: the valid rows rounded up to 16)
+        const int ncols = tile_cols(ti);
         float rowsum = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          load_logits<kBiasSmem>(sbuf + half * 64, half * 64, ti, tsl, biasrow, cb,
-                                 selmask, nkb, x);
+          if (half == 1 && ncols <= 64) break;
           uint32_t p16[16];
-          float cs = exp32_at(x, 0, c, m_ref, p16);
-          tmem_st16_issue(sbuf + half * 32, p16);
-          cs += exp32_at(x, 32, c, m_ref, p16);
-          tmem_st16_issue(sbuf + half * 32 + 16, p16);
-          if (!(cs >= 0x1p-40f && cs <= 0x1p40f)) {
-            const float mt = max64(x);
-            m_true = fmaxf(m_true, ti.exact ? mt * tsl : mt);
+          float cs;
+          if (half == 1 && ncols <= 96) {
+            load_logits32_exact(sbuf + 64, 64, ti, x);      // exact tiles only (summary: 128)
+            cs = exp32_at(x, 0, c, m_ref, p16);
+            tmem_st16_issue(sbuf + 32, p16);
+            if (!(cs >= 0x1p-40f && cs <= 0x1p40f)) m_true = fmaxf(m_true, max32(x) * tsl);
+          } else {
+            load_logits<kBiasSmem>(sbuf + half * 64, half * 64, ti, tsl, biasrow, cb,
+                                   selmask, nkb, x);
+            cs = exp32_at(x, 0, c, m_ref, p16);
+            tmem_st16_issue(sbuf + half * 32, p16);
+            cs += exp32_at(x, 32, c, m_ref, p16);
+            tmem_st16_issue(sbuf + half * 32 + 16, p16);
+            if (!(cs >= 0x1p-40f && cs <= 0x1p40f)) {
+              const float mt = max64(x);
+              m_true = fmaxf(m_true, ti.exact ? mt * tsl : mt);
+            }
           }
           rowsum += cs;
         }

@@ -93,8 +93,8 @@ SPARK_API const char* spark_status_string(int status);
  * the kernel sets SPARK_DEVERR_TIMEOUT in the device error word, stops every CTA of the
  * launch, waits (with the default limit) for its own copies and MMAs in flight, frees its
  * tensor memory and returns, so the context stays usable and the error is read with
- * spark_bsa_read_error.  0 makes every wait that is not complete at its first test expire
- * (used by a test of that path).  Process-wide (all devices and threads); atomic. */
+ * spark_bsa_read_error.  0 makes every wait expire at once, without looking at its barrier
+ * (a deterministic test of that path).  Process-wide (all devices and threads); atomic. */
 SPARK_API void spark_bsa_set_wait_limit_ns(uint64_t limit_ns);
 SPARK_API uint64_t spark_bsa_get_wait_limit_ns(void);
 
@@ -366,6 +366,31 @@ SPARK_API spark_status spark_bsa_forward_host(const void* Q, const void* K, cons
                                               void* workspace, size_t workspace_bytes,
                                               void* compute_stream, void* h2d_stream,
                                               void* d2h_stream);
+
+/* The same host-buffer pipeline for the other variants: nc context (sink) rows per head
+ * (Kc, Vc: HOST [H,nc,d] of `dtype`, copied per chunk with the chunk's heads; NULL when nc is
+ * 0; the semantics of spark_bsa_forward_ctx), and FP8 logits when fp8_logits is non-zero (the
+ * semantics of spark_bsa_forward_fp8; d = 128).  The result equals the device-buffer call of
+ * the same variant bit for bit.
+ *   - `staging`: spark_bsa_host_staging_size_ex bytes (it includes the context rows);
+ *     `workspace`: spark_bsa_workspace_size_fp8(min(heads_per_chunk, H), ..., nc) bytes with
+ *     FP8 logits, else spark_bsa_workspace_size_ctx(min(heads_per_chunk, H), ..., nc).
+ *   - Everything else as for spark_bsa_forward_host, which is this call with nc = 0 and no
+ *     FP8. */
+SPARK_API size_t spark_bsa_host_staging_size_ex(int H, int N, int d, int dtype, int nqb, int nkb,
+                                                int heads_per_chunk, int nc);
+
+SPARK_API spark_status spark_bsa_forward_host_ex(const void* Q, const void* K, const void* V,
+                                                 const void* Kc, const void* Vc, int nc,
+                                                 int fp8_logits, int dtype, int H, int N, int d,
+                                                 const int32_t* q_perm, const int32_t* k_perm,
+                                                 const int32_t* q_block_offsets, int nqb,
+                                                 const int32_t* k_block_offsets, int nkb,
+                                                 double topk_ratio, void* out,
+                                                 int heads_per_chunk, void* staging,
+                                                 size_t staging_bytes, void* workspace,
+                                                 size_t workspace_bytes, void* compute_stream,
+                                                 void* h2d_stream, void* d2h_stream);
 
 /* ---- Spark-Reblock token partitioner ----
  * Spark-H3 blog, section "Spark-Reblock": queries are grouped under the Mahalanobis cosine
