@@ -42,6 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attention_768p_dram.json")
 KERNELS = ["gather_q", "anchor", "gather_kv_summary", "route", "attend"]
 KERNELS_FP8 = ["gather_q", "anchor", "gather_kv_summary", "route", "quantize", "attend"]
+KERNELS_FUSED = ["gather_q", "anchor", "gather_kv_summary", "attend"]
 
 
 def parse_args():
@@ -58,9 +59,10 @@ def parse_args():
                          "quantised per group after the routing), bf16 values")
     ap.add_argument("--summaries", choices=["reweight", "meanpool"], default="reweight",
                     help="meanpool: the baseline BSA compressed branch (comparator)")
-    ap.add_argument("--routing", choices=["topk", "threshold"], default="topk",
+    ap.add_argument("--routing", choices=["topk", "threshold", "fused"], default="topk",
                     help="threshold: mu + tau*sigma per query block, capped at the Top-K k "
-                         "(comparator)")
+                         "(comparator); fused: the Top-K routing inside the attention kernel "
+                         "(no routing launch)")
     ap.add_argument("--tau", type=float, default=1.0)
     ap.add_argument("--reblock-steps", type=int, default=5,
                     help="timed calls of the Spark-Reblock partitioner on the same Q and K, "
@@ -179,12 +181,15 @@ class HotPath:
             if self.nc:
                 self.Kc8 = torch.empty(H, self.nc, d, dtype=u8, device=device)
                 self.kc_scale = torch.empty(H, (self.nc + 127) // 128, dtype=f32, device=device)
-        self.kernels = KERNELS_FP8 if fp8 else KERNELS
+        self.kernels = KERNELS_FP8 if fp8 else (KERNELS_FUSED if routing == "fused" else KERNELS)
         # comparators: mean-pool summaries, threshold routing with per-row counts
         self.summaries, self.routing, self.tau = summaries, routing, tau
-        if routing == "threshold":
+        if routing in ("threshold", "fused"):
             if fp8 or self.nc:
-                raise SystemExit("threshold routing runs without fp8 and context here")
+                raise SystemExit(f"{routing} routing runs without fp8 and context here")
+        if routing == "fused" and not L.spark_bsa_fused_supported(self.d, self.nkb, float(ratio)):
+            raise SystemExit("routing inside the attention kernel does not support this shape")
+        if routing == "threshold":
             self.count = torch.empty(self.H, self.nqb, dtype=torch.int32, device=device)
 
     def _p(self, t):
@@ -218,6 +223,16 @@ class HotPath:
                                                   p(v["kbar"]), p(v["k_tilde"]), p(v["v_tilde"]),
                                                   p(v["cbias"]), err, s)
         rec(3)
+        if self.routing == "fused":
+            st |= L.spark_bsa_attend_fused(p(v["Qp"]), p(v["Kp"]), p(v["Vp"]), p(v["k_tilde"]),
+                                           p(v["v_tilde"]), p(v["cbias"]), p(v["qbar_blocks"]),
+                                           p(v["kbar"]), k, p(x["q_perm"]), p(x["q_offsets"]),
+                                           nqb, p(x["k_offsets"]), nkb, H, N, d, p(self.out),
+                                           self.dtype_code, p(v["sel"]), err, s)
+            rec(4)
+            if st != 0:
+                raise RuntimeError(f"a step entry point failed (status bits {st})")
+            return
         if self.routing == "threshold":
             st |= L.spark_bsa_route_threshold(p(v["qbar_blocks"]), p(v["kbar"]), H, nqb, nkb, d,
                                               float(self.tau), k, p(v["sel"]), p(self.count),
@@ -796,7 +811,7 @@ def main():
                                                            FALLBACK_PEAKS["bf16_tflops"]) *
                                       (0.75 if hp.fp8 else 1.0)},
         "kernels": kernels,
-        "gpu_launches": (5 + (2 if hp.convert_ctx else 0) +
+        "gpu_launches": ((4 if args.routing == "fused" else 5) + (2 if hp.convert_ctx else 0) +
                          ((4 if hp.nc else 3) if hp.fp8 else 0)) * args.steps,
         "clocks": clock_info,
         "e2e": e2e,

@@ -28,7 +28,8 @@ __all__ = [
     "spark_bsa_attend_fp8", "spark_bsa_workspace_size_fp8", "spark_bsa_forward_fp8",
     "spark_bsa_gather_kv_meanpool", "spark_bsa_route_threshold", "spark_bsa_attend_var",
     "spark_bsa_set_wait_limit_ns", "spark_bsa_get_wait_limit_ns",
-    "spark_bsa_host_staging_size_ex",
+    "spark_bsa_host_staging_size_ex", "spark_bsa_fused_supported", "spark_bsa_forward_fused",
+    "spark_bsa_attend_fused",
 ]
 
 SPARK_BF16, SPARK_F32 = 0, 1
@@ -45,7 +46,8 @@ EXPORTED = [
     "spark_bsa_attend_fp8", "spark_bsa_workspace_size_fp8", "spark_bsa_forward_fp8",
     "spark_bsa_gather_kv_meanpool", "spark_bsa_route_threshold", "spark_bsa_attend_var",
     "spark_bsa_set_wait_limit_ns", "spark_bsa_get_wait_limit_ns",
-    "spark_bsa_host_staging_size_ex", "spark_bsa_forward_host_ex",
+    "spark_bsa_host_staging_size_ex", "spark_bsa_forward_host_ex", "spark_bsa_fused_supported",
+    "spark_bsa_forward_fused", "spark_bsa_attend_fused",
 ]
 REBLOCK_MODES = {"q_reuse_k": 0, "separate": 1}
 
@@ -117,6 +119,11 @@ def lib():
         "spark_reblock_level": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
         "spark_bsa_host_staging_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
         "spark_bsa_host_staging_size_ex": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
+        "spark_bsa_fused_supported": (_I, [_I, _I, _D]),
+        "spark_bsa_forward_fused": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _I, _D,
+                                         _P, _P, _SZ, _P]),
+        "spark_bsa_attend_fused": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _P, _I,
+                                        _I, _I, _I, _P, _I, _P, _P, _P]),
         "spark_bsa_forward_host_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P,
                                            _P, _I, _P, _I, _D, _P, _I, _P, _SZ, _P, _SZ, _P,
                                            _P, _P]),
@@ -263,6 +270,62 @@ def spark_bsa_forward(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, topk_ratio,
                                  _ptr(workspace), workspace.numel(), _stream(stream))
     _check("spark_bsa_forward", st)
     return out, workspace, layout
+
+
+def spark_bsa_fused_supported(d: int, nkb: int, topk_ratio: float) -> bool:
+    return bool(lib().spark_bsa_fused_supported(int(d), int(nkb), float(topk_ratio)))
+
+
+def spark_bsa_forward_fused(Q, K, V, q_perm, k_perm, q_offsets, k_offsets, topk_ratio, out=None,
+                            workspace=None, stream=None):
+    """spark_bsa_forward with the routing inside the attention kernel; returns (out, workspace,
+    layout) with the selections copied to the workspace's sel region."""
+    _need(Q, "Q", (torch.bfloat16, torch.float32))
+    dev = Q.device
+    for n, t in (("K", K), ("V", V)):
+        _need(t, n, Q.dtype, dev)
+    H, N, d = Q.shape
+    for n, t in (("q_perm", q_perm), ("k_perm", k_perm), ("q_offsets", q_offsets),
+                 ("k_offsets", k_offsets)):
+        _need(t, n, torch.int32, dev)
+    nqb, nkb = q_offsets.numel() - 1, k_offsets.numel() - 1
+    layout = spark_bsa_workspace_layout(H, N, d, nqb, nkb, topk_ratio)
+    if out is None:
+        out = torch.empty_like(Q)
+    _need(out, "out", Q.dtype, dev)
+    if workspace is None:
+        workspace = torch.empty(layout.total, dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    st = lib().spark_bsa_forward_fused(_ptr(Q), _ptr(K), _ptr(V), _code(Q.dtype), H, N, d,
+                                       _ptr(q_perm), _ptr(k_perm), _ptr(q_offsets), nqb,
+                                       _ptr(k_offsets), nkb, float(topk_ratio), _ptr(out),
+                                       _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("spark_bsa_forward_fused", st)
+    return out, workspace, layout
+
+
+def spark_bsa_attend_fused(Qp, Kp, Vp, k_tilde, v_tilde, cbias, qbar_blocks, kbar, k, q_perm,
+                           q_offsets, k_offsets, out_dtype=torch.bfloat16, out=None, sel_out=None,
+                           err=None, stream=None):
+    _need(Qp, "Qp", torch.bfloat16)
+    dev = Qp.device
+    H, N, d = Qp.shape
+    for n, t, dt in (("Kp", Kp, torch.bfloat16), ("Vp", Vp, torch.bfloat16),
+                     ("k_tilde", k_tilde, torch.bfloat16), ("v_tilde", v_tilde, torch.bfloat16),
+                     ("cbias", cbias, torch.float32), ("qbar_blocks", qbar_blocks, torch.float32),
+                     ("kbar", kbar, torch.float32), ("q_perm", q_perm, torch.int32),
+                     ("q_offsets", q_offsets, torch.int32), ("k_offsets", k_offsets, torch.int32)):
+        _need(t, n, dt, dev)
+    nqb, nkb = q_offsets.numel() - 1, k_offsets.numel() - 1
+    if out is None:
+        out = torch.empty(H, N, d, dtype=out_dtype, device=dev)
+    st = lib().spark_bsa_attend_fused(_ptr(Qp), _ptr(Kp), _ptr(Vp), _ptr(k_tilde), _ptr(v_tilde),
+                                      _ptr(cbias), _ptr(qbar_blocks), _ptr(kbar), int(k),
+                                      _ptr(q_perm), _ptr(q_offsets), nqb, _ptr(k_offsets), nkb,
+                                      H, N, d, _ptr(out), _code(out.dtype), _ptr(sel_out),
+                                      _ptr(err), _stream(stream))
+    _check("spark_bsa_attend_fused", st)
+    return out
 
 
 def spark_bsa_read_error(err_word: torch.Tensor, stream=None) -> int:

@@ -150,6 +150,33 @@ spark_status attend_impl(const void* Qp, const void* Kp, const void* Vp, const v
                                  H, N, d, out, out_dtype, err, s, sel_count));
 }
 
+// The attention with the routing inside: the selection of every query block is computed by the
+// kernel from the block means (sel_out receives a copy when not null).
+spark_status attend_fused_impl(const void* Qp, const void* Kp, const void* Vp,
+                               const void* k_tilde, const void* v_tilde, const float* cbias,
+                               const float* qbar_blocks, const float* kbar, int k,
+                               const void* Kc, const void* Vc, int nc, const int32_t* q_perm,
+                               const int32_t* q_offsets, int nqb, const int32_t* k_offsets,
+                               int nkb, int H, int N, int d, void* out, int out_dtype,
+                               uint32_t* err, int32_t* sel_out, cudaStream_t s) {
+  if (!attend_fused_supported(d, nkb, k)) return SPARK_ERR_UNSUPPORTED;
+  AttendMaps maps;
+  if (!encode_rows_map(&maps.q, Qp, H, N, d) || !encode_rows_map(&maps.k, Kp, H, N, d) ||
+      !encode_rows_map(&maps.v, Vp, H, N, d) || !encode_rows_map(&maps.kt, k_tilde, H, nkb, d) ||
+      !encode_rows_map(&maps.vt, v_tilde, H, nkb, d))
+    return SPARK_ERR_CUDA;
+  if (nc > 0) {
+    if (!encode_rows_map(&maps.kc, Kc, H, nc, d) || !encode_rows_map(&maps.vc, Vc, H, nc, d))
+      return SPARK_ERR_CUDA;
+  } else {
+    maps.kc = maps.k;                            // never loaded: the kernel has no context tile
+    maps.vc = maps.v;
+  }
+  return from_cuda(launch_attend_fused(maps, nc, cbias, qbar_blocks, kbar, k, q_perm, q_offsets,
+                                       nqb, k_offsets, nkb, H, N, d, out, out_dtype, err, sel_out,
+                                       s));
+}
+
 // FP8 logits: e4m3 Qp8/Kp8/kt8/Kc8 with their group scales, bf16 values.
 spark_status attend_fp8_impl(const void* Qp8, const float* q_scale, const void* Kp8,
                              const float* k_scale, const void* Vp, const void* kt8,
@@ -217,7 +244,7 @@ spark_status forward_impl(const void* Q, const void* K, const void* V, const voi
                           const int32_t* q_block_offsets, int nqb,
                           const int32_t* k_block_offsets, int nkb, double topk_ratio, void* out,
                           void* workspace, size_t workspace_bytes, cudaStream_t s,
-                          bool fp8 = false) {
+                          bool fp8 = false, bool fused = false) {
   if (!Q || !K || !V || !q_perm || !k_perm || !q_block_offsets || !k_block_offsets || !out)
     return SPARK_ERR_INVALID_ARG;
   if (dtype != SPARK_BF16 && dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
@@ -229,6 +256,7 @@ spark_status forward_impl(const void* Q, const void* K, const void* V, const voi
   if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16))
     return SPARK_ERR_INVALID_ARG;
   if (fp8 && d != 128) return SPARK_ERR_UNSUPPORTED;
+  if (fused && (fp8 || !attend_fused_supported(d, nkb, L.k))) return SPARK_ERR_UNSUPPORTED;
   const size_t cbytes = nc > 0 ? context_bytes(H, nc, d) : 0;
   const size_t fp8_bytes = fp8 ? fp8_layout(H, N, d, nqb, nkb, nc).total : 0;
   if (workspace == nullptr || workspace_bytes < L.total + 2 * cbytes + fp8_bytes ||
@@ -258,7 +286,7 @@ spark_status forward_impl(const void* Q, const void* K, const void* V, const voi
   if (launch_gather_kv_summary(K, V, dtype, H, N, d, k_perm, k_block_offsets, nkb, qbar, Kp, Vp,
                                kbar, kt, vt, cbias, err, s) != cudaSuccess)
     return SPARK_ERR_CUDA;
-  if (launch_route(qbar_blocks, kbar, H, nqb, nkb, d, L.k, sel, err, s) != cudaSuccess)
+  if (!fused && launch_route(qbar_blocks, kbar, H, nqb, nkb, d, L.k, sel, err, s) != cudaSuccess)
     return SPARK_ERR_CUDA;
   const void* Kca = Kc;                          // bf16 context rows are read in place
   const void* Vca = Vc;
@@ -270,6 +298,10 @@ spark_status forward_impl(const void* Q, const void* K, const void* V, const voi
     Kca = Kcb;
     Vca = Vcb;
   }
+  if (fused)   // the selection is made inside the attention kernel and copied to the workspace
+    return attend_fused_impl(Qp, Kp, Vp, kt, vt, cbias, qbar_blocks, kbar, L.k, Kca, Vca, nc,
+                             q_perm, q_block_offsets, nqb, k_block_offsets, nkb, H, N, d, out,
+                             dtype, err, sel, s);
   if (!fp8)
     return attend_impl(Qp, Kp, Vp, kt, vt, cbias, sel, L.k, Kca, Vca, nc, q_perm,
                        q_block_offsets, nqb, k_block_offsets, nkb, H, N, d, out, dtype, err, s);
@@ -499,6 +531,46 @@ spark_status spark_bsa_forward(const void* Q, const void* K, const void* V, int 
   return forward_impl(Q, K, V, nullptr, nullptr, 0, dtype, H, N, d, q_perm, k_perm,
                       q_block_offsets, nqb, k_block_offsets, nkb, topk_ratio, out, workspace,
                       workspace_bytes, as_stream(stream));
+}
+
+// ------------------------------------------------------- routing inside the attention kernel
+
+int spark_bsa_fused_supported(int d, int nkb, double topk_ratio) {
+  const int k = topk_count(nkb, topk_ratio);
+  return (k >= 1 && nkb >= 1 && nkb <= kMaxNkb && attend_fused_supported(d, nkb, k)) ? 1 : 0;
+}
+
+spark_status spark_bsa_forward_fused(const void* Q, const void* K, const void* V, int dtype,
+                                     int H, int N, int d, const int32_t* q_perm,
+                                     const int32_t* k_perm, const int32_t* q_block_offsets,
+                                     int nqb, const int32_t* k_block_offsets, int nkb,
+                                     double topk_ratio, void* out, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  return forward_impl(Q, K, V, nullptr, nullptr, 0, dtype, H, N, d, q_perm, k_perm,
+                      q_block_offsets, nqb, k_block_offsets, nkb, topk_ratio, out, workspace,
+                      workspace_bytes, as_stream(stream), false, true);
+}
+
+spark_status spark_bsa_attend_fused(const void* Qp, const void* Kp, const void* Vp,
+                                    const void* k_tilde, const void* v_tilde, const float* cbias,
+                                    const float* qbar_blocks, const float* kbar, int k,
+                                    const int32_t* q_perm, const int32_t* q_block_offsets,
+                                    int nqb, const int32_t* k_block_offsets, int nkb, int H,
+                                    int N, int d, void* out, int out_dtype, int32_t* sel_out,
+                                    uint32_t* err, void* stream) {
+  if (!Qp || !Kp || !Vp || !k_tilde || !v_tilde || !cbias || !qbar_blocks || !kbar ||
+      !q_perm || !q_block_offsets || !k_block_offsets || !out)
+    return SPARK_ERR_INVALID_ARG;
+  if (out_dtype != SPARK_BF16 && out_dtype != SPARK_F32) return SPARK_ERR_INVALID_ARG;
+  spark_status st = check_sizes(H, N, d, nqb, nkb);
+  if (st != SPARK_OK) return st;
+  if (k < 1 || k > nkb) return SPARK_ERR_INVALID_ARG;
+  if (!aligned(Qp, 16) || !aligned(Kp, 16) || !aligned(Vp, 16) || !aligned(k_tilde, 16) ||
+      !aligned(v_tilde, 16) || !aligned(out, 16))
+    return SPARK_ERR_INVALID_ARG;
+  return attend_fused_impl(Qp, Kp, Vp, k_tilde, v_tilde, cbias, qbar_blocks, kbar, k, nullptr,
+                           nullptr, 0, q_perm, q_block_offsets, nqb, k_block_offsets, nkb, H, N,
+                           d, out, out_dtype, err, sel_out, as_stream(stream));
 }
 
 // ----------------------------------------------------------- threshold routing (comparator)

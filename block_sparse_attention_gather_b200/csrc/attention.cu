@@ -43,6 +43,7 @@
 // Every wait is bounded by the launch parameter wait_ns (the library's process-wide setting,
 // 4 s by default); on expiry the kernel flags kErrTimeout, stops every role, drains the copies
 // and MMAs it issued (waits bounded by the default limit), frees TMEM and returns.
+#include "route_step.cuh"
 #include "spark_kernels.cuh"
 
 namespace spark {
@@ -211,10 +212,6 @@ __device__ __forceinline__ float max64(const float (&x)[64]) {
   return fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
 }
 
-// Every kPolyEvery-th pair of exponentials is computed on the FMA pipe (exp2_poly_x2) instead
-// of MUFU, whose throughput per SM matches the tensor cores' for this tile shape (0: none).
-constexpr int kPolyEvery = 0;
-
 // p = 2^(x*c - m) for the 32 columns x[j0 .. j0+31], packed to bf16 pairs; returns their sum.
 __device__ __forceinline__ float exp32_at(const float (&x)[64], int j0, float c, float m,
                                           uint32_t (&pk)[16]) {
@@ -224,15 +221,9 @@ __device__ __forceinline__ float exp32_at(const float (&x)[64], int j0, float c,
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const uint64_t a2 = f2_fma(f2_pack(x[j0 + 2 * j], x[j0 + 2 * j + 1]), c2, nm2);
-    float p0, p1;
-    if (kPolyEvery > 0 && j % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
-      f2_unpack(exp2_poly_x2(a2), p0, p1);
-    } else {
-      float a0, a1;
-      f2_unpack(a2, a0, a1);
-      p0 = ex2_approx(a0);
-      p1 = ex2_approx(a1);
-    }
+    float a0, a1;
+    f2_unpack(a2, a0, a1);
+    const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
     sum2[j & 1] = f2_add(sum2[j & 1], f2_pack(p0, p1));
     pk[j] = pack_bf16(p0, p1);
   }
@@ -243,7 +234,7 @@ __device__ __forceinline__ float exp32_at(const float (&x)[64], int j0, float c,
 
 }  // namespace
 
-template <int D, bool kBiasSmem, bool kFp8>
+template <int D, bool kBiasSmem, bool kFp8, bool kFused, bool kVarTiles>
 __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kt,
@@ -253,8 +244,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     const int32_t* __restrict__ q_perm,
     const int32_t* __restrict__ q_offsets, int nqb, const int32_t* __restrict__ k_offsets,
     int nkb, int N, void* __restrict__ out, int out_dtype, uint32_t* err, const Fp8Scales sc,
-    uint64_t wait_ns) {
+    uint64_t wait_ns, int H, const float* __restrict__ qbar_blocks,
+    const float* __restrict__ kbar, int32_t* __restrict__ sel_out) {
   static_assert(!kFp8 || D == 128, "FP8 logits: d = 128 (one 128-byte row per key)");
+  static_assert(!kFused || (kBiasSmem && !kFp8), "in-kernel routing: bf16, bias row in smem");
   constexpr int QK_BYTES = 128 * D * (kFp8 ? 1 : 2);   // one Q or K tile
   constexpr int V_BYTES = 128 * D * 2;                 // one V tile (bf16)
   constexpr int QK_ATOMS = kFp8 ? 1 : D / 64;          // 128-byte swizzle atoms across a row
@@ -269,13 +262,39 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   Barriers* bars = reinterpret_cast<Barriers*>(vst + kVStages * V_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint32_t* selmask = reinterpret_cast<uint32_t*>(tmem_slot + 4);
-  // summary-row offsets of this CTA in log2 units, -inf for selected blocks and padding
-  // (16-byte aligned explicitly: the softmax reads it with float4 loads)
-  float* biasrow = reinterpret_cast<float*>(
-      (reinterpret_cast<uintptr_t>(selmask + (nkb + 31) / 32) + 15) & ~static_cast<uintptr_t>(15));
+  // Per query block: a bit per selected key block and the summary-row offsets in log2 units
+  // (-inf for selected blocks and padding; 16-byte aligned: the softmax reads them with float4
+  // loads).  With in-kernel routing there are two of each plus the selection itself: the
+  // current query block's and the next one's, which the K producer routes meanwhile.
+  const int nwords = (nkb + 31) / 32;
+  const int nbias = kBiasSmem ? (nkb + 127) / 128 * 128 : 0;
+  uint32_t* selmask_b[2];
+  float* biasrow_b[2];
+  int32_t* sel_s_b[2] = {nullptr, nullptr};
+  RouteSmem rsm{nullptr, nullptr, nullptr};
+  {
+    uint8_t* p = reinterpret_cast<uint8_t*>(tmem_slot + 4);
+    auto carve = [&](size_t bytes) {
+      p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15));
+      uint8_t* at = p;
+      p += bytes;
+      return at;
+    };
+    for (int b = 0; b < (kFused ? 2 : 1); ++b) {
+      selmask_b[b] = reinterpret_cast<uint32_t*>(carve(static_cast<size_t>(nwords) * 4));
+      biasrow_b[b] = reinterpret_cast<float*>(carve(static_cast<size_t>(nbias) * 4));
+    }
+    if (kFused) {
+      for (int b = 0; b < 2; ++b) sel_s_b[b] = reinterpret_cast<int32_t*>(carve(kcap * 4u));
+      rsm.keys = reinterpret_cast<uint32_t*>(carve(static_cast<size_t>(nkb) * 4));
+      rsm.hist = reinterpret_cast<uint32_t*>(carve(256 * 4));
+      rsm.qn = reinterpret_cast<float*>(carve(D * 4));
+    } else {
+      selmask_b[1] = selmask_b[0];
+      biasrow_b[1] = biasrow_b[0];
+    }
+  }
 
-  const int A = blockIdx.x, h = blockIdx.y;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   __shared__ int s_skip, s_rerun;
   // [group][row]: first-tile maxima (the reference), then sums and maxima for the epilogue
@@ -286,16 +305,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   }
   __syncthreads();
   if (s_skip) return;                                      // uniform: no work, nothing held
-  // selected blocks of this query block: kcap, or its own count (threshold routing) when
-  // sel_count is given; rows of sel are kcap apart either way
-  const int k = sel_count ? max(0, min(sel_count[static_cast<size_t>(h) * nqb + A], kcap)) : kcap;
-  const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
+  // Query blocks of this CTA: one, (blockIdx.x, blockIdx.y), or with in-kernel routing every
+  // gridDim.x-th of the H*nqb (head-major) starting at blockIdx.x.
+  const int n_items = kFused ? H * nqb : 1;
+  int item = kFused ? static_cast<int>(blockIdx.x) : 0;
+  if (kFused && item >= n_items) return;
   const int nxt = (nc + 127) / 128;                 // context tiles
-  const int T = k + nxt + nct;
-  const int32_t* sel_row = sel + (static_cast<size_t>(h) * nqb + A) * kcap;
-  const int nwords = (nkb + 31) / 32;
-  const float* cb = cbias + static_cast<size_t>(h) * nkb;
-  const int qlo = q_offsets[A];
 
   if (tid == 0) {
     mbar_init(&bars->qfull, 1);
@@ -312,10 +327,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     *abort_flag = 0;
     mbar_fence_init();
   }
-  for (int i = tid; i < nwords; i += kThreads) selmask[i] = 0u;
-  if (kBiasSmem)
-    for (int i = tid; i < nct * 128; i += kThreads)
-      biasrow[i] = (i < nkb) ? cb[i] * kLog2e : -INFINITY;
+  if (!kFused) {
+    // the selection comes from the routing kernel: build the mask and the bias row from it
+    const int h = blockIdx.y;
+    const int k = sel_count ? max(0, min(sel_count[static_cast<size_t>(h) * nqb + blockIdx.x], kcap))
+                            : kcap;
+    const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
+    const float* cb = cbias + static_cast<size_t>(h) * nkb;
+    for (int i = tid; i < nwords; i += kThreads) selmask_b[0][i] = 0u;
+    if (kBiasSmem)
+      for (int i = tid; i < nct * 128; i += kThreads)
+        biasrow_b[0][i] = (i < nkb) ? cb[i] * kLog2e : -INFINITY;
+  }
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -323,17 +346,52 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  for (int i = tid; i < k; i += kThreads) {
-    const int B = sel_row[i];
-    if (B >= 0 && B < nkb) {
-      atomicOr(&selmask[B >> 5], 1u << (B & 31));
-      if (kBiasSmem) biasrow[B] = -INFINITY;
-    } else {
-      flag_error(err, kErrSel);
+  if (!kFused) {
+    const int h = blockIdx.y, A = blockIdx.x;
+    const int k = sel_count ? max(0, min(sel_count[static_cast<size_t>(h) * nqb + A], kcap)) : kcap;
+    const int32_t* srow = sel + (static_cast<size_t>(h) * nqb + A) * kcap;
+    for (int i = tid; i < k; i += kThreads) {
+      const int B = srow[i];
+      if (B >= 0 && B < nkb) {
+        atomicOr(&selmask_b[0][B >> 5], 1u << (B & 31));
+        if (kBiasSmem) biasrow_b[0][B] = -INFINITY;
+      } else {
+        flag_error(err, kErrSel);
+      }
     }
+  }
+  // In-kernel routing: the K producer routes this CTA's first query block before any tile.
+  RouteJob job = route_job_none();
+  if (kFused && warp == kWarpK) {
+    job = route_job(item / nqb, item % nqb, 0);
+    while (job.stage != kRjDone)
+      route_step<D>(job, rsm, qbar_blocks, kbar, cbias, nqb, nkb, kcap, sel_s_b[0],
+                    selmask_b[0], biasrow_b[0], sel_out, lane);
   }
   __syncthreads();
   const uint32_t tbase = *tmem_slot;
+  // Barrier phases count over the CTA's whole life: tiles (both passes of every query block),
+  // passes (the `done` barrier) and query blocks (the Q tile).
+  int tiles_base = 0, passes_base = 0, items_done = 0;
+  int issued = 0;                                  // producers: loads issued so far
+  for (int cur = 0;; cur ^= 1) {
+  const int A = kFused ? item % nqb : static_cast<int>(blockIdx.x);
+  const int h = kFused ? item / nqb : static_cast<int>(blockIdx.y);
+  // selected blocks of this query block: kcap, or its own count (threshold routing) when
+  // sel_count is given; rows of sel are kcap apart either way
+  const int k = sel_count ? max(0, min(sel_count[static_cast<size_t>(h) * nqb + A], kcap)) : kcap;
+  const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
+  const int T = k + nxt + nct;
+  const int32_t* sel_row = kFused ? sel_s_b[cur] : sel + (static_cast<size_t>(h) * nqb + A) * kcap;
+  const float* cb = cbias + static_cast<size_t>(h) * nkb;
+  const uint32_t* selmask = selmask_b[cur];
+  const float* biasrow = biasrow_b[cur];
+  const int qlo = q_offsets[A];
+  if (kFused && warp == kWarpK) {
+    // route the CTA's next query block into the other buffers while this one is attended
+    const int nitem = item + static_cast<int>(gridDim.x);
+    job = nitem < n_items ? route_job(nitem / nqb, nitem % nqb, cur ^ 1) : route_job_none();
+  }
 
   // Pass 0 exponentiates every tile against a fixed reference per row (the larger of the two
   // groups' first-tile maxima) and records the maximum of every chunk whose sum is out of
@@ -343,9 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   float m_true = -INFINITY;                        // softmax threads: row maximum (log2 units)
   float m_ref0 = 0.f;                              //   pass 0's reference of the row
   bool rerun_row = false;                          //   the row left the window in pass 0
-  int issued = 0;                                  // producers: loads issued over both passes
+  int npasses = 1;
   for (int pass = 0; pass < 2; ++pass) {
-    const int tg0 = pass * T;                      // tile counter of this pass's first tile
+    const int tg0 = tiles_base + pass * T;         // tile counter of this pass's first tile
+    const uint32_t done_par = static_cast<uint32_t>(passes_base + pass) & 1u;
     if (warp == kWarpK || warp == kWarpV) {
       // ----------------------------------------------------------- TMA producers
       // The whole warp runs the loop (warp-uniform stage indices and coordinates); one elected
@@ -391,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
                                         wait_ns)))
           break;
         if (elect_one()) {
-          if (is_k) bars->kn[s] = static_cast<uint32_t>(tile_cols(ti));   // before the arrive
+          if (kVarTiles && is_k) bars->kn[s] = static_cast<uint32_t>(tile_cols(ti));   // before the arrive
           mbar_arrive_expect_tx(&full[s], tile_bytes);
           const CUtensorMap* map = ti.src == kSrcVideo ? mx : (ti.src == kSrcContext ? mc : ms);
           for (int a = 0; a < atoms; ++a)
@@ -401,12 +460,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         issued = tg + 1;
         if (t + 1 < T)
           next = tile_info<false>(t + 1, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
+        // one bounded step of the next query block's routing per K tile
+        if (kFused && is_k && job.stage != kRjDone)
+          route_step<D>(job, rsm, qbar_blocks, kbar, cbias, nqb, nkb, kcap, sel_s_b[job.buf],
+                        selmask_b[job.buf], biasrow_b[job.buf], sel_out, lane);
       }
       // every load this pass issued has landed before the pass ends (after an abort some were
       // never consumed; otherwise these phases are complete already and the waits return at once)
       for (int tg = max(tg0, issued - stages); tg < issued; ++tg)
         wait_bounded_ignore_abort(&full[tg % stages], (tg / stages) & 1);
-      if (is_k) wait_bounded_ignore_abort(&bars->qfull, 0);
+      if (is_k) wait_bounded_ignore_abort(&bars->qfull, items_done & 1);
     } else if (warp == kWarpMma) {
       // ---------------------------------------------------------------- MMA issuer
       // The whole warp runs the issue loop, so stage indices and descriptors are warp-uniform
@@ -421,7 +484,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       const uint64_t qd = sdesc_sw128(smem_u32(qst), 16, 1024);
       const uint64_t kdesc0 = sdesc_sw128(smem_u32(kst), 16, 1024);
       const uint64_t vdesc0 = sdesc_sw128(smem_u32(vst), 16384, 1024);
-      bool ok = pass > 0 || __all_sync(kAll, mbar_wait(&bars->qfull, 0, abort_flag, err, wait_ns));
+      bool ok = pass > 0 ||
+                __all_sync(kAll, mbar_wait(&bars->qfull, items_done & 1, abort_flag, err, wait_ns));
       // S(t) of this pass into buffer (tg0 + t) % 3
       auto issue_s = [&](int t) -> bool {
         const int tg = tg0 + t;
@@ -431,11 +495,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
           return false;
         const uint32_t dcol = tbase + (tg % 3) * 128;
         const uint64_t kd = kdesc0 + static_cast<uint64_t>(s * (QK_BYTES >> 4));
-        // S covers the tile's keys only (N = its valid rows rounded up to 16)
-        const uint32_t ncols = bars->kn[s];
+        // variable tiles: S covers the tile's keys only (N = its valid rows rounded up to 16)
+        const uint32_t ncols = kVarTiles ? bars->kn[s] : 128u;
         const uint32_t idSn = idS_base | ((ncols >> 3) << 17);
         if (elect_one()) {
-          bars->bn[tg % 3] = ncols;
+          if (kVarTiles) bars->bn[tg % 3] = ncols;
           if constexpr (kFp8) {
             // 32 e4m3 values of d = 32 bytes per MMA, all inside the one 128-byte atom row
 #pragma unroll
@@ -468,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         const uint32_t pcol = tbase + (tg % 3) * 128;               // P(t) over S(t)
         if (elect_one()) {
           // the tile's keys only, 16 per MMA (P past them is never read)
-          const int nk = static_cast<int>(bars->bn[tg % 3] >> 4);
+          const int nk = kVarTiles ? static_cast<int>(bars->bn[tg % 3] >> 4) : 8;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             if (kk < nk)
@@ -484,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       // every MMA complete: the softmax epilogue reads O, and TMEM is reused or freed after
       if (elect_one()) tc_commit(&bars->done);
       __syncwarp();
-      wait_bounded_ignore_abort(&bars->done, pass);
+      wait_bounded_ignore_abort(&bars->done, done_par);
     } else {
       // ---------------------------------------------------------------- softmax rows
       const int q4 = warp & 3, grp = warp >> 2;          // row quarter, tile group
@@ -546,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         // and cannot drive the row sum out of [2^-60, 2^60] (fewer than 2^16 chunks per row),
         // so only chunks outside that range (rare) take their maximum.
         // only the columns the MMAs covered (exact tiles: the valid rows rounded up to 16)
-        const int ncols = tile_cols(ti);
+        const int ncols = kVarTiles ? tile_cols(ti) : 128;
         float rowsum = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -579,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       }
       // ---- epilogue: O / (l_0 + l_1), scattered to the original token order
       bool fine = ok && T > 0;
-      if (fine) fine = __all_sync(0xffffffffu, mbar_wait(&bars->done, pass, abort_flag, err, wait_ns));
+      if (fine) fine = __all_sync(0xffffffffu, mbar_wait(&bars->done, done_par, abort_flag, err, wait_ns));
       ex_l[grp][row] = l_run;
       ex_mt[grp][row] = m_true;
       named_bar_sync(1 + q4, 64);
@@ -637,6 +701,24 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     __syncthreads();
     tc_fence_after_sync();
     if (pass == 1 || !s_rerun || *abort_flag) break;   // uniform: written before the barrier
+    npasses = 2;
+  }
+  tiles_base += npasses * T;
+  passes_base += npasses;
+  ++items_done;
+  if (!kFused) break;
+  // the next query block's routing completes before it starts (few tiles, or an abort)
+  if (warp == kWarpK)
+    while (job.stage != kRjDone && !*abort_flag)
+      route_step<D>(job, rsm, qbar_blocks, kbar, cbias, nqb, nkb, kcap, sel_s_b[job.buf],
+                    selmask_b[job.buf], biasrow_b[job.buf], sel_out, lane);
+  if (tid == 0) {
+    s_rerun = 0;
+    s_skip = launch_timed_out(err) ? 1 : 0;
+  }
+  __syncthreads();
+  item += static_cast<int>(gridDim.x);
+  if (*abort_flag || s_skip || item >= n_items) break;   // uniform: written before the barrier
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -651,16 +733,33 @@ static bool bias_in_smem(int nkb, int k) {
   return nct > 0 && nct * 128 <= kMaxSmemBias;
 }
 
-static size_t attend_smem_bytes(int d, int nkb, int k, bool fp8) {
+static size_t align16(size_t b) { return (b + 15) & ~static_cast<size_t>(15); }
+
+// Dynamic shared memory of a launch: 1 KB of alignment slack, the Q tile, the K and V rings,
+// the barriers, then (16-byte aligned each) the selection mask and bias row of one query block,
+// or with in-kernel routing two of each plus two selections, the routing keys, a histogram and
+// the query-block mean.
+static size_t attend_smem_bytes(int d, int nkb, int k, bool fp8, bool fused = false) {
   const size_t qk = static_cast<size_t>(128) * d * (fp8 ? 1 : 2);
   const size_t v = static_cast<size_t>(128) * d * 2;
-  const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
-  const size_t words = (nkb + 31) / 32 + 4;          // + 16 bytes of alignment slack
-  const size_t bias = bias_in_smem(nkb, k) ? static_cast<size_t>(nct) * 128 * 4 : 0;
-  return 1024 + (1 + kKStages) * qk + kVStages * v + sizeof(Barriers) + 16 + words * 4 + bias;
+  const size_t words = static_cast<size_t>((nkb + 31) / 32) * 4;
+  const size_t bias = bias_in_smem(nkb, k) || fused ? static_cast<size_t>((nkb + 127) / 128) * 128 * 4
+                                                    : 0;
+  size_t b = 1024 + (1 + kKStages) * qk + kVStages * v + sizeof(Barriers) + 16;
+  const int nbuf = fused ? 2 : 1;
+  b += nbuf * (align16(words) + 16 + align16(bias) + 16);
+  if (fused) b += 2 * (align16(static_cast<size_t>(k) * 4) + 16) +
+                  align16(static_cast<size_t>(nkb) * 4) + 16 + 256 * 4 + 16 + d * 4 + 16;
+  return b;
 }
 
-template <int D, bool kBiasSmem, bool kFp8>
+constexpr size_t kSmemLimit = 232448;   // 227 KB of opt-in shared memory per CTA
+
+// All key blocks hold exactly 128 tokens (sizes are 1..128 and sum to N) - then every exact
+// tile is a full MMA tile and the kernel without per-tile widths runs.
+static bool all_blocks_full(int N, int nkb) { return static_cast<long long>(nkb) * 128 == N; }
+
+template <int D, bool kBiasSmem, bool kFp8, bool kVar>
 static cudaError_t launch_attend_t(const AttendMaps& m, int nc, const float* cbias,
                                    const int32_t* sel, int k, const int32_t* sel_count,
                                    const int32_t* q_perm, const int32_t* q_offsets,
@@ -669,15 +768,32 @@ static cudaError_t launch_attend_t(const AttendMaps& m, int nc, const float* cbi
                                    cudaStream_t s) {
   // with per-row counts any row may have summary tiles: size for k < nkb
   const size_t smem = attend_smem_bytes(D, nkb, sel_count ? 0 : k, kFp8);
-  cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, kBiasSmem, kFp8>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = attend_kernel<D, kBiasSmem, kFp8, false, kVar>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(nqb, H);
-  attend_kernel<D, kBiasSmem, kFp8><<<grid, kThreads, smem, s>>>(
-      m.q, m.k, m.v, m.kt, m.vt, m.kc, m.vc, nc, cbias, sel, k, sel_count, q_perm, q_offsets,
-      nqb, k_offsets, nkb, N, out, out_dtype, err, sc, wait_limit_ns());
+  kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.kt, m.vt, m.kc, m.vc, nc, cbias, sel, k,
+                                    sel_count, q_perm, q_offsets, nqb, k_offsets, nkb, N, out,
+                                    out_dtype, err, sc, wait_limit_ns(), H, nullptr, nullptr,
+                                    nullptr);
   return cudaGetLastError();
+}
+
+template <int D, bool kBiasSmem, bool kFp8>
+static cudaError_t launch_attend_v(const AttendMaps& m, int nc, const float* cbias,
+                                   const int32_t* sel, int k, const int32_t* sel_count,
+                                   const int32_t* q_perm, const int32_t* q_offsets,
+                                   int nqb, const int32_t* k_offsets, int nkb, int H, int N,
+                                   void* out, int out_dtype, uint32_t* err, const Fp8Scales& sc,
+                                   cudaStream_t s) {
+  return all_blocks_full(N, nkb)
+             ? launch_attend_t<D, kBiasSmem, kFp8, false>(m, nc, cbias, sel, k, sel_count, q_perm,
+                                                          q_offsets, nqb, k_offsets, nkb, H, N,
+                                                          out, out_dtype, err, sc, s)
+             : launch_attend_t<D, kBiasSmem, kFp8, true>(m, nc, cbias, sel, k, sel_count, q_perm,
+                                                         q_offsets, nqb, k_offsets, nkb, H, N,
+                                                         out, out_dtype, err, sc, s);
 }
 
 cudaError_t launch_attend(const AttendMaps& maps, int nc, const float* cbias,
@@ -688,16 +804,16 @@ cudaError_t launch_attend(const AttendMaps& maps, int nc, const float* cbias,
   const bool bs = bias_in_smem(nkb, sel_count ? 0 : k);
   const Fp8Scales none{nullptr, nullptr, nullptr, nullptr};
   if (d == 128)
-    return bs ? launch_attend_t<128, true, false>(maps, nc, cbias, sel, k, sel_count, q_perm,
+    return bs ? launch_attend_v<128, true, false>(maps, nc, cbias, sel, k, sel_count, q_perm,
                                                   q_offsets, nqb, k_offsets, nkb, H, N, out,
                                                   out_dtype, err, none, s)
-              : launch_attend_t<128, false, false>(maps, nc, cbias, sel, k, sel_count, q_perm,
+              : launch_attend_v<128, false, false>(maps, nc, cbias, sel, k, sel_count, q_perm,
                                                    q_offsets, nqb, k_offsets, nkb, H, N, out,
                                                    out_dtype, err, none, s);
-  return bs ? launch_attend_t<64, true, false>(maps, nc, cbias, sel, k, sel_count, q_perm,
+  return bs ? launch_attend_v<64, true, false>(maps, nc, cbias, sel, k, sel_count, q_perm,
                                                q_offsets, nqb, k_offsets, nkb, H, N, out,
                                                out_dtype, err, none, s)
-            : launch_attend_t<64, false, false>(maps, nc, cbias, sel, k, sel_count, q_perm,
+            : launch_attend_v<64, false, false>(maps, nc, cbias, sel, k, sel_count, q_perm,
                                                 q_offsets, nqb, k_offsets, nkb, H, N, out,
                                                 out_dtype, err, none, s);
 }
@@ -711,12 +827,56 @@ cudaError_t launch_attend_fp8(const AttendMaps& maps, const float* q_scale,
                               cudaStream_t s) {
   const Fp8Scales sc{q_scale, k_scale, kt_scale, kc_scale};
   return bias_in_smem(nkb, k)
-             ? launch_attend_t<128, true, true>(maps, nc, cbias, sel, k, nullptr, q_perm,
+             ? launch_attend_v<128, true, true>(maps, nc, cbias, sel, k, nullptr, q_perm,
                                                 q_offsets, nqb, k_offsets, nkb, H, N, out,
                                                 out_dtype, err, sc, s)
-             : launch_attend_t<128, false, true>(maps, nc, cbias, sel, k, nullptr, q_perm,
+             : launch_attend_v<128, false, true>(maps, nc, cbias, sel, k, nullptr, q_perm,
                                                  q_offsets, nqb, k_offsets, nkb, H, N, out,
                                                  out_dtype, err, sc, s);
+}
+
+bool attend_fused_supported(int d, int nkb, int k) {
+  return d == 128 && k < nkb && bias_in_smem(nkb, k) &&
+         attend_smem_bytes(d, nkb, k, false, true) <= kSmemLimit;
+}
+
+template <bool kVar>
+static cudaError_t launch_fused_t(const AttendMaps& m, int nc, const float* cbias,
+                                  const float* qbar_blocks, const float* kbar, int k,
+                                  const int32_t* q_perm, const int32_t* q_offsets, int nqb,
+                                  const int32_t* k_offsets, int nkb, int H, int N, void* out,
+                                  int out_dtype, uint32_t* err, int32_t* sel_out,
+                                  cudaStream_t s) {
+  const size_t smem = attend_smem_bytes(128, nkb, k, false, true);
+  auto kern = attend_kernel<128, true, false, true, kVar>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int dev = 0, nsm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  const long long items = static_cast<long long>(H) * nqb;
+  const int grid = static_cast<int>(items < nsm ? items : nsm);   // one persistent CTA per SM
+  const Fp8Scales none{nullptr, nullptr, nullptr, nullptr};
+  kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.kt, m.vt, m.kc, m.vc, nc, cbias, nullptr, k,
+                                    nullptr, q_perm, q_offsets, nqb, k_offsets, nkb, N, out,
+                                    out_dtype, err, none, wait_limit_ns(), H, qbar_blocks, kbar,
+                                    sel_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attend_fused(const AttendMaps& maps, int nc, const float* cbias,
+                                const float* qbar_blocks, const float* kbar, int k,
+                                const int32_t* q_perm, const int32_t* q_offsets, int nqb,
+                                const int32_t* k_offsets, int nkb, int H, int N, int d, void* out,
+                                int out_dtype, uint32_t* err, int32_t* sel_out, cudaStream_t s) {
+  if (!attend_fused_supported(d, nkb, k)) return cudaErrorInvalidValue;
+  return all_blocks_full(N, nkb)
+             ? launch_fused_t<false>(maps, nc, cbias, qbar_blocks, kbar, k, q_perm, q_offsets,
+                                     nqb, k_offsets, nkb, H, N, out, out_dtype, err, sel_out, s)
+             : launch_fused_t<true>(maps, nc, cbias, qbar_blocks, kbar, k, q_perm, q_offsets,
+                                    nqb, k_offsets, nkb, H, N, out, out_dtype, err, sel_out, s);
 }
 
 }  // namespace spark

@@ -11,13 +11,11 @@
 //            load is a warp-wide broadcast of four rows.  The scores of the R
 //            rows stay in shared memory as order-preserving uint32 keys.  The positive factor
 //            1/sqrt(d) is left out: it does not change the order.
-//   phase 2  one warp per row: an exact radix select (up to four 8-bit passes over the keys,
-//            histogram updates aggregated over the lanes that share a digit) finds the k-th
-//            largest key T and how many keys equal to T are still needed; it stops early once
-//            every key under the digits found so far is needed, comparing keys on those digits
-//            only.  A ballot scan in ascending block order then writes every B with key > T
-//            and the lowest-indexed keys == T, so the selection is stored ascending and ties go
-//            to the smaller block index.
+//   phase 2  one warp per row: an exact radix select (four 8-bit passes over the keys) finds
+//            the k-th largest key T and how many keys equal to T are still needed; a ballot
+//            scan in ascending block order then writes every B with key > T and the
+//            lowest-indexed keys == T, so the selection is stored ascending and ties go to
+//            the smaller block index.
 #include "spark_kernels.cuh"
 
 namespace spark {
@@ -181,15 +179,9 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(const float* __restr
       for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = lane; i < 256; i += 32) wh[i] = 0;
         __syncwarp();
-        // lanes holding the same digit add once, with their count (scores of a row share
-        // their top bits, so most lanes of a step fall into one or two bins)
-        for (int B0 = 0; B0 < nkb; B0 += 32) {
-          const int B = B0 + lane;
-          const uint32_t u = krow[min(B, nkb - 1)];
-          const bool in = B < nkb && (u & pmask) == prefix;
-          const uint32_t dig = in ? (u >> shift) & 255u : 256u + lane;
-          const uint32_t same = __match_any_sync(0xffffffffu, dig);
-          if (in && lane == __ffs(same) - 1) atomicAdd(&wh[dig], static_cast<uint32_t>(__popc(same)));
+        for (int B = lane; B < nkb; B += 32) {
+          const uint32_t u = krow[B];
+          if ((u & pmask) == prefix) atomicAdd(&wh[(u >> shift) & 255u], 1u);
         }
         __syncwarp();
         // lane l owns digits [8l, 8l+8); suffix sums give count(digit >= x)
@@ -224,20 +216,16 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(const float* __restr
         prefix |= static_cast<uint32_t>(dd) << shift;
         pmask |= 255u << shift;
         __syncwarp();
-        // every key left under the prefix is taken: the remaining bits cannot change the set
-        if (static_cast<uint32_t>(need) == wh[dd]) break;
       }
     } else {
       prefix = 0;                      // k == nkb: every key is taken
       need = nkb;
     }
-    // keys compared on the prefix's bits: above it taken, equal to it taken in ascending block
-    // order until `need` (the lowest-indexed ties), below it left
     const uint32_t T = prefix;
     int taken = 0, eq_seen = 0;
     for (int B0 = 0; B0 < nkb; B0 += 32) {
       const int B = B0 + lane;
-      const uint32_t u = ((B < nkb) ? krow[B] : 0u) & pmask;
+      const uint32_t u = (B < nkb) ? krow[B] : 0u;
       const bool valid = B < nkb;
       const bool gt = valid && (kr == nkb || u > T);
       const bool eq = valid && kr < nkb && u == T;

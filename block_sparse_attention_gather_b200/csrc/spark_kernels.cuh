@@ -61,6 +61,17 @@ cudaError_t launch_attend(const AttendMaps& maps, int nc, const float* cbias,
                           int H, int N, int d, void* out, int out_dtype, uint32_t* err,
                           cudaStream_t s, const int32_t* sel_count = nullptr);
 
+// The attention with the routing inside (d = 128, bf16, Top-K): one persistent CTA per SM
+// walks the query blocks head-major; its K producer scores and selects the next query block
+// (from qbar_blocks [H,nqb,d] and kbar [H,d,nkb], the routing kernel's arithmetic) while the
+// current one is attended.  sel_out (optional [H,nqb,k]) receives a copy of every selection.
+bool attend_fused_supported(int d, int nkb, int k);
+cudaError_t launch_attend_fused(const AttendMaps& maps, int nc, const float* cbias,
+                                const float* qbar_blocks, const float* kbar, int k,
+                                const int32_t* q_perm, const int32_t* q_offsets, int nqb,
+                                const int32_t* k_offsets, int nkb, int H, int N, int d, void* out,
+                                int out_dtype, uint32_t* err, int32_t* sel_out, cudaStream_t s);
+
 // 3-D bf16 tensor map [H][rows][d], box 64 columns x 128 rows, 128-byte swizzle (api.cu).
 bool encode_rows_map(CUtensorMap* m, const void* base, int H, int rows, int d);
 // 3-D e4m3 (byte) tensor map [H][rows][d], box 128 bytes x 128 rows, 128-byte swizzle.

@@ -340,41 +340,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 }
 __device__ __forceinline__ uint64_t f2_splat(float v) { return f2_pack(v, v); }
 
-// 2^a for a pair of fp32 arguments on the FMA and integer pipes instead of MUFU.  a is clamped
-// to [-126, 127] (so 2^a stays finite: a tiny positive value below the range, a huge finite one
-// above, both of which the callers' range checks treat as MUFU's 0 / inf), split as a = j + f
-// with j = round(a) (adding 1.5 * 2^23 leaves j in the low mantissa bits) and f in
-// [-0.5, 0.5]; 2^f is a cubic fitted here for the smallest largest relative error on
-// [-0.5, 0.5] (7.5e-5, below bf16's rounding of the result), and j is added to its exponent
-// field (the magic constant's own bits vanish in the 23-bit shift).
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t a2) {
-  float a0, a1;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(a2));
-  a0 = fminf(fmaxf(a0, -126.f), 127.f);
-  a1 = fminf(fmaxf(a1, -126.f), 127.f);
-  uint64_t x2, t2, r2, f2, p2;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(x2) : "f"(a0), "f"(a1));
-  const uint64_t magic2 = 0x4B4000004B400000ull;           // 1.5 * 2^23 in both lanes
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t2) : "l"(x2), "l"(magic2));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r2) : "l"(t2), "l"(magic2));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f2) : "l"(x2), "l"(r2));
-  // the cubic's coefficients 0.0551716685, 0.2426111251, 0.6932609677, 0.9999280572 (fp32
-  // bits, both lanes)
-  const uint64_t c3 = 0x3D61FBB03D61FBB0ull, c2 = 0x3E786F0D3E786F0Dull,
-                 c1 = 0x3F31798D3F31798Dull, c0 = 0x3F7FFB493F7FFB49ull;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p2) : "l"(f2), "l"(c3), "l"(c2));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p2) : "l"(f2), "l"(p2), "l"(c1));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p2) : "l"(f2), "l"(p2), "l"(c0));
-  uint32_t t0, t1, q0, q1;
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t2));
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(q0), "=r"(q1) : "l"(p2));
-  q0 = t0 * (1u << 23) + q0;
-  q1 = t1 * (1u << 23) + q1;
-  uint64_t out;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(out) : "r"(q0), "r"(q1));
-  return out;
-}
-
 // three-input maximum (sm_100)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;

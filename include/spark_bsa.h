@@ -451,6 +451,44 @@ SPARK_API spark_status spark_reblock_level(int H, int N, int d, int block, int l
                                            const int32_t* perm_in, int32_t* perm_out,
                                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Routing inside the attention kernel ----
+ * Spark-H3 blog, "Related Works" (Sol-Attn joins dynamic routing, sparse computation and the
+ * approximation correction in one online-softmax pass) and "Discussion" (block-mean scoring,
+ * fixed Top-K budget): the same forward pass as spark_bsa_forward with the block scoring and
+ * Top-K selection moved into the attention kernel.  One persistent CTA per SM walks the query
+ * blocks head-major; while it attends one query block, its K-tile producer warp scores the
+ * next one against every key-block mean and selects the Top-K in shared memory, so there is no
+ * routing launch and the selection is never read back from global memory.  The arithmetic is
+ * the routing kernel's (sequential fp32 FMA over d, exact radix select, ties to the smaller
+ * block), so selections and outputs equal spark_bsa_forward's bit for bit.
+ *   - bf16 attention operands, d = 128, Top-K with k < nkb, and a problem small enough for
+ *     two selections, two bias rows and the routing keys to fit in shared memory next to the
+ *     tiles: spark_bsa_fused_supported(d, nkb, ratio) says whether it does (nkb <= 2468 at
+ *     ratio 0.1, <= 2180 at 0.3); otherwise these calls return SPARK_ERR_UNSUPPORTED.
+ *   - spark_bsa_forward_fused: arguments, workspace and outputs of spark_bsa_forward; the
+ *     workspace's sel region receives a copy of every selection (for inspection).
+ *   - spark_bsa_attend_fused: the attention step on caller buffers with the block means of
+ *     steps 1 and 2 (qbar_blocks fp32 [H,nqb,d], kbar fp32 [H,d,nkb]) instead of a selection;
+ *     `sel_out` (int32 [H,nqb,k], may be NULL) receives the selections. */
+SPARK_API int spark_bsa_fused_supported(int d, int nkb, double topk_ratio);
+
+SPARK_API spark_status spark_bsa_forward_fused(const void* Q, const void* K, const void* V,
+                                               int dtype, int H, int N, int d,
+                                               const int32_t* q_perm, const int32_t* k_perm,
+                                               const int32_t* q_block_offsets, int nqb,
+                                               const int32_t* k_block_offsets, int nkb,
+                                               double topk_ratio, void* out, void* workspace,
+                                               size_t workspace_bytes, void* stream);
+
+SPARK_API spark_status spark_bsa_attend_fused(const void* Qp, const void* Kp, const void* Vp,
+                                              const void* k_tilde, const void* v_tilde,
+                                              const float* cbias, const float* qbar_blocks,
+                                              const float* kbar, int k, const int32_t* q_perm,
+                                              const int32_t* q_block_offsets, int nqb,
+                                              const int32_t* k_block_offsets, int nkb, int H,
+                                              int N, int d, void* out, int out_dtype,
+                                              int32_t* sel_out, uint32_t* err, void* stream);
+
 /* ---- Forward pass without any allocation ----
  * No counterpart in the pages: this entry point exists for callers that cannot allocate
  * device memory while they run (a memory budget owned by a host framework, work recorded into
