@@ -187,7 +187,7 @@ class HotPath:
         if routing in ("threshold", "fused"):
             if fp8 or self.nc:
                 raise SystemExit(f"{routing} routing runs without fp8 and context here")
-        if routing == "fused" and not L.spark_bsa_fused_supported(self.d, self.nkb, float(ratio)):
+        if routing == "fused" and not self.L.spark_bsa_fused_supported(self.d, self.nkb, float(ratio)):
             raise SystemExit("routing inside the attention kernel does not support this shape")
         if routing == "threshold":
             self.count = torch.empty(self.H, self.nqb, dtype=torch.int32, device=device)
