@@ -20,22 +20,32 @@
 //              rows take their recorded maximum as the reference - each chunk whose sum is out
 //              of range records its maximum, which is within a few units of the row's - and the
 //              other rows keep theirs.
-//   warp 8     TMA producer (the warp runs the loop, one elected lane issues): the Q tile once,
-//              then K tiles (3-stage ring; a stage is free again
-//              once the S MMA that read it has completed, signalled by that S buffer's barrier).
+//   warp 8     TMA producer: the Q tile once, then K tiles (3-stage ring; a stage is free
+//              again once the S MMA that read it has completed, signalled by that S buffer's
+//              barrier).
 //   warp 9     TMA producer of V tiles (2-stage ring).
-//   warp 10    MMA issuer (the warp runs the loop, one elected lane issues): S(t) = Q K^T (both from shared memory) into TMEM
-//              buffer t%3, O += P(t) V(t) (P read from TMEM, V an MN-major shared-memory
-//              operand).  Issue order S(0), S(1), S(2), PV(0), S(3), PV(1), S(4), ...: MMAs
-//              of one thread execute in order, so S(t+3) overwrites its buffer only after
-//              PV(t) has consumed P(t).  With three buffers the next S of a group is ready
-//              while the group still works on its current tile.
+//   warp 10    MMA issuer: S(t) = Q K^T (both from shared memory) into TMEM buffer t%3,
+//              O += P(t) V(t) (P read from TMEM, V an MN-major shared-memory operand).  Issue
+//              order S(0), S(1), S(2), PV(0), S(3), PV(1), S(4), ...: MMAs of one thread execute
+//              in order, so S(t+3) overwrites its buffer only after PV(t) has consumed P(t).
+//              With three buffers the next S of a group is ready while the group still works
+//              on its current tile.
+//   Warps 8-10 run their loops warp-uniformly (stage indices, coordinates and descriptors are
+//   the same in every lane) and one elected lane issues the copies, MMAs and commits: issuing
+//   from a single divergent lane measured 8% slower at 768p.
 //
 // Tile list of a CTA: the k selected blocks in ascending order (a 128-row TMA box starting at
 // the block's first row; rows past the block are masked), then ceil(nc/128) tiles of the
 // head's context tokens (same blog section: context/sink tokens stay exact, outside the Top-K
 // budget; rows past nc masked), then ceil(nkb/128) tiles of the summary rows (rows past nkb
-// are zero-filled by TMA and masked, selected blocks masked).
+// are zero-filled by TMA and masked, selected blocks masked).  When some key block is shorter
+// than 128 rows (kVarTiles), an exact tile's S MMA has N = its rows rounded up to 16, its PV
+// takes only that many keys, and the softmax covers only those columns.
+//
+// With the routing inside (kPersist: Spark-H3 blog, "Related Works", Sol-Attn's single pass
+// over routing and attention): one persistent CTA per SM walks the query blocks head-major, and
+// a 12th warp scores and selects the NEXT query block (route_step.cuh, the routing kernel's
+// arithmetic) into a second set of shared-memory buffers while the current one is attended.
 //
 // TMEM columns (512 allocated, one CTA per SM): S/P buffers [0,128), [128,256), [256,384),
 // O [384,384+D).
@@ -53,7 +63,9 @@ namespace {
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
 constexpr int kWarpK = 8, kWarpV = 9, kWarpMma = 10;
-constexpr int kThreads = 352;
+constexpr int kWarpRoute = 11;              // with in-kernel routing only
+constexpr int kThreads = 352;               // 11 warps
+constexpr int kThreadsFused = 384;          // 12 warps: 3 per SM sub-partition, 168 registers each
 constexpr uint32_t kColO = 384;             // S/P buffer b at column 128*b (b < 3)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMaxSmemBias = 6144;          // summary offsets kept in shared memory (floats)
@@ -234,8 +246,8 @@ __device__ __forceinline__ float exp32_at(const float (&x)[64], int j0, float c,
 
 }  // namespace
 
-template <int D, bool kBiasSmem, bool kFp8, bool kFused, bool kVarTiles>
-__global__ void __launch_bounds__(kThreads, 1) attend_kernel(
+template <int D, bool kBiasSmem, bool kFp8, bool kPersist, bool kRoute, bool kVarTiles>
+__global__ void __launch_bounds__(kPersist ? kThreadsFused : kThreads, 1) attend_kernel(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kt,
     const __grid_constant__ CUtensorMap map_vt, const __grid_constant__ CUtensorMap map_kc,
@@ -247,7 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     uint64_t wait_ns, int H, const float* __restrict__ qbar_blocks,
     const float* __restrict__ kbar, int32_t* __restrict__ sel_out) {
   static_assert(!kFp8 || D == 128, "FP8 logits: d = 128 (one 128-byte row per key)");
-  static_assert(!kFused || (kBiasSmem && !kFp8), "in-kernel routing: bf16, bias row in smem");
+  static_assert(!kPersist || (kBiasSmem && !kFp8), "persistent CTAs: bf16, bias row in smem");
+  static_assert(!kRoute || kPersist, "in-kernel routing runs in persistent CTAs");
   constexpr int QK_BYTES = 128 * D * (kFp8 ? 1 : 2);   // one Q or K tile
   constexpr int V_BYTES = 128 * D * 2;                 // one V tile (bf16)
   constexpr int QK_ATOMS = kFp8 ? 1 : D / 64;          // 128-byte swizzle atoms across a row
@@ -280,15 +293,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       p += bytes;
       return at;
     };
-    for (int b = 0; b < (kFused ? 2 : 1); ++b) {
+    for (int b = 0; b < (kPersist ? 2 : 1); ++b) {
       selmask_b[b] = reinterpret_cast<uint32_t*>(carve(static_cast<size_t>(nwords) * 4));
       biasrow_b[b] = reinterpret_cast<float*>(carve(static_cast<size_t>(nbias) * 4));
     }
-    if (kFused) {
+    if (kPersist) {
       for (int b = 0; b < 2; ++b) sel_s_b[b] = reinterpret_cast<int32_t*>(carve(kcap * 4u));
-      rsm.keys = reinterpret_cast<uint32_t*>(carve(static_cast<size_t>(nkb) * 4));
-      rsm.hist = reinterpret_cast<uint32_t*>(carve(256 * 4));
-      rsm.qn = reinterpret_cast<float*>(carve(D * 4));
+      if (kRoute) {
+        rsm.keys = reinterpret_cast<uint32_t*>(carve(static_cast<size_t>(nkb) * 4));
+        rsm.hist = reinterpret_cast<uint32_t*>(carve(256 * 4));
+        rsm.qn = reinterpret_cast<float*>(carve(D * 4));
+      }
     } else {
       selmask_b[1] = selmask_b[0];
       biasrow_b[1] = biasrow_b[0];
@@ -299,20 +314,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   __shared__ int s_skip, s_rerun;
   // [group][row]: first-tile maxima (the reference), then sums and maxima for the epilogue
   __shared__ float ex_m[2][128], ex_l[2][128], ex_mt[2][128];
-  if (tid == 0) {
-    s_skip = launch_timed_out(err) ? 1 : 0;                // an earlier CTA gave up
-    s_rerun = 0;
-  }
-  __syncthreads();
-  if (s_skip) return;                                      // uniform: no work, nothing held
   // Query blocks of this CTA: one, (blockIdx.x, blockIdx.y), or with in-kernel routing every
   // gridDim.x-th of the H*nqb (head-major) starting at blockIdx.x.
-  const int n_items = kFused ? H * nqb : 1;
-  int item = kFused ? static_cast<int>(blockIdx.x) : 0;
-  if (kFused && item >= n_items) return;
+  const int n_items = kPersist ? H * nqb : 1;
+  int item = kPersist ? static_cast<int>(blockIdx.x) : 0;
+  if (kPersist && item >= n_items) return;
   const int nxt = (nc + 127) / 128;                 // context tiles
 
   if (tid == 0) {
+    s_skip = launch_timed_out(err) ? 1 : 0;                // an earlier CTA gave up
+    s_rerun = 0;
     mbar_init(&bars->qfull, 1);
     for (int s = 0; s < kKStages; ++s) mbar_init(&bars->kfull[s], 1);
     for (int s = 0; s < kVStages; ++s) {
@@ -327,18 +338,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (!kFused) {
-    // the selection comes from the routing kernel: build the mask and the bias row from it
-    const int h = blockIdx.y;
-    const int k = sel_count ? max(0, min(sel_count[static_cast<size_t>(h) * nqb + blockIdx.x], kcap))
-                            : kcap;
-    const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
-    const float* cb = cbias + static_cast<size_t>(h) * nkb;
-    for (int i = tid; i < nwords; i += kThreads) selmask_b[0][i] = 0u;
-    if (kBiasSmem)
-      for (int i = tid; i < nct * 128; i += kThreads)
-        biasrow_b[0][i] = (i < nkb) ? cb[i] * kLog2e : -INFINITY;
-  }
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -346,11 +345,24 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  if (!kFused) {
+  if (s_skip) {                                            // uniform: give back TMEM and leave
+    if (warp == 0) tmem_dealloc(*tmem_slot, 512);
+    return;
+  }
+  if (!kPersist && warp < 8) {
+    // The selection comes from the routing kernel.  The softmax warps build the mask and the
+    // bias row (the only readers) while the producers and the MMA warp already start.
     const int h = blockIdx.y, A = blockIdx.x;
     const int k = sel_count ? max(0, min(sel_count[static_cast<size_t>(h) * nqb + A], kcap)) : kcap;
+    const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
+    const float* cb = cbias + static_cast<size_t>(h) * nkb;
+    for (int i = tid; i < nwords; i += 256) selmask_b[0][i] = 0u;
+    if (kBiasSmem)
+      for (int i = tid; i < nct * 128; i += 256)
+        biasrow_b[0][i] = (i < nkb) ? cb[i] * kLog2e : -INFINITY;
+    named_bar_sync(5, 256);
     const int32_t* srow = sel + (static_cast<size_t>(h) * nqb + A) * kcap;
-    for (int i = tid; i < k; i += kThreads) {
+    for (int i = tid; i < k; i += 256) {
       const int B = srow[i];
       if (B >= 0 && B < nkb) {
         atomicOr(&selmask_b[0][B >> 5], 1u << (B & 31));
@@ -359,35 +371,39 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         flag_error(err, kErrSel);
       }
     }
+    named_bar_sync(5, 256);
   }
-  // In-kernel routing: the K producer routes this CTA's first query block before any tile.
+  // Persistent CTAs: the 12th warp routes this CTA's first query block (selection, mask and
+  // bias row) before any tile.
   RouteJob job = route_job_none();
-  if (kFused && warp == kWarpK) {
-    job = route_job(item / nqb, item % nqb, 0);
-    while (job.stage != kRjDone)
-      route_step<D>(job, rsm, qbar_blocks, kbar, cbias, nqb, nkb, kcap, sel_s_b[0],
-                    selmask_b[0], biasrow_b[0], sel_out, lane);
+  if (kPersist) {
+    if (warp == kWarpRoute) {
+      job = route_job(item / nqb, item % nqb, 0);
+      while (job.stage != kRjDone)
+        route_step<D>(job, rsm, qbar_blocks, kbar, cbias, nqb, nkb, kcap, sel_s_b[0],
+                      selmask_b[0], biasrow_b[0], sel_out, lane);
+    }
+    __syncthreads();
   }
-  __syncthreads();
   const uint32_t tbase = *tmem_slot;
   // Barrier phases count over the CTA's whole life: tiles (both passes of every query block),
   // passes (the `done` barrier) and query blocks (the Q tile).
   int tiles_base = 0, passes_base = 0, items_done = 0;
   int issued = 0;                                  // producers: loads issued so far
   for (int cur = 0;; cur ^= 1) {
-  const int A = kFused ? item % nqb : static_cast<int>(blockIdx.x);
-  const int h = kFused ? item / nqb : static_cast<int>(blockIdx.y);
+  const int A = kPersist ? item % nqb : static_cast<int>(blockIdx.x);
+  const int h = kPersist ? item / nqb : static_cast<int>(blockIdx.y);
   // selected blocks of this query block: kcap, or its own count (threshold routing) when
   // sel_count is given; rows of sel are kcap apart either way
   const int k = sel_count ? max(0, min(sel_count[static_cast<size_t>(h) * nqb + A], kcap)) : kcap;
   const int nct = (k < nkb) ? (nkb + 127) / 128 : 0;
   const int T = k + nxt + nct;
-  const int32_t* sel_row = kFused ? sel_s_b[cur] : sel + (static_cast<size_t>(h) * nqb + A) * kcap;
+  const int32_t* sel_row = kPersist ? sel_s_b[cur] : sel + (static_cast<size_t>(h) * nqb + A) * kcap;
   const float* cb = cbias + static_cast<size_t>(h) * nkb;
   const uint32_t* selmask = selmask_b[cur];
   const float* biasrow = biasrow_b[cur];
   const int qlo = q_offsets[A];
-  if (kFused && warp == kWarpK) {
+  if (kPersist && warp == kWarpRoute) {
     // route the CTA's next query block into the other buffers while this one is attended
     const int nitem = item + static_cast<int>(gridDim.x);
     job = nitem < n_items ? route_job(nitem / nqb, nitem % nqb, cur ^ 1) : route_job_none();
@@ -460,10 +476,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
         issued = tg + 1;
         if (t + 1 < T)
           next = tile_info<false>(t + 1, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
-        // one bounded step of the next query block's routing per K tile
-        if (kFused && is_k && job.stage != kRjDone)
-          route_step<D>(job, rsm, qbar_blocks, kbar, cbias, nqb, nkb, kcap, sel_s_b[job.buf],
-                        selmask_b[job.buf], biasrow_b[job.buf], sel_out, lane);
       }
       // every load this pass issued has landed before the pass ends (after an abort some were
       // never consumed; otherwise these phases are complete already and the waits return at once)
@@ -549,7 +561,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
       if (elect_one()) tc_commit(&bars->done);
       __syncwarp();
       wait_bounded_ignore_abort(&bars->done, done_par);
-    } else {
+    } else if (kPersist && warp == kWarpRoute) {
+      // ------------------------------------------------------------------ routing warp
+      // the next query block's scores and Top-K, while the MMAs and the softmax run this one
+      if (pass == 0)
+        while (job.stage != kRjDone && !*abort_flag)
+          route_step<D>(job, rsm, qbar_blocks, kbar, cbias, nqb, nkb, kcap, sel_s_b[job.buf],
+                        selmask_b[job.buf], biasrow_b[job.buf], sel_out, lane);
+    } else if (warp < 8) {
       // ---------------------------------------------------------------- softmax rows
       const int q4 = warp & 3, grp = warp >> 2;          // row quarter, tile group
       const int row = q4 * 32 + lane;                    // 0..127 == TMEM lane
@@ -706,9 +725,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(
   tiles_base += npasses * T;
   passes_base += npasses;
   ++items_done;
-  if (!kFused) break;
-  // the next query block's routing completes before it starts (few tiles, or an abort)
-  if (warp == kWarpK)
+  if (!kPersist) break;
+  // the next query block's routing completes before it starts
+  if (kPersist && warp == kWarpRoute)
     while (job.stage != kRjDone && !*abort_flag)
       route_step<D>(job, rsm, qbar_blocks, kbar, cbias, nqb, nkb, kcap, sel_s_b[job.buf],
                     selmask_b[job.buf], biasrow_b[job.buf], sel_out, lane);
@@ -739,17 +758,18 @@ static size_t align16(size_t b) { return (b + 15) & ~static_cast<size_t>(15); }
 // the barriers, then (16-byte aligned each) the selection mask and bias row of one query block,
 // or with in-kernel routing two of each plus two selections, the routing keys, a histogram and
 // the query-block mean.
-static size_t attend_smem_bytes(int d, int nkb, int k, bool fp8, bool fused = false) {
+static size_t attend_smem_bytes(int d, int nkb, int k, bool fp8, bool persist = false,
+                                bool route = false) {
   const size_t qk = static_cast<size_t>(128) * d * (fp8 ? 1 : 2);
   const size_t v = static_cast<size_t>(128) * d * 2;
   const size_t words = static_cast<size_t>((nkb + 31) / 32) * 4;
-  const size_t bias = bias_in_smem(nkb, k) || fused ? static_cast<size_t>((nkb + 127) / 128) * 128 * 4
-                                                    : 0;
+  const size_t bias = bias_in_smem(nkb, k) || persist
+                          ? static_cast<size_t>((nkb + 127) / 128) * 128 * 4 : 0;
   size_t b = 1024 + (1 + kKStages) * qk + kVStages * v + sizeof(Barriers) + 16;
-  const int nbuf = fused ? 2 : 1;
+  const int nbuf = persist ? 2 : 1;
   b += nbuf * (align16(words) + 16 + align16(bias) + 16);
-  if (fused) b += 2 * (align16(static_cast<size_t>(k) * 4) + 16) +
-                  align16(static_cast<size_t>(nkb) * 4) + 16 + 256 * 4 + 16 + d * 4 + 16;
+  if (persist) b += 2 * (align16(static_cast<size_t>(k) * 4) + 16);
+  if (route) b += align16(static_cast<size_t>(nkb) * 4) + 16 + 256 * 4 + 16 + d * 4 + 16;
   return b;
 }
 
@@ -758,6 +778,14 @@ constexpr size_t kSmemLimit = 232448;   // 227 KB of opt-in shared memory per CT
 // All key blocks hold exactly 128 tokens (sizes are 1..128 and sum to N) - then every exact
 // tile is a full MMA tile and the kernel without per-tile widths runs.
 static bool all_blocks_full(int N, int nkb) { return static_cast<long long>(nkb) * 128 == N; }
+
+static cudaError_t persistent_grid(long long items, int* grid) {
+  int dev = 0, nsm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  *grid = static_cast<int>(items < nsm ? items : nsm);   // one persistent CTA per SM
+  return e;
+}
 
 template <int D, bool kBiasSmem, bool kFp8, bool kVar>
 static cudaError_t launch_attend_t(const AttendMaps& m, int nc, const float* cbias,
@@ -768,7 +796,7 @@ static cudaError_t launch_attend_t(const AttendMaps& m, int nc, const float* cbi
                                    cudaStream_t s) {
   // with per-row counts any row may have summary tiles: size for k < nkb
   const size_t smem = attend_smem_bytes(D, nkb, sel_count ? 0 : k, kFp8);
-  auto kern = attend_kernel<D, kBiasSmem, kFp8, false, kVar>;
+  auto kern = attend_kernel<D, kBiasSmem, kFp8, false, false, kVar>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -837,7 +865,7 @@ cudaError_t launch_attend_fp8(const AttendMaps& maps, const float* q_scale,
 
 bool attend_fused_supported(int d, int nkb, int k) {
   return d == 128 && k < nkb && bias_in_smem(nkb, k) &&
-         attend_smem_bytes(d, nkb, k, false, true) <= kSmemLimit;
+         attend_smem_bytes(d, nkb, k, false, true, true) <= kSmemLimit;
 }
 
 template <bool kVar>
@@ -847,19 +875,15 @@ static cudaError_t launch_fused_t(const AttendMaps& m, int nc, const float* cbia
                                   const int32_t* k_offsets, int nkb, int H, int N, void* out,
                                   int out_dtype, uint32_t* err, int32_t* sel_out,
                                   cudaStream_t s) {
-  const size_t smem = attend_smem_bytes(128, nkb, k, false, true);
-  auto kern = attend_kernel<128, true, false, true, kVar>;
+  const size_t smem = attend_smem_bytes(128, nkb, k, false, true, true);
+  auto kern = attend_kernel<128, true, false, true, true, kVar>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  int dev = 0, nsm = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-    return e;
-  const long long items = static_cast<long long>(H) * nqb;
-  const int grid = static_cast<int>(items < nsm ? items : nsm);   // one persistent CTA per SM
+  int grid = 0;
+  if ((e = persistent_grid(static_cast<long long>(H) * nqb, &grid)) != cudaSuccess) return e;
   const Fp8Scales none{nullptr, nullptr, nullptr, nullptr};
-  kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.kt, m.vt, m.kc, m.vc, nc, cbias, nullptr, k,
+  kern<<<grid, kThreadsFused, smem, s>>>(m.q, m.k, m.v, m.kt, m.vt, m.kc, m.vc, nc, cbias, nullptr, k,
                                     nullptr, q_perm, q_offsets, nqb, k_offsets, nkb, N, out,
                                     out_dtype, err, none, wait_limit_ns(), H, qbar_blocks, kbar,
                                     sel_out);

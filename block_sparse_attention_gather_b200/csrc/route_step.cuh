@@ -1,7 +1,6 @@
-// Block scoring + Top-K of ONE query block by one warp, cut into short bounded steps so that a
-// warp with other duties (the attention kernel's K-tile producer) can interleave it with its
-// own work: the routing of the next query block runs while the current one is attended, and the
-// selection never leaves shared memory (Spark-H3 blog, "Discussion": blocks scored from
+// Block scoring + Top-K of ONE query block by one warp, in short bounded steps: the attention
+// kernel's routing warp runs them for the next query block while the current one is attended,
+// and the selection never leaves shared memory (Spark-H3 blog, "Discussion": blocks scored from
 // block-level means; "Spark-Reblock": a fixed Top-K budget).
 //
 // The arithmetic is that of route_kernel (route.cu): each score is a sequential fp32 FMA over
@@ -86,7 +85,7 @@ __device__ __forceinline__ void route_step(RouteJob& j, const RouteSmem& rs,
       const int B = j.pos + lane;
       const float* kb = kbar + static_cast<size_t>(j.h) * D * nkb + min(B, nkb - 1);
       float acc = 0.f;
-      constexpr int kE = D < 64 ? D : 64;        // loads in flight per lane
+      constexpr int kE = D;                      // loads in flight per lane (one round trip)
 #pragma unroll 1
       for (int e0 = 0; e0 < D; e0 += kE) {
         float v[kE];
