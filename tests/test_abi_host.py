@@ -255,3 +255,39 @@ def test_missing_library_fails_loudly(tmp_path):
             "try:\n    n.lib()\nexcept RuntimeError as e:\n    print('RAISED', 'no fallback' in str(e))")
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
     assert "RAISED True" in r.stdout, r.stderr
+
+
+def test_wait_limit_is_a_process_wide_setting(L):
+    from block_sparse_attention_gather_b200 import (spark_bsa_get_wait_limit_ns,
+                                                    spark_bsa_set_wait_limit_ns)
+    assert spark_bsa_get_wait_limit_ns() == 4_000_000_000         # 4 s by default
+    try:
+        spark_bsa_set_wait_limit_ns(123)
+        assert spark_bsa_get_wait_limit_ns() == 123
+        spark_bsa_set_wait_limit_ns(0)
+        assert spark_bsa_get_wait_limit_ns() == 0
+    finally:
+        spark_bsa_set_wait_limit_ns(4_000_000_000)
+
+
+def test_fused_routing_support_follows_shared_memory(L):
+    from block_sparse_attention_gather_b200 import spark_bsa_fused_supported
+    assert spark_bsa_fused_supported(128, 1890, 0.1)              # 768p
+    assert spark_bsa_fused_supported(128, 473, 0.1)               # 384p
+    assert not spark_bsa_fused_supported(64, 1890, 0.1)           # d = 64
+    assert not spark_bsa_fused_supported(128, 1890, 1.0)          # no compressed branch
+    assert not spark_bsa_fused_supported(128, 2540, 0.1)          # routing state too large
+    p = ctypes.c_void_p(0x100000)
+    # d = 64: refused before anything is launched
+    assert L.spark_bsa_forward_fused(p, p, p, 0, 1, 1024, 64, p, p, p, 16, p, 16,
+                                     ctypes.c_double(0.125), p, p, ctypes.c_size_t(1 << 40),
+                                     None) == 2
+
+
+def test_host_pipeline_staging_grows_with_context_rows(L):
+    from block_sparse_attention_gather_b200 import spark_bsa_host_staging_size_ex
+    import torch
+    base = spark_bsa_host_staging_size_ex(24, 241920, 128, torch.bfloat16, 1890, 1890, 1, 0)
+    ctx = spark_bsa_host_staging_size_ex(24, 241920, 128, torch.bfloat16, 1890, 1890, 1, 512)
+    assert base > 0 and ctx >= base + 2 * 2 * 512 * 128 * 2      # Kc, Vc in both slots
+    assert spark_bsa_host_staging_size_ex(24, 241920, 128, torch.bfloat16, 1890, 1890, 1, -1) == 0
