@@ -314,18 +314,32 @@ def attention_flops(hp):
 
 
 def attention_issued_flops(hp):
-    """Tensor-core FLOPs the attention kernel issues, padding included: every key tile is a
-    128 x 128 box (M = 128 query rows, N = 128 keys) multiplied over d for S = Q K^T and again
-    for O += P V, so a (head, query block) with T tiles issues 4 * 128 * 128 * d * T whatever
-    the sizes of its blocks.  T = selected blocks + context tiles + summary tiles."""
+    """Tensor-core FLOPs the attention kernel issues, padding included: every tile multiplies a
+    128-row query tile (M = 128 whatever the query block's size) against its keys, over d for
+    S = Q K^T and again for O += P V.  A summary tile covers 128 keys.  An exact tile (a
+    selected key block or a context tile) covers 128 keys when every key block holds 128 tokens,
+    else its valid rows rounded up to 16 (the kernel's variable-width tiles); so a (head, query
+    block) issues 4 * 128 * d * (sum of its tiles' keys)."""
+    ko = hp.x["k_offsets"].long()
+    ks = (ko[1:] - ko[:-1])
+    full = hp.nkb * 128 == hp.N
+    width = torch.full_like(ks, 128) if full else ((ks + 15) // 16 * 16).clamp(16, 128)
     nct = -(-hp.nkb // 128)
-    nxt = -(-hp.nc // 128)
+    ctx = 0
+    if hp.nc:
+        rows = [min(128, hp.nc - y) for y in range(0, hp.nc, 128)]
+        ctx = sum(128 if full else min(128, max(16, -(-r // 16) * 16)) for r in rows)
+    sel = hp.v["sel"].long()                                 # [H,nqb,k]
+    wsel = width.to(sel.device)[sel.clamp(0, hp.nkb - 1)]    # [H,nqb,k]
     if getattr(hp, "routing", "topk") == "threshold":
-        cnt = hp.count.long().cpu()
-        tiles = (cnt + nxt + torch.where(cnt < hp.nkb, nct, 0)).sum().item()
+        cnt = hp.count.long().to(sel.device)
+        valid = torch.arange(sel.shape[-1], device=sel.device)[None, None, :] < cnt[..., None]
+        exact = (wsel * valid).sum(-1)
+        summ = torch.where(cnt < hp.nkb, nct * 128, 0)
+        keys = (exact + ctx + summ).sum().item()
     else:
-        tiles = hp.H * hp.nqb * (hp.k + nxt + (nct if hp.k < hp.nkb else 0))
-    return 4.0 * 128 * 128 * hp.d * float(tiles)
+        keys = wsel.sum().item() + hp.H * hp.nqb * (ctx + (nct * 128 if hp.k < hp.nkb else 0))
+    return 4.0 * 128 * hp.d * float(keys)
 
 
 def kernel_bytes(hp):

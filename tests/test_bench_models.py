@@ -64,3 +64,18 @@ def test_attention_flops_with_threshold_counts():
     hp.count = torch.tensor([[1, 0]], dtype=torch.int32)
     expect = 4 * 32 * (3 * (6 + 2) + 5 * (0 + 3))
     assert bench.attention_flops(hp) == expect
+
+
+def test_issued_flops_follow_the_kernels_tiles():
+    # short key blocks (variable tiles): an exact tile covers its rows rounded up to 16; the one
+    # summary tile covers 128 keys; 7 context rows make one tile of 16; M is always 128
+    hp = fake_hotpath([3, 5], [4, 2, 6], [[[2], [0]]], d=64, nc=7)
+    expect = 4 * 128 * 64 * ((16 + 16 + 128) + (16 + 16 + 128))
+    assert bench.attention_issued_flops(hp) == expect
+    # every key block full (128 rows): every exact tile covers 128 keys, context too
+    hp = fake_hotpath([128, 128, 128], [128, 128, 128], [[[2], [0], [1]]], d=64, nc=7)
+    expect = 4 * 128 * 64 * 3 * (128 + 128 + 128)
+    assert bench.attention_issued_flops(hp) == expect
+    # k = nkb: no summary tile
+    hp = fake_hotpath([40], [40, 70], [[[0, 1]]], d=32)
+    assert bench.attention_issued_flops(hp) == 4 * 128 * 32 * (48 + 80)
