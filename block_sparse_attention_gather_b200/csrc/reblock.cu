@@ -954,15 +954,56 @@ __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, boo
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
+// The power iterations of one node from its second moment S (shared memory, [128][128]) and
+// column sums sxv (thread t: dimension t), 128 threads: mu = sum x / n, then kPowerIters steps
+// v <- w / |w|, w = S v / n - (mu . v) mu, from v0 = (1,...,1)/sqrt(d).  Writes mu and v of
+// node g.  Shared by rb_cov_node_kernel and the single-chunk form of rb_cov_tc_kernel, so both
+// take the same arithmetic.
+__device__ __forceinline__ void rb_node_power(const float* Ssm, float sxv, float n, int t,
+                                              float* vs, float* red, float* s_val, int h, int g,
+                                              int nnodes, float* __restrict__ mu,
+                                              float* __restrict__ vnode) {
+  const float m = sxv / n;
+  float v = rsqrtf(128.f);
+  auto block_sum = [&](float x) {
+    x = warp_sum(x);
+    __syncthreads();
+    if (t % 32 == 0) red[t / 32] = x;
+    __syncthreads();
+    if (t == 0) *s_val = red[0] + red[1] + red[2] + red[3];
+    __syncthreads();
+    return *s_val;
+  };
+  for (int it = 0; it < kPowerIters; ++it) {
+    vs[t] = v;
+    __syncthreads();
+    float sv = 0.f;
+    for (int j = 0; j < 128; ++j) sv = fmaf(Ssm[j * 128 + t], vs[j], sv);   // S symmetric
+    const float muv = block_sum(m * v);
+    const float w = sv / n - muv * m;
+    const float nrm2 = block_sum(w * w);
+    v = nrm2 > 0.f ? w * rsqrtf(nrm2) : v;
+  }
+  const size_t at = (static_cast<size_t>(h) * nnodes + g) * 128 + t;
+  mu[at] = m;
+  vnode[at] = v;
+}
+
 // One chunk of a node: rows gathered by the permutation into 128-token tiles (cp.async, each
 // 16-byte piece written to its place in the 128-byte swizzled layout, zero past the chunk
-// end), the next tile in flight while the tensor core consumes the current one.
+// end), the next tile in flight while the tensor core consumes the current one.  kSingle: every
+// node of the level is one chunk, so the CTA holds the node's whole second moment and runs its
+// power iterations itself (mu, v of the node) instead of writing the 66 KB partial for
+// rb_cov_node_kernel.
+template <bool kSingle>
 __global__ void __launch_bounds__(128) rb_cov_tc_kernel(const __nv_bfloat16* __restrict__ X,
                                                         const int32_t* __restrict__ perm, int N,
                                                         const int4* __restrict__ cchunks,
                                                         int ncch, float* __restrict__ cpart,
                                                         uint32_t* __restrict__ err,
-                                                        uint64_t wait_ns) {
+                                                        uint64_t wait_ns, int nnodes,
+                                                        float* __restrict__ mu,
+                                                        float* __restrict__ vnode) {
   extern __shared__ uint8_t rb_tc_raw[];
   uint8_t* st = align1024(rb_tc_raw);                    // 2 stages x 32 KB
   uint64_t* mdone = reinterpret_cast<uint64_t*>(st + 2 * kTcTile);   // [2]
@@ -1059,8 +1100,46 @@ __global__ void __launch_bounds__(128) rb_cov_tc_kernel(const __nv_bfloat16* __r
   __syncthreads();
   const bool fine = ok && !*abort_flag;
   tc_fence_after_sync();
-  float* out = cpart + (static_cast<size_t>(h) * ncch + c) * kCovStride;
   const int row = warp * 32 + (tid % 32);
+  if constexpr (kSingle) {
+    // S from TMEM into the (now idle) tile stages, the column sums in thread order, then the
+    // power iterations - the values rb_cov_node_kernel would read back from the partial
+    float* Ssm = reinterpret_cast<float*>(st);          // [128][128] = both 32 KB stages
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t r[32];
+      if (fine) {
+        tmem_ld32(tbase + (static_cast<uint32_t>(warp * 32) << 16) + cc * 32, r);
+      } else {
+        for (int j = 0; j < 32; ++j) r[j] = 0u;
+      }
+      float4* dst = reinterpret_cast<float4*>(Ssm + row * 128 + cc * 32);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                             __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) red[tid * 8 + j] = sx[j];
+    __syncthreads();
+    float sxv = 0.f;
+    {
+      const int dim = tid, cc = dim / 8, j = dim % 8;
+      float a = 0.f;
+      for (int g = 0; g < 8; ++g) a += red[(g * 16 + cc) * 8 + j];
+      sxv = 0.f + (fine ? a : 0.f);                     // the node's sum over its one chunk
+    }
+    __shared__ float vs[128], pred[4], s_val;
+    rb_node_power(Ssm, sxv, static_cast<float>(ch.z - ch.y), tid, vs, pred, &s_val, h, ch.x,
+                  nnodes, mu, vnode);
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after_sync();
+      tmem_dealloc(tbase, 128);
+    }
+    return;
+  }
+  float* out = cpart + (static_cast<size_t>(h) * ncch + c) * kCovStride;
   for (int cc = 0; cc < 4; ++cc) {
     uint32_t r[32];
     if (fine) {
@@ -1122,30 +1201,7 @@ __global__ void __launch_bounds__(128) rb_cov_node_kernel(const float* __restric
   }
   float sxv = 0.f;
   for (int c = cn.x; c < cn.y; ++c) sxv += cpart[(static_cast<size_t>(h) * ncch + c) * kCovStride + 128 * 128 + t];
-  const float m = sxv / n;
-  float v = rsqrtf(128.f);
-  auto block_sum = [&](float x) {
-    x = warp_sum(x);
-    __syncthreads();
-    if (t % 32 == 0) red[t / 32] = x;
-    __syncthreads();
-    if (t == 0) s_val = red[0] + red[1] + red[2] + red[3];
-    __syncthreads();
-    return s_val;
-  };
-  for (int it = 0; it < kPowerIters; ++it) {
-    vs[t] = v;
-    __syncthreads();
-    float sv = 0.f;
-    for (int j = 0; j < 128; ++j) sv = fmaf(Ssm[j * 128 + t], vs[j], sv);   // S symmetric
-    const float muv = block_sum(m * v);
-    const float w = sv / n - muv * m;
-    const float nrm2 = block_sum(w * w);
-    v = nrm2 > 0.f ? w * rsqrtf(nrm2) : v;
-  }
-  const size_t at = (static_cast<size_t>(h) * nnodes + g) * 128 + t;
-  mu[at] = m;
-  vnode[at] = v;
+  rb_node_power(Ssm, sxv, n, t, vs, red, &s_val, h, g, nnodes, mu, vnode);
 }
 
 // ------------------------------------------------------------------ host side
@@ -1358,16 +1414,25 @@ static cudaError_t level_t(int H, int N, int block, int level, const int32_t* pe
     float* cpart = reinterpret_cast<float*>(ws + L.cpart);
     uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.err);
     const size_t smem = 1024 + 2 * kTcTile + 3 * 8 + 16 + 256 * 4 + 128 * 8 * 4;
-    e = cudaFuncSetAttribute(rb_cov_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    rb_cov_tc_kernel<<<dim3(lm.ncch, H), 128, smem, s>>>(X, perm_in, N, cchunks, lm.ncch, cpart,
-                                                         err, wait_limit_ns());
-    const size_t nsmem = 128 * 128 * 4;
-    e = cudaFuncSetAttribute(rb_cov_node_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(nsmem));
-    if (e != cudaSuccess) return e;
-    rb_cov_node_kernel<<<gn, 128, nsmem, s>>>(cpart, lm.ncch, cnodes, nodes, nn, mu, v);
+    if (lm.ncch == nn) {
+      // every node is one chunk: moments and power iterations in one kernel
+      e = cudaFuncSetAttribute(rb_cov_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      rb_cov_tc_kernel<true><<<dim3(lm.ncch, H), 128, smem, s>>>(
+          X, perm_in, N, cchunks, lm.ncch, cpart, err, wait_limit_ns(), nn, mu, v);
+    } else {
+      e = cudaFuncSetAttribute(rb_cov_tc_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      rb_cov_tc_kernel<false><<<dim3(lm.ncch, H), 128, smem, s>>>(
+          X, perm_in, N, cchunks, lm.ncch, cpart, err, wait_limit_ns(), nn, mu, v);
+      const size_t nsmem = 128 * 128 * 4;
+      e = cudaFuncSetAttribute(rb_cov_node_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(nsmem));
+      if (e != cudaSuccess) return e;
+      rb_cov_node_kernel<<<gn, 128, nsmem, s>>>(cpart, lm.ncch, cnodes, nodes, nn, mu, v);
+    }
   } else {
     rb_power_kernel<D, true><<<gc, kRbThreads, 0, s>>>(X, perm_in, N, chunks, nc, v, nn, part);
     rb_node_reduce_kernel<D, true><<<gn, D, 0, s>>>(part, nc, nodes, nn, mu, v);

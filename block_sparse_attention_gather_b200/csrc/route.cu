@@ -25,7 +25,7 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kCols = 2;          // key blocks a thread scores at once
-constexpr int kChunk = 8;         // d-elements of each kbar_B held in registers at a time
+constexpr int kChunk = 16;        // d-elements of each kbar_B held in registers at a time
 constexpr bool kPrefetch = true;  // load the next chunk while the current one is in use
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -176,7 +176,23 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(const float* __restr
     uint32_t prefix = 0, pmask = 0;
     int need = kr;                     // still to take among keys matching `prefix`
     if (kr < nkb) {
-      for (int shift = 24; shift >= 0; shift -= 8) {
+      // digits shared by every key of the row (a row's scores share their top bits) are known
+      // without a histogram: start at the first digit where the smallest and largest key differ
+      uint32_t kmin = 0xffffffffu, kmax = 0u;
+      for (int B = lane; B < nkb; B += 32) {
+        const uint32_t u = krow[B];
+        kmin = min(kmin, u);
+        kmax = max(kmax, u);
+      }
+      kmin = __reduce_min_sync(0xffffffffu, kmin);
+      kmax = __reduce_max_sync(0xffffffffu, kmax);
+      int shift0 = 24;
+      while (shift0 > 0 && ((kmin ^ kmax) >> shift0) == 0u) {
+        prefix |= kmin & (255u << shift0);
+        pmask |= 255u << shift0;
+        shift0 -= 8;
+      }
+      for (int shift = shift0; shift >= 0; shift -= 8) {
         for (int i = lane; i < 256; i += 32) wh[i] = 0;
         __syncwarp();
         for (int B = lane; B < nkb; B += 32) {
@@ -215,17 +231,20 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(const float* __restr
         need -= static_cast<int>(gt);
         prefix |= static_cast<uint32_t>(dd) << shift;
         pmask |= 255u << shift;
+        const bool all_taken = static_cast<uint32_t>(need) == wh[dd];
         __syncwarp();
+        // every key left under the prefix is taken: the remaining digits cannot change the set
+        if (all_taken) break;
       }
     } else {
       prefix = 0;                      // k == nkb: every key is taken
       need = nkb;
     }
-    const uint32_t T = prefix;
+    const uint32_t T = prefix;         // compared on the resolved digits only
     int taken = 0, eq_seen = 0;
     for (int B0 = 0; B0 < nkb; B0 += 32) {
       const int B = B0 + lane;
-      const uint32_t u = (B < nkb) ? krow[B] : 0u;
+      const uint32_t u = ((B < nkb) ? krow[B] : 0u) & pmask;
       const bool valid = B < nkb;
       const bool gt = valid && (kr == nkb || u > T);
       const bool eq = valid && kr < nkb && u == T;
