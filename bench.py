@@ -498,9 +498,9 @@ def run_reference(args, world, rank):
 REBLOCK_METRIC = "ms/call of the Spark-Reblock partitioner (q_reuse_k), 768p shape"
 
 
-def reblock_level_min_nodes(N, block):
-    """Smallest node (in tokens) of every level of the partitioner's block tree: an m-block
-    node gives ceil(m/2) blocks to its left child; the last block takes the remainder."""
+def reblock_level_node_sizes(N, block):
+    """(smallest, largest) node (in tokens) of every level of the partitioner's block tree: an
+    m-block node gives ceil(m/2) blocks to its left child; the last block takes the remainder."""
     nb = -(-N // block)
     off = lambda b: N if b >= nb else b * block
     out, frontier = [], [(0, nb)]
@@ -512,9 +512,28 @@ def reblock_level_min_nodes(N, block):
                 sizes.append(off(hi) - off(lo))
                 nxt += [(lo, mid), (mid, hi)]
         if sizes:
-            out.append(min(sizes))
+            out.append((min(sizes), max(sizes)))
         frontier = nxt
     return out
+
+
+def reblock_level_min_nodes(N, block):
+    """Smallest node (in tokens) of every level of the partitioner's block tree."""
+    return [lo for lo, _ in reblock_level_node_sizes(N, block)]
+
+
+def reblock_launches_per_call(N, d, block, moment_min_node=256, moment_chunk=16384):
+    """Kernel launches of one partitioner call: 4 whitening kernels, the identity order and the
+    offsets, and per level 11 selection/scatter kernels plus the moment kernels - one when every
+    node is a single moment chunk (it runs the power iterations itself), else two - or, below
+    moment_min_node tokens or at d = 64, 8 power-pass kernels."""
+    n = 6
+    for lo, hi in reblock_level_node_sizes(N, block):
+        if d == 128 and lo >= moment_min_node:
+            n += 11 + (1 if hi <= moment_chunk else 2)
+        else:
+            n += 11 + 8
+    return n
 
 
 def reblock_bytes_flops(H, N, d, block, e_in, power_iters=4, moment_min_node=256):
@@ -591,8 +610,7 @@ def measure_reblock(Q, K, block, steps, warmup, world, device, sample_clocks=Tru
     return {"ms": ms, "prep_ms": prep_ms, "levels_ms": part_ms, "flops": flops,
             "prep_bytes": prep_bytes, "level_bytes": level_bytes, "levels": lay.levels,
             "clocks": clock_info,
-            "launches_per_call": 6 + sum(11 + (2 if (d == 128 and m >= 256) else 8)
-                                         for m in reblock_level_min_nodes(N, block))}
+            "launches_per_call": reblock_launches_per_call(N, d, block)}
 
 
 def run_reblock(args, world, rank, local):
@@ -630,8 +648,6 @@ def run_reblock(args, world, rank, local):
                         "units": ("tcgen05 bf16 MMAs, fp32 accumulation" if
                                   Q.dtype == torch.bfloat16 and d == 128 else "fp32 CUDA cores")},
                     "levels": {"ms": part_ms, "GB/s": gbs, "bytes": level_bytes}},
-        # per call: 4 whitening kernels, the identity order, offsets, and per level 11
-        # selection/scatter kernels plus 8 power-pass kernels or 2 node-moment kernels
         "gpu_launches": r["launches_per_call"] * args.steps,
         "clocks": r["clocks"],
     }
