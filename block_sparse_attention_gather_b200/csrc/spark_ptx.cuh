@@ -97,14 +97,25 @@ __device__ __forceinline__ bool launch_timed_out(const uint32_t* err) {
 // under 0.2 ms poll without suspending (a suspended test may sleep until the phase completes).
 // A limit of 0 makes every wait expire at once, without testing the barrier: the expiry path
 // then runs deterministically (a test of it).
+// The slow path is a separate function, so the hot loops that wait inline only one test.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
+                                            volatile int* abort_flag, uint32_t* err,
+                                            uint64_t limit_ns);
+
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* err, uint64_t limit_ns = kWaitLimitNs) {
+  if (limit_ns != 0 && mbar_test(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, err, limit_ns);
+}
+
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
+                                            volatile int* abort_flag, uint32_t* err,
+                                            uint64_t limit_ns) {
   if (limit_ns == 0) {
     flag_error(err, kErrTimeout);
     *abort_flag = 1;
     return false;
   }
-  if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   const bool sleep = limit_ns >= 200000ull;
   for (;;) {
