@@ -361,16 +361,27 @@ def file_hash(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+# The attention kernel's compiled code depends on these sources.
+ATTENTION_SOURCES = ("attention.cu", "spark_ptx.cuh", "spark_kernels.cuh", "route_step.cuh")
+
+
+def attention_sources_hash():
+    h = hashlib.sha256()
+    for name in ATTENTION_SOURCES:
+        with open(os.path.join(ROOT, "block_sparse_attention_gather_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def profiled_traffic(hp):
     """DRAM bytes per attention launch from the committed ncu summary, if it was taken on the
-    current kernel source (else None)."""
+    current kernel sources (else None)."""
     try:
         with open(PROFILE_SUMMARY) as f:
             prof = json.load(f)
     except (OSError, ValueError):
         return None
-    src = os.path.join(ROOT, "block_sparse_attention_gather_b200", "csrc", "attention.cu")
-    if prof.get("attention_cu_sha256_16") != file_hash(src):
+    if prof.get("attention_sources_sha256_16") != attention_sources_hash():
         return None
     per_unit = prof.get("dram_bytes_per_query_block")
     if per_unit is None:

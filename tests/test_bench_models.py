@@ -45,15 +45,20 @@ def test_kernel_byte_models():
 
 def test_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     hp = fake_hotpath([64] * 4, [64] * 4, [[[0], [1], [2], [3]]], H=2)
-    src = bench.os.path.join(bench.ROOT, "block_sparse_attention_gather_b200", "csrc",
-                             "attention.cu")
     prof = tmp_path / "dram.json"
-    prof.write_text(json.dumps({"attention_cu_sha256_16": bench.file_hash(src),
+    prof.write_text(json.dumps({"attention_sources_sha256_16": bench.attention_sources_hash(),
                                 "dram_bytes_per_query_block": 1000.0}))
     monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(prof))
     assert bench.profiled_traffic(hp) == 1000.0 * 2 * 4
-    prof.write_text(json.dumps({"attention_cu_sha256_16": "0" * 16,
+    prof.write_text(json.dumps({"attention_sources_sha256_16": "0" * 16,
                                 "dram_bytes_per_query_block": 1000.0}))
+    assert bench.profiled_traffic(hp) is None
+    # a change to any source the kernel is compiled from invalidates the capture
+    monkeypatch.setattr(bench, "ATTENTION_SOURCES", bench.ATTENTION_SOURCES[:1])
+    prof.write_text(json.dumps({"attention_sources_sha256_16": bench.attention_sources_hash(),
+                                "dram_bytes_per_query_block": 1000.0}))
+    monkeypatch.undo()
+    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(prof))
     assert bench.profiled_traffic(hp) is None
 
 
