@@ -53,7 +53,10 @@
 // Every wait is bounded by the launch parameter wait_ns (the library's process-wide setting,
 // 4 s by default); on expiry the kernel flags kErrTimeout, stops every role, drains the copies
 // and MMAs it issued (waits bounded by the default limit), frees TMEM and returns.
+#include <type_traits>
+
 #include "route_step.cuh"
+
 #include "spark_kernels.cuh"
 
 namespace spark {
@@ -152,22 +155,33 @@ __device__ __forceinline__ int tile_cols(const TileInfo& ti) {
 // raw scores (the scale is applied in the exponent) with columns past the block set to -inf;
 // summary tiles give s*sl + offset (offset -inf for selected blocks and padding), sl being the
 // logit scale in log2 units (times the FP8 scales).
-template <bool kBiasSmem>
-__device__ __forceinline__ void load_logits(uint32_t taddr, int col0, const TileInfo& ti,
-                                            float sl, const float* biasrow,
-                                            const float* cb, const uint32_t* selmask, int nkb,
-                                            float (&x)[64]) {
+// Exact tiles: raw scores (the scale is applied in the exponent), columns past the block's
+// rows set to -inf.
+__device__ __forceinline__ void load_logits_exact(uint32_t taddr, int col0, const TileInfo& ti,
+                                                  float (&x)[64]) {
   uint32_t r[64];
   tmem_ld64(taddr, r);
 #pragma unroll
   for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(r[j]);
-  if (ti.exact) {
-    if (ti.nvalid < col0 + 64) {
+  if (ti.nvalid < col0 + 64) {
 #pragma unroll
-      for (int j = 0; j < 64; ++j)
-        if (col0 + j >= ti.nvalid) x[j] = -INFINITY;
-    }
-  } else if (kBiasSmem) {
+    for (int j = 0; j < 64; ++j)
+      if (col0 + j >= ti.nvalid) x[j] = -INFINITY;
+  }
+}
+
+// Summary tiles: s*sl + offset (offset -inf for selected blocks and padding), sl being the logit
+// scale in log2 units (times the FP8 scales).
+template <bool kBiasSmem>
+__device__ __forceinline__ void load_logits_summary(uint32_t taddr, int col0, const TileInfo& ti,
+                                                    float sl, const float* biasrow,
+                                                    const float* cb, const uint32_t* selmask,
+                                                    int nkb, float (&x)[64]) {
+  uint32_t r[64];
+  tmem_ld64(taddr, r);
+#pragma unroll
+  for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(r[j]);
+  if (kBiasSmem) {
     const float4* br = reinterpret_cast<const float4*>(biasrow + ti.y + col0);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -188,6 +202,19 @@ __device__ __forceinline__ void load_logits(uint32_t taddr, int col0, const Tile
       x[j] = live ? fmaf(x[j], sl, c * kLog2e) : -INFINITY;
     }
   }
+}
+
+// Reads 64 columns of this thread's S row (TMEM) and turns them into logits, for a tile of
+// either kind (the reference of the first tiles).
+template <bool kBiasSmem>
+__device__ __forceinline__ void load_logits(uint32_t taddr, int col0, const TileInfo& ti,
+                                            float sl, const float* biasrow,
+                                            const float* cb, const uint32_t* selmask, int nkb,
+                                            float (&x)[64]) {
+  if (ti.exact)
+    load_logits_exact(taddr, col0, ti, x);
+  else
+    load_logits_summary<kBiasSmem>(taddr, col0, ti, sl, biasrow, cb, selmask, nkb, x);
 }
 
 // The 32 columns col0 .. col0+31 of an exact tile into x[0..31] (columns past the valid rows
@@ -610,26 +637,33 @@ __global__ void __launch_bounds__(kPersist ? kThreadsFused : kThreads, 1) attend
       if (!(m_ref > -INFINITY)) m_ref = 0.f;
       if (pass == 0) m_ref0 = m_ref;
       TileInfo next = tile_info<kFp8>(grp, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
-      for (int t = grp; ok && t < T; t += 2) {
+      // One tile of this group; the exact tiles (selected blocks, then context rows) come
+      // before the summary tiles, so each kind runs in a loop of its own that carries only its
+      // own logit path.
+      // kind: 1 exact, 2 summary, 0 either (decided per tile)
+      auto tile = [&](int t, auto kind) -> bool {
+        constexpr int kKind = decltype(kind)::value;
         const TileInfo ti = next;
         const int tg = tg0 + t;
         const int b = tg % 3;
         if (pass > 0 || t >= 2) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&bars->sfull[b], (tg / 3) & 1, abort_flag, err, wait_ns));
-          if (!ok) break;
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait(&bars->sfull[b], (tg / 3) & 1, abort_flag, err, wait_ns)))
+            return false;
           tc_fence_after_sync();
         }
         if (t + 2 < T)
           next = tile_info<kFp8>(t + 2, k, nxt, nc, sel_row, k_offsets, nkb, N, sc, h);
         const uint32_t sbuf = tbase + lane_off + b * 128;
         const float tsl = scale_log2 * ti.ks;
-        const float c = ti.exact ? tsl : 1.f;
+        const bool exact = kKind == 1 || (kKind == 0 && ti.exact);
+        const float c = exact ? tsl : 1.f;
         // The row maximum is only needed for a repeat, and only to within a few units: a
         // chunk whose sum stays in [2^-40, 2^40] has its maximum within 40 of the reference
         // and cannot drive the row sum out of [2^-60, 2^60] (fewer than 2^16 chunks per row),
         // so only chunks outside that range (rare) take their maximum.
         // only the columns the MMAs covered (exact tiles: the valid rows rounded up to 16)
-        const int ncols = kVarTiles ? tile_cols(ti) : 128;
+        const int ncols = (kVarTiles && kKind != 2) ? tile_cols(ti) : 128;
         float rowsum = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -642,15 +676,21 @@ __global__ void __launch_bounds__(kPersist ? kThreadsFused : kThreads, 1) attend
             tmem_st16_issue(sbuf + 32, p16);
             if (!(cs >= 0x1p-40f && cs <= 0x1p40f)) m_true = fmaxf(m_true, max32(x) * tsl);
           } else {
-            load_logits<kBiasSmem>(sbuf + half * 64, half * 64, ti, tsl, biasrow, cb,
-                                   selmask, nkb, x);
+            if constexpr (kKind == 1)
+              load_logits_exact(sbuf + half * 64, half * 64, ti, x);
+            else if constexpr (kKind == 2)
+              load_logits_summary<kBiasSmem>(sbuf + half * 64, half * 64, ti, tsl, biasrow, cb,
+                                             selmask, nkb, x);
+            else
+              load_logits<kBiasSmem>(sbuf + half * 64, half * 64, ti, tsl, biasrow, cb, selmask,
+                                     nkb, x);
             cs = exp32_at(x, 0, c, m_ref, p16);
             tmem_st16_issue(sbuf + half * 32, p16);
             cs += exp32_at(x, 32, c, m_ref, p16);
             tmem_st16_issue(sbuf + half * 32 + 16, p16);
             if (!(cs >= 0x1p-40f && cs <= 0x1p40f)) {
               const float mt = max64(x);
-              m_true = fmaxf(m_true, ti.exact ? mt * tsl : mt);
+              m_true = fmaxf(m_true, exact ? mt * tsl : mt);
             }
           }
           rowsum += cs;
@@ -659,6 +699,16 @@ __global__ void __launch_bounds__(kPersist ? kThreadsFused : kThreads, 1) attend
         tmem_wait_st();                                 // P complete before it is signalled
         tc_fence_before_sync();
         mbar_arrive(&bars->pready[b]);
+        return true;
+      };
+      int t = grp;
+      if constexpr (kFp8 || kPersist) {
+        // one loop (split, these instantiations spill more registers)
+        for (; ok && t < T; t += 2) ok = tile(t, std::integral_constant<int, 0>{});
+      } else {
+        const int t_exact = k + nxt;                     // tiles before the summary tiles
+        for (; ok && t < T && t < t_exact; t += 2) ok = tile(t, std::integral_constant<int, 1>{});
+        for (; ok && t < T; t += 2) ok = tile(t, std::integral_constant<int, 2>{});
       }
       // ---- epilogue: O / (l_0 + l_1), scattered to the original token order
       bool fine = ok && T > 0;
