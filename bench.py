@@ -672,15 +672,15 @@ def run_reblock(args, world, rank, local):
 
 def main():
     args = parse_args()
+    if args.impl == "reference":
+        # the CPU oracle needs no process group and no GPU: rank 0 times it, the other ranks of
+        # a multi-rank launch exit at once
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")),
+                      int(os.environ.get("RANK", "0")))
+        return
     world, rank, local = init_dist()
     if args.op == "reblock" and args.impl == "ours":
         run_reblock(args, world, rank, local)
-        return
-    if args.impl == "reference":
-        run_reference(args, world, rank)
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
         return
     if args.warmup < 3:
         raise SystemExit("at least 3 warm-up steps are required")
